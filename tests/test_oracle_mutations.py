@@ -1,0 +1,56 @@
+"""The oracle's pins must catch plausible mistakes (CPU only).
+
+Each case plants one mistake in a copy of the oracle's C source (a dropped term,
+a wrong index, a transposed operand, a wrong rounding rule), builds it, and runs
+the oracle pin suites against that build in a child process.  The child must
+fail; a mutant that passes every pin would mean the pins do not pin.
+"""
+
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "pa_oracle.c")
+
+MUTANTS = {
+    "offset_from_quotient": ("int64_t off = l % block_size;", "int64_t off = (l / block_size) % block_size;"),
+    "block_from_position": ("int64_t phys = table[l / block_size];", "int64_t phys = table[0];"),
+    "scale_dropped": ("    s *= scale;\n", "\n"),
+    "no_max_shift": ("double p = exp(scratch[j - lo] - m);", "double p = exp(scratch[j - lo]);"),
+    "gqa_interleaved": ("int h = kvh * group + g;\n        int64_t qrow", "int h = g * num_kv_heads + kvh;\n        int64_t qrow"),
+    "kv_swapped": ("acc += scratch[j - lo] * V[", "acc += scratch[j - lo] * K["),
+    "slot_offset_swapped": ("int64_t b = s / block_size, o = s % block_size;", "int64_t o = s / block_size, b = s % block_size;"),
+    "fp8_scale_multiplied": ("float yk = xk / k_scale;", "float yk = xk * k_scale;"),
+    "e4m3_ties_odd": ("c = (lo & 1) ? hi : lo;", "c = (lo & 1) ? lo : hi;"),
+    "e4m3_bias_off": ("v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 11);"),
+    "merge_unweighted": ("double w = lp * exp(m[r * max_parts + p] - M);", "double w = exp(m[r * max_parts + p] - M);"),
+    "f16_subnormal": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
+    "dequant_scale_dropped": ("        k *= k_scale;\n", "\n"),
+    "copy_wrong_direction": ("memcpy((char*)key_caches[l] + dst * block_bytes, (char*)key_caches[l] + src * block_bytes,",
+                             "memcpy((char*)key_caches[l] + src * block_bytes, (char*)key_caches[l] + dst * block_bytes,"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    with tempfile.TemporaryDirectory() as tmp:
+        csrc = os.path.join(tmp, "mutant.c")
+        lib = os.path.join(tmp, "libmutant.so")
+        with open(csrc, "w") as f:
+            f.write(src.replace(old, new))
+        subprocess.run(["gcc", "-std=c11", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", lib,
+                        csrc, "-lm"], check=True)
+        env = dict(os.environ, PA_ORACLE_LIB_OVERRIDE=lib)
+        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                            os.path.join(ROOT, "tests", "test_oracle_formats.py"),
+                            os.path.join(ROOT, "tests", "test_oracle_cache_ops.py"),
+                            os.path.join(ROOT, "tests", "test_oracle_decode.py")],
+                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
