@@ -1,0 +1,454 @@
+"""Benchmark of the paged decode hot path on B200: one JSON line on rank 0.
+
+A step is one pass of the whole path over one batch of the workload: the cache
+write of every sequence's new token(s) (reshape_and_cache), the copy-on-write
+block copies where the workload has them (copy_blocks), and the paged decode
+attention (decode kernel, plus the log-sum-exp reduce for sequences longer than
+one partition).  Inputs are resident in HBM when the timed region starts.
+
+Metric: achieved HBM GB/s of algorithmic bytes (K/V read + Q read + output write
++ block tables + sequence lengths for the decode; read + written bytes for the
+cache writes and copies), whole job, plus decode tokens/s and context tokens/s
+per layer.  The working set (over 1 GB for the default workload) is far larger
+than the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Multi-GPU: the path shards with no exchange, so N ranks run N independent
+replicas (weak scaling); timing is the max over ranks of CUDA-event time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_413_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged-attn decode: achieved HBM GB/s (% of B200 peak), seq-tokens/s per layer"
+DEFAULT_CONFIG = "llama2_7b"
+FALLBACK_HBM_GBS = 6650.0
+TORCH_DT = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+DESCR = {
+    "tiny": "4 seqs L={1,17,33,100}, 4 heads MHA, d64, fp16, pool 64 blocks",
+    "llama2_7b": "Llama-2-7B layer: 64 seqs, 32 heads MHA, d128, L~U[128,2048], fp16 KV, "
+                 "block 16, shuffled pool 1.1x",
+    "llama2_70b_gqa": "Llama-2-70B layer: 256 seqs, 64 q heads / 8 kv heads, d128, "
+                      "L~U[512,768], bf16 KV, block 16, shuffled pool 1.1x",
+    "long_splitk": "8 seqs x 32768 tokens, 32 q / 8 kv heads, d128, bf16 KV, 512-token "
+                   "partitions + LSE reduce",
+    "beam_cow_fp8": "64 prompts x 4 beams, 1032 shared tokens + 4 own, 32 q / 8 kv heads, "
+                    "d128, FP8 E4M3 KV, copy-on-write copies per step",
+}
+
+
+# ---------------------------------------------------------------- bytes model
+def decode_bytes(wl: W.Workload, out_dtype: str) -> int:
+    cfg = wl.cfg
+    L = wl.seq_lens.numpy().astype(np.int64)
+    kv = int(L.sum()) * cfg.num_kv_heads * cfg.head_dim * 2 * W.ELT_BYTES[cfg.cache_dtype]
+    qo = len(L) * cfg.num_heads * cfg.head_dim * (W.ELT_BYTES[cfg.q_dtype] +
+                                                   W.ELT_BYTES[out_dtype])
+    tables = int(np.ceil(L / cfg.block_size).sum()) * 4 + 4 * len(L)
+    return kv + qo + tables
+
+
+def unique_kv_bytes(wl: W.Workload) -> int:
+    """K/V bytes of distinct physical blocks the decode reads (shared prefixes once)."""
+    cfg = wl.cfg
+    bt = wl.block_tables.numpy()
+    L = wl.seq_lens.numpy()
+    slots = set()
+    for i, n in enumerate(L):
+        for pos_blk in range(int(math.ceil(n / cfg.block_size))):
+            b = int(bt[i, pos_blk])
+            used = min(cfg.block_size, int(n) - pos_blk * cfg.block_size)
+            slots.add((b, used))
+    per_tok = cfg.num_kv_heads * cfg.head_dim * 2 * W.ELT_BYTES[cfg.cache_dtype]
+    best = {}
+    for b, used in slots:
+        best[b] = max(best.get(b, 0), used)
+    return sum(best.values()) * per_tok
+
+
+def cache_write_bytes(wl: W.Workload) -> int:
+    cfg = wl.cfg
+    t = wl.slot_mapping.numel()
+    per = cfg.num_kv_heads * cfg.head_dim * 2
+    return t * per * (W.ELT_BYTES[wl.src_dtype] + W.ELT_BYTES[cfg.cache_dtype]) + 8 * t
+
+
+def copy_bytes(wl: W.Workload) -> int:
+    if wl.block_mapping is None or wl.block_mapping.numel() == 0:
+        return 0
+    cfg = wl.cfg
+    block = cfg.block_size * cfg.num_kv_heads * cfg.head_dim * W.ELT_BYTES[cfg.cache_dtype]
+    return wl.block_mapping.shape[0] * (2 * 2 * block + 16)
+
+
+# ---------------------------------------------------------------- helpers
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(config: str):
+    """DRAM bytes per decode launch from the committed ncu summary of this workload,
+    valid only while the decode source is the one that was profiled."""
+    path = os.path.join(ROOT, "profiles", f"paged_attention_decode_{config}.md")
+    src = os.path.join(ROOT, "paged_kv_cache_413_b200", "csrc", "pa_decode.cu")
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        m = re.search(r"decode_source_sha256_16:\s*([0-9a-f]{16})", text)
+        t = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+        if m and t and m.group(1) == sha:
+            return int(t.group(1))
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(wl: W.Workload, seqs, out_dtype: str):
+    """Run the oracle (cache write of the sampled sequences' tokens + decode of them).
+    Returns (seconds, algorithmic bytes of the sample)."""
+    import oracle
+
+    cfg = wl.cfg
+    seqs = np.asarray(seqs)
+    T = cfg.new_tokens_per_seq
+    new = np.concatenate([np.arange(s * T, (s + 1) * T) for s in seqs])
+    nt = torch.as_tensor(new)
+    t0 = time.perf_counter()
+    kc, vc = oracle.reshape_and_cache(wl.new_key[nt], wl.new_value[nt], wl.key_cache,
+                                      wl.value_cache, wl.slot_mapping.numpy()[new],
+                                      src_dtype=wl.src_dtype, cache_dtype=cfg.cache_dtype,
+                                      k_scale=wl.k_scale, v_scale=wl.v_scale, inplace=True)
+    idx = torch.as_tensor(seqs)
+    oracle.paged_attention_decode(wl.query[idx], kc, vc, wl.block_tables.numpy()[seqs],
+                                  wl.seq_lens.numpy()[seqs], scale=wl.scale,
+                                  q_dtype=cfg.q_dtype, cache_dtype=cfg.cache_dtype,
+                                  k_scale=wl.k_scale, v_scale=wl.v_scale)
+    dt = time.perf_counter() - t0
+    L = wl.seq_lens.numpy()[seqs].astype(np.int64)
+    b = int(L.sum()) * cfg.num_kv_heads * cfg.head_dim * 2 * W.ELT_BYTES[cfg.cache_dtype]
+    b += len(seqs) * cfg.num_heads * cfg.head_dim * (W.ELT_BYTES[cfg.q_dtype] +
+                                                      W.ELT_BYTES[out_dtype])
+    b += int(np.ceil(L / cfg.block_size).sum()) * 4 + 4 * len(seqs)
+    b += len(new) * cfg.num_kv_heads * cfg.head_dim * 2 * (W.ELT_BYTES[wl.src_dtype] +
+                                                          W.ELT_BYTES[cfg.cache_dtype])
+    return dt, b
+
+
+def cpu_baseline(wl: W.Workload, out_dtype: str, budget_s: float = 12.0):
+    """The oracle timed on a bounded sample of the workload's sequences."""
+    import oracle
+
+    n = wl.seq_lens.numel()
+    order = np.random.default_rng(0).permutation(n)
+    dt1, _ = oracle_sample(wl, order[:1], out_dtype)              # calibration
+    k = int(max(1, min(n, budget_s / max(dt1, 1e-4))))
+    dt, b = oracle_sample(wl, order[:k], out_dtype)
+    return {"value": b / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{k} of {n} sequences of the workload (cache write of their new "
+                      f"tokens + fp64 decode), {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args, rank, world, local_rank):
+    import paged_kv_cache_413_b200 as pa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = W.CONFIGS[args.config]
+    wl = W.make_workload(cfg, seed=cfg.seed + 1000 * rank) if rank else W.make_workload(cfg)
+    out_dtype = cfg.out_dtype
+    f = lambda t: None if t is None else t.to(dev)
+    kc, vc = f(wl.key_cache), f(wl.value_cache)
+    q, bt, sl = f(wl.query), f(wl.block_tables), f(wl.seq_lens)
+    nk, nv, sm = f(wl.new_key), f(wl.new_value), f(wl.slot_mapping)
+    bm = f(wl.block_mapping) if wl.block_mapping is not None and wl.block_mapping.numel() else None
+    max_len = int(wl.seq_lens.max())
+    part = args.partition if args.partition is not None else cfg.partition_size
+    ws_n = pa.pa_paged_attention_workspace_size(q.shape[0], cfg.num_heads, cfg.head_dim, max_len,
+                                                part)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+    out = torch.empty(q.shape, dtype=TORCH_DT[out_dtype], device=dev)
+    stream = torch.cuda.current_stream(dev)
+    if wl.prefix_key is not None:  # copy-on-write workload: fill the shared prefix once
+        pa.pa_reshape_and_cache(f(wl.prefix_key), f(wl.prefix_value), kc, vc,
+                                f(wl.prefix_slot_mapping), k_scale=wl.k_scale,
+                                v_scale=wl.v_scale)
+    part_eff = part if part > 0 else 512
+    reduce_runs = max_len > part_eff
+    launches = 1 + 1 + (1 if reduce_runs else 0) + (1 if bm is not None else 0)
+
+    ev = []
+
+    def step(timed: bool):
+        if bm is not None:
+            pa.pa_copy_blocks([kc], [vc], bm)
+        pa.pa_reshape_and_cache(nk, nv, kc, vc, sm, k_scale=wl.k_scale, v_scale=wl.v_scale)
+        if timed:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        pa.pa_paged_attention_decode(out, q, kc, vc, bt, sl, max_seq_len=max_len, scale=wl.scale,
+                                     k_scale=wl.k_scale, v_scale=wl.v_scale,
+                                     partition_size=part, workspace=ws)
+        if timed:
+            e1.record(stream)
+            ev.append((e0, e1))
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize(dev)
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error bits set during warm-up")
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.__enter__()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    if sampler:
+        sampler.__exit__(None, None, None)
+    elapsed_ms = t0.elapsed_time(t1)
+    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        t = torch.tensor([elapsed_ms, decode_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms, decode_ms = t.tolist()
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error bits set during the timed steps")
+
+    step_bytes = decode_bytes(wl, out_dtype) + cache_write_bytes(wl) + copy_bytes(wl)
+    ms_per_step = elapsed_ms / args.steps
+    value = step_bytes * world * args.steps / (elapsed_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda t: None if t is None else t.pin_memory()
+    h_q, h_nk, h_nv, h_sm = pin(wl.query), pin(wl.new_key), pin(wl.new_value), pin(wl.slot_mapping)
+    h_bt, h_sl = pin(wl.block_tables), pin(wl.seq_lens)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_nk, h_nv, h_sm, h_bt, h_sl))
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = max(10, args.steps // 4)
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        nk.copy_(h_nk, non_blocking=True)
+        nv.copy_(h_nv, non_blocking=True)
+        sm.copy_(h_sm, non_blocking=True)
+        bt.copy_(h_bt, non_blocking=True)
+        sl.copy_(h_sl, non_blocking=True)
+        step(False)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = a0.elapsed_time(a1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e_value = step_bytes * world * e2e_steps / (e2e_ms * 1e-3) / 1e9
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    dec_b = decode_bytes(wl, out_dtype)
+    achieved = dec_b / (decode_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(args.config)
+    L = wl.seq_lens.numpy().astype(np.int64)
+    n_seqs = len(L)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "kv_dtype": cfg.cache_dtype, "data": "synthetic",
+        "config": {"workload": f"{args.config}: {DESCR[args.config]}",
+                   "partition_tokens": part_eff, "out_dtype": out_dtype,
+                   "l2": "no flush: inputs larger than L2 (%.2f GB read per step vs 126 MB L2)"
+                         % (dec_b / 1e9),
+                   "parallelism": f"replicas x{world}"},
+        "pct_of_peak": round(100.0 * value / peak, 2),
+        "decode_tokens_per_s_per_layer": round(n_seqs * world / (ms_per_step * 1e-3), 1),
+        "context_tokens_per_s_per_layer": round(int(L.sum()) * world / (ms_per_step * 1e-3), 1),
+        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (+ LSE reduce)",
+                     "achieved": round(achieved, 2), "peak": peak,
+                     "peak_kind": f"{peak_kind} (hbm_gbs, copy burst)", "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes_per_launch": dec_b,
+                     "launch_ms": round(decode_ms, 5)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": round(e2e_ms / e2e_steps, 5)},
+        "gpu_launches": launches * args.steps,
+        "clocks": sampler.summary() if sampler else None,
+    }
+    if wl.prefix_key is not None:
+        line["unique_kv_bytes_per_step"] = unique_kv_bytes(wl)
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, out_dtype)
+    return line
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step a bounded sample (one sequence)."""
+    if rank != 0:
+        return None
+    import oracle
+
+    cfg = W.CONFIGS[args.config]
+    wl = W.make_workload(cfg)
+    n = wl.seq_lens.numel()
+    order = np.random.default_rng(0).permutation(n)
+    for i in range(args.warmup):
+        oracle_sample(wl, order[i % n:i % n + 1], cfg.out_dtype)
+    total_t, total_b = 0.0, 0
+    for i in range(args.steps):
+        dt, b = oracle_sample(wl, order[i % n:i % n + 1], cfg.out_dtype)
+        total_t += dt
+        total_b += b
+    v = total_b / total_t / 1e9
+    return {"metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total_t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"{args.config}: {DESCR[args.config]}",
+                       "sample_per_step": "one sequence (its cache write + fp64 decode)"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"one of {n} sequences per step, {args.steps} steps"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group(
+                "nccl", timeout=datetime.timedelta(seconds=120),
+                device_id=torch.device("cuda", local_rank))
+        try:
+            line = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -156,16 +156,22 @@ def e4m3_encode(x) -> np.ndarray:
 
 
 def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, *, src_dtype: str,
-                      cache_dtype: str, k_scale: float = 1.0, v_scale: float = 1.0):
-    """Return new (key_cache, value_cache) numpy storage arrays with the tokens written.
+                      cache_dtype: str, k_scale: float = 1.0, v_scale: float = 1.0,
+                      inplace: bool = False):
+    """Return (key_cache, value_cache) numpy storage arrays with the tokens written.
 
     key, value: [T, H_kv, D] of ``src_dtype``; caches: [NB, H_kv, BS, D] of
-    ``cache_dtype``; slot_mapping: [T] int64 (negative = skip).
+    ``cache_dtype``; slot_mapping: [T] int64 (negative = skip).  The caches are
+    copied first unless ``inplace`` (then contiguous host caches are written).
     """
     k = _raw(key, src_dtype)
     v = _raw(value, src_dtype)
-    kc = _raw(key_cache, cache_dtype).copy()
-    vc = _raw(value_cache, cache_dtype).copy()
+    kc = _raw(key_cache, cache_dtype)
+    vc = _raw(value_cache, cache_dtype)
+    if not inplace:
+        kc, vc = kc.copy(), vc.copy()
+    elif not (kc.flags.writeable and vc.flags.writeable):
+        raise ValueError("in-place cache write needs writeable host caches")
     sm = np.ascontiguousarray(np.asarray(slot_mapping, dtype=np.int64))
     nb, hkv, bs, d = kc.shape
     t = sm.shape[0]

@@ -1,0 +1,154 @@
+// pa_cache.cu -- cache-write and block-copy kernels (sm_100a).
+//
+// reshape_and_cache: the step of the memory flow that stores a new token's K and
+// V rows into the slot the block manager registered for it ("vLLM 推理优化技术深度
+// 调研报告" sec 2, memory flow; "vLLM 是什么…" sec 2, a new block only when the
+// current one is full).  Optional fused FP8 E4M3 quantisation with a per-tensor
+// scale ("vLLM推理引擎PagedAttention原理与性能优化实战" sec 5.2).
+//
+// copy_blocks: the copy step of copy-on-write ("vLLM推理引擎PagedAttention原理与
+// 性能优化实战" sec 3.2).
+//
+// Both are pure data movement bound by HBM; every access is a 16-byte vector
+// (8-byte for the E4M3 stores), consecutive threads touch consecutive addresses.
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+__device__ unsigned int g_cache_err;
+
+// Quantise 8 packed 16-bit values (one uint4) to 8 E4M3 bytes (one uint2):
+// IEEE fp32 division by the scale, then round-nearest-even with saturation.
+template <typename Tsrc>
+__device__ __forceinline__ uint2 quantise8(uint4 x, float scale) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  uint16_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = unpack2(w[i], Tsrc{});
+    q[i] = pack2_e4m3(__fdiv_rn(f.x, scale), __fdiv_rn(f.y, scale));
+  }
+  return make_uint2(uint32_t(q[0]) | (uint32_t(q[1]) << 16),
+                    uint32_t(q[2]) | (uint32_t(q[3]) << 16));
+}
+
+// One CTA per token; each thread moves 8 elements of K and 8 of V per step.
+template <typename Tsrc, bool kQuant>
+__global__ void __launch_bounds__(128) reshape_and_cache_kernel(
+    const uint16_t* __restrict__ key, const uint16_t* __restrict__ value,
+    uint8_t* __restrict__ key_cache, uint8_t* __restrict__ value_cache,
+    const int64_t* __restrict__ slot_mapping, int num_kv_heads, int head_dim,
+    int64_t num_slots, float k_scale, float v_scale) {
+  const int64_t t = blockIdx.x;
+  const int64_t slot = slot_mapping[t];
+  if (slot < 0) return;  // padding token
+  if (slot >= num_slots) {
+    if (threadIdx.x == 0) atomicOr(&g_cache_err, PA_DEVERR_SLOT_RANGE);
+    return;
+  }
+  const int64_t blk = slot / kBlockSize, off = slot % kBlockSize;
+  const int row = num_kv_heads * head_dim;  // elements of one token
+  const int chunks = row >> 3;
+  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+    const int e = c << 3;
+    const int h = e / head_dim, d = e - h * head_dim;
+    const int64_t src = t * row + e;
+    const int64_t dst = ((blk * num_kv_heads + h) * kBlockSize + off) * head_dim + d;
+    const uint4 kx = __ldg(reinterpret_cast<const uint4*>(key + src));
+    const uint4 vx = __ldg(reinterpret_cast<const uint4*>(value + src));
+    if constexpr (!kQuant) {
+      *reinterpret_cast<uint4*>(key_cache + dst * 2) = kx;
+      *reinterpret_cast<uint4*>(value_cache + dst * 2) = vx;
+    } else {
+      *reinterpret_cast<uint2*>(key_cache + dst) = quantise8<Tsrc>(kx, k_scale);
+      *reinterpret_cast<uint2*>(value_cache + dst) = quantise8<Tsrc>(vx, v_scale);
+    }
+  }
+}
+
+struct LayerPtrs {
+  uint8_t* k[kMaxLayersPerLaunch];
+  uint8_t* v[kMaxLayersPerLaunch];
+};
+
+// grid = (pairs, layers, 2): one CTA copies one block of one layer's K or V.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(LayerPtrs ptrs,
+                                                          const int64_t* __restrict__ mapping,
+                                                          int64_t block_bytes,
+                                                          int64_t num_blocks) {
+  const int64_t src = mapping[2 * blockIdx.x], dst = mapping[2 * blockIdx.x + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+      atomicOr(&g_cache_err, PA_DEVERR_COPY_RANGE);
+    return;
+  }
+  uint8_t* base = blockIdx.z ? ptrs.v[blockIdx.y] : ptrs.k[blockIdx.y];
+  const uint4* s = reinterpret_cast<const uint4*>(base + src * block_bytes);
+  uint4* d = reinterpret_cast<uint4*>(base + dst * block_bytes);
+  const int64_t n = block_bytes >> 4;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) d[i] = __ldg(s + i);
+}
+
+}  // namespace
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
+                                     void* value_cache, const int64_t* slot_mapping,
+                                     int num_tokens, int num_kv_heads, int head_dim,
+                                     int64_t num_blocks, pa_dtype src_dtype,
+                                     pa_dtype cache_dtype, float k_scale, float v_scale,
+                                     cudaStream_t stream) {
+  const dim3 grid(num_tokens), block(128);
+  const int64_t num_slots = num_blocks * kBlockSize;
+  auto k = static_cast<const uint16_t*>(key);
+  auto v = static_cast<const uint16_t*>(value);
+  auto kc = static_cast<uint8_t*>(key_cache);
+  auto vc = static_cast<uint8_t*>(value_cache);
+  if (cache_dtype != PA_FP8_E4M3) {
+    reshape_and_cache_kernel<__half, false><<<grid, block, 0, stream>>>(
+        k, v, kc, vc, slot_mapping, num_kv_heads, head_dim, num_slots, k_scale, v_scale);
+  } else if (src_dtype == PA_F16) {
+    reshape_and_cache_kernel<__half, true><<<grid, block, 0, stream>>>(
+        k, v, kc, vc, slot_mapping, num_kv_heads, head_dim, num_slots, k_scale, v_scale);
+  } else {
+    reshape_and_cache_kernel<__nv_bfloat16, true><<<grid, block, 0, stream>>>(
+        k, v, kc, vc, slot_mapping, num_kv_heads, head_dim, num_slots, k_scale, v_scale);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_copy_blocks(void* const* key_caches, void* const* value_caches,
+                               int num_layers, const int64_t* block_mapping, int num_pairs,
+                               size_t block_bytes, int64_t num_blocks, cudaStream_t stream) {
+  for (int l0 = 0; l0 < num_layers; l0 += kMaxLayersPerLaunch) {
+    const int nl = num_layers - l0 < kMaxLayersPerLaunch ? num_layers - l0 : kMaxLayersPerLaunch;
+    LayerPtrs p{};
+    for (int i = 0; i < nl; ++i) {
+      p.k[i] = static_cast<uint8_t*>(key_caches[l0 + i]);
+      p.v[i] = static_cast<uint8_t*>(value_caches[l0 + i]);
+    }
+    copy_blocks_kernel<<<dim3(num_pairs, nl, 2), 256, 0, stream>>>(
+        p, block_mapping, static_cast<int64_t>(block_bytes), num_blocks);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t read_and_clear_cache_errors(unsigned* bits, cudaStream_t stream) {
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_cache_err, sizeof v, 0,
+                                            cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_cache_err, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,
+                              stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  *bits |= v;
+  return e;
+}
+
+}  // namespace pa

@@ -1,0 +1,75 @@
+// pa_internal.h -- host-side launchers shared between the kernel files and the
+// C ABI layer (pa_api.cpp).  Arguments are already validated when these run.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+constexpr int kBlockSize = 16;            // tokens per physical block
+constexpr int kDefaultPartition = 512;     // tokens per split-K partition
+constexpr int kMaxLayersPerLaunch = 64;    // copy_blocks: layer pointers per launch
+
+struct WorkspaceLayout {
+  size_t m_off, l_off, o_off, total;       // byte offsets of the m, l, o sections
+  int max_parts;                           // partitions of the longest sequence
+};
+
+// Partition size in tokens for a requested value (0 = default).
+inline int resolve_partition(int requested) {
+  return requested > 0 ? requested : kDefaultPartition;
+}
+
+inline WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim,
+                                        int max_seq_len, int partition) {
+  WorkspaceLayout w{};
+  w.max_parts = max_seq_len > 0 ? (max_seq_len + partition - 1) / partition : 0;
+  if (w.max_parts <= 1) return w;  // no workspace needed
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t rows = size_t(num_seqs) * num_heads * w.max_parts;
+  w.m_off = 0;
+  w.l_off = up(rows * sizeof(float));
+  w.o_off = w.l_off + up(rows * sizeof(float));
+  w.total = w.o_off + up(rows * size_t(head_dim) * sizeof(float));
+  return w;
+}
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
+                                     void* value_cache, const int64_t* slot_mapping,
+                                     int num_tokens, int num_kv_heads, int head_dim,
+                                     int64_t num_blocks, pa_dtype src_dtype,
+                                     pa_dtype cache_dtype, float k_scale, float v_scale,
+                                     cudaStream_t stream);
+
+cudaError_t launch_copy_blocks(void* const* key_caches, void* const* value_caches,
+                               int num_layers, const int64_t* block_mapping, int num_pairs,
+                               size_t block_bytes, int64_t num_blocks, cudaStream_t stream);
+
+struct DecodeArgs {
+  void* out;
+  const void* query;
+  const void* key_cache;
+  const void* value_cache;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  int max_blocks_per_seq, num_seqs, max_seq_len, num_heads, num_kv_heads, head_dim;
+  int64_t num_blocks;
+  float scale, k_scale, v_scale;
+  pa_dtype q_dtype, cache_dtype, out_dtype;
+  int partition;                 // resolved, tokens
+  WorkspaceLayout ws;
+  void* workspace;
+};
+
+// PA_OK, PA_ERR_UNSUPPORTED (no kernel for the combination) or PA_ERR_CUDA.
+int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Read and clear the device error words of the kernel files (synchronises stream).
+cudaError_t read_and_clear_cache_errors(unsigned* bits, cudaStream_t stream);
+cudaError_t read_and_clear_decode_errors(unsigned* bits, cudaStream_t stream);
+
+}  // namespace pa
