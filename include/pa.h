@@ -163,6 +163,40 @@ int pa_copy_blocks(void* const* key_caches, void* const* value_caches, int num_l
                    const int64_t* block_mapping, int num_pairs, size_t block_bytes,
                    int64_t num_blocks, void* stream);
 
+/* Size of the library's own decode scratch (see below): 16 MiB per GPU. */
+#define PA_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)
+
+/*
+ * pa_paged_attention_decode_static_workspace -- pa_paged_attention_decode for
+ * callers that cannot allocate device memory.  The pages have no counterpart to
+ * this entry point; it exists for the library's users.
+ *
+ * Who needs it: a plugin inside a host process that owns every device allocation
+ * and gives its plugins no allocator; a serving engine that has already reserved
+ * nearly all HBM for its KV block pool, so that a late cudaMalloc would fail (and
+ * cudaMalloc / cudaFree would also synchronise the device mid-step).
+ *
+ * Same arguments, layouts and results as pa_paged_attention_decode, minus the
+ * workspace: the split-partition scratch lives in a fixed array of
+ * PA_STATIC_WORKSPACE_BYTES in the library's own device memory, which every GPU
+ * that loads the library's device code holds until the process exits.  This
+ * function allocates nothing and calls no allocating routine.
+ *   - Sizes whose pa_paged_attention_workspace_size() exceeds
+ *     PA_STATIC_WORKSPACE_BYTES are rejected with PA_ERR_WORKSPACE.
+ *   - The first call on a device that needs scratch looks up the array's device
+ *     address (cudaGetSymbolAddress, with that device current) and caches it;
+ *     make that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls whose work overlaps
+ *     on the GPU (other streams, other host threads) race on it: serialise them.
+ */
+int pa_paged_attention_decode_static_workspace(
+    void* out, const void* query, const void* key_cache, const void* value_cache,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+    int max_seq_len, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int64_t num_blocks, float scale, pa_dtype q_dtype, pa_dtype cache_dtype, pa_dtype out_dtype,
+    float k_scale, float v_scale, int partition_size, void* stream);
+
 /* Human-readable name of a pa_status value (static storage). */
 const char* pa_status_string(int status);
 

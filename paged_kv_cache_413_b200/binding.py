@@ -25,7 +25,8 @@ DEVERR = {0x1: "SLOT_RANGE", 0x2: "BLOCK_RANGE", 0x4: "SEQ_LEN", 0x8: "PIPE_TIME
           0x10: "COPY_RANGE"}
 EXPORTS = ("pa_reshape_and_cache", "pa_paged_attention_workspace_size",
            "pa_paged_attention_decode", "pa_copy_blocks", "pa_status_string",
-           "pa_get_device_error")
+           "pa_get_device_error", "pa_paged_attention_decode_static_workspace")
+PA_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 _DTYPE = {torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.float32: PA_F32,
           torch.float8_e4m3fn: PA_FP8_E4M3}
@@ -62,6 +63,9 @@ def library() -> ctypes.CDLL:
             lib.pa_paged_attention_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, I, L, F,
                                                       I, I, I, F, F, I, P, S, P]
             lib.pa_paged_attention_decode.restype = I
+            lib.pa_paged_attention_decode_static_workspace.argtypes = [
+                P, P, P, P, P, I, P, I, I, I, I, I, I, L, F, I, I, I, F, F, I, P]
+            lib.pa_paged_attention_decode_static_workspace.restype = I
             lib.pa_copy_blocks.argtypes = [P, P, I, P, I, S, L, P]
             lib.pa_copy_blocks.restype = I
             lib.pa_status_string.argtypes = [I]
@@ -145,6 +149,35 @@ def pa_paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache:
         block_tables.shape[1], _dev(seq_lens, "seq_lens"), b, int(max_seq_len), h, hkv, d, bs,
         nb, float(scale), _dt(query, "query"), _dt(key_cache, "key_cache"), _dt(out, "out"),
         float(k_scale), float(v_scale), int(partition_size), ws_ptr, ws_bytes, _stream(stream)))
+
+
+def pa_paged_attention_decode_static_workspace(out: torch.Tensor, query: torch.Tensor,
+                                               key_cache: torch.Tensor, value_cache: torch.Tensor,
+                                               block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                                               *, max_seq_len: int, scale: float,
+                                               k_scale: float = 1.0, v_scale: float = 1.0,
+                                               partition_size: int = 0, stream=None) -> None:
+    """Decode without a caller workspace, for callers that cannot allocate device memory
+    (plugins whose host owns all allocations; engines that gave nearly all HBM to the KV
+    pool).  The scratch is the library's fixed 16 MiB per-GPU array: sizes that need more
+    raise PaError(PA_ERR_WORKSPACE); calls that overlap on the GPU race on it."""
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    b, h, d = query.shape
+    nb, hkv, bs, d2 = key_cache.shape
+    if out.shape != query.shape or d2 != d or value_cache.shape != key_cache.shape or \
+            block_tables.dim() != 2 or block_tables.shape[0] != b or seq_lens.shape != (b,):
+        raise ValueError("shape mismatch")
+    status = library().pa_paged_attention_decode_static_workspace(
+        _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
+        _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+        block_tables.shape[1], _dev(seq_lens, "seq_lens"), b, int(max_seq_len), h, hkv, d, bs,
+        nb, float(scale), _dt(query, "query"), _dt(key_cache, "key_cache"), _dt(out, "out"),
+        float(k_scale), float(v_scale), int(partition_size), _stream(stream))
+    if status == -3:
+        raise PaError("pa_paged_attention_decode_static_workspace (needs more than the "
+                      f"{PA_STATIC_WORKSPACE_BYTES} bytes of static scratch)", status)
+    _check("pa_paged_attention_decode_static_workspace", status)
 
 
 def pa_copy_blocks(key_caches: list, value_caches: list, block_mapping: torch.Tensor, *,
