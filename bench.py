@@ -242,8 +242,8 @@ def run_ours(args, rank, world, local_rank):
     bm = f(wl.block_mapping) if wl.block_mapping is not None and wl.block_mapping.numel() else None
     max_len = int(wl.seq_lens.max())
     part = args.partition if args.partition is not None else cfg.partition_size
-    ws_n = pa.pa_paged_attention_workspace_size(q.shape[0], cfg.num_heads, cfg.head_dim, max_len,
-                                                part)
+    ws_n = pa.pa_paged_attention_workspace_size(q.shape[0], cfg.num_heads, cfg.num_kv_heads,
+                                                cfg.head_dim, max_len, part)
     ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
     out = torch.empty(q.shape, dtype=TORCH_DT[out_dtype], device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -251,7 +251,8 @@ def run_ours(args, rank, world, local_rank):
         pa.pa_reshape_and_cache(f(wl.prefix_key), f(wl.prefix_value), kc, vc,
                                 f(wl.prefix_slot_mapping), k_scale=wl.k_scale,
                                 v_scale=wl.v_scale)
-    part_eff = part if part > 0 else 512
+    part_eff = pa.pa_paged_attention_partition_size(q.shape[0], cfg.num_heads, cfg.num_kv_heads,
+                                                    max_len, part)
     reduce_runs = max_len > part_eff
     launches = 1 + 1 + (1 if reduce_runs else 0) + (1 if bm is not None else 0)
 

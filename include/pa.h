@@ -95,8 +95,12 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
  * pa_paged_attention_workspace_size -- bytes of device workspace that
  * pa_paged_attention_decode needs for these sizes (0 when every sequence fits in
  * one partition, i.e. max_seq_len <= the partition size).
- * partition_size: 0 = the library's default (512 tokens), else a positive
- * multiple of the block size.  Returns 0 also for invalid arguments.
+ * partition_size: 0 = the library's default, else a positive multiple of the
+ * block size.  The default keeps a sequence whole when the batch has at least
+ * 2048 (sequence, head group) units, a head group being the largest of 8, 4, 2, 1
+ * query heads dividing num_heads / num_kv_heads; otherwise it splits sequences
+ * into enough partitions of at least 256 tokens to reach 2048 units.
+ * Returns 0 also for invalid arguments.
  *
  * Workspace layout (fp32, each section 256-byte aligned), P = ceil(max_seq_len /
  * partition):  m[num_seqs][num_heads][P], l[num_seqs][num_heads][P],
@@ -104,8 +108,16 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
  * score m (natural-log units), the sum l of exp(score - m) and the normalised
  * partial output o.
  */
-size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int head_dim,
-                                         int max_seq_len, int partition_size);
+size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int max_seq_len, int partition_size);
+
+/*
+ * pa_paged_attention_partition_size -- the partition length in tokens that
+ * pa_paged_attention_decode uses for these sizes and this request (0 = default,
+ * as described above).  Host only.  Returns 0 for invalid arguments.
+ */
+int pa_paged_attention_partition_size(int num_seqs, int num_heads, int num_kv_heads,
+                                      int max_seq_len, int partition_size);
 
 /*
  * pa_paged_attention_decode -- one query token per sequence attends over its
@@ -127,7 +139,8 @@ size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int head_d
  *   scale         the softmax scale (normally 1/sqrt(head_dim))
  *   k_scale,
  *   v_scale       FP8 dequantisation scales; ignored for F16/BF16 caches
- *   partition_size  0 = default (512), else a positive multiple of block_size
+ *   partition_size  0 = default (see the size function), else a positive
+ *                 multiple of block_size
  *   workspace     device buffer of at least pa_paged_attention_workspace_size()
  *                 bytes (may be NULL when that size is 0); contents on entry are
  *                 ignored, on exit unspecified

@@ -24,6 +24,7 @@ STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED",
 DEVERR = {0x1: "SLOT_RANGE", 0x2: "BLOCK_RANGE", 0x4: "SEQ_LEN", 0x8: "PIPE_TIMEOUT",
           0x10: "COPY_RANGE"}
 EXPORTS = ("pa_reshape_and_cache", "pa_paged_attention_workspace_size",
+           "pa_paged_attention_partition_size",
            "pa_paged_attention_decode", "pa_copy_blocks", "pa_status_string",
            "pa_get_device_error", "pa_paged_attention_decode_static_workspace")
 PA_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
@@ -58,8 +59,10 @@ def library() -> ctypes.CDLL:
                              ctypes.c_size_t)
             lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, L, I, I, F, F, P]
             lib.pa_reshape_and_cache.restype = I
-            lib.pa_paged_attention_workspace_size.argtypes = [I, I, I, I, I]
+            lib.pa_paged_attention_workspace_size.argtypes = [I, I, I, I, I, I]
             lib.pa_paged_attention_workspace_size.restype = S
+            lib.pa_paged_attention_partition_size.argtypes = [I, I, I, I, I]
+            lib.pa_paged_attention_partition_size.restype = I
             lib.pa_paged_attention_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, I, L, F,
                                                       I, I, I, F, F, I, P, S, P]
             lib.pa_paged_attention_decode.restype = I
@@ -120,9 +123,17 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torc
         _stream(stream)))
 
 
-def pa_paged_attention_workspace_size(num_seqs: int, num_heads: int, head_dim: int,
+def pa_paged_attention_workspace_size(num_seqs: int, num_heads: int, num_kv_heads: int,
+                                      head_dim: int, max_seq_len: int,
+                                      partition_size: int = 0) -> int:
+    return int(library().pa_paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads,
+                                                            head_dim, max_seq_len,
+                                                            partition_size))
+
+
+def pa_paged_attention_partition_size(num_seqs: int, num_heads: int, num_kv_heads: int,
                                       max_seq_len: int, partition_size: int = 0) -> int:
-    return int(library().pa_paged_attention_workspace_size(num_seqs, num_heads, head_dim,
+    return int(library().pa_paged_attention_partition_size(num_seqs, num_heads, num_kv_heads,
                                                             max_seq_len, partition_size))
 
 

@@ -47,13 +47,23 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
       num_blocks, src_dtype, cache_dtype, k_scale, v_scale, static_cast<cudaStream_t>(stream)));
 }
 
-size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int head_dim,
-                                         int max_seq_len, int partition_size) {
-  if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_seq_len < 0 || partition_size < 0 ||
+size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int max_seq_len, int partition_size) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+      head_dim <= 0 || max_seq_len < 0 || partition_size < 0 ||
       partition_size % pa::kBlockSize != 0)
     return 0;
-  const int part = pa::resolve_partition(partition_size);
+  const int part =
+      pa::resolve_partition(partition_size, num_seqs, num_heads, num_kv_heads, max_seq_len);
   return pa::workspace_layout(num_seqs, num_heads, head_dim, max_seq_len, part).total;
+}
+
+int pa_paged_attention_partition_size(int num_seqs, int num_heads, int num_kv_heads,
+                                      int max_seq_len, int partition_size) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+      max_seq_len < 0 || partition_size < 0 || partition_size % pa::kBlockSize != 0)
+    return 0;
+  return pa::resolve_partition(partition_size, num_seqs, num_heads, num_kv_heads, max_seq_len);
 }
 
 int pa_paged_attention_decode(void* out, const void* query, const void* key_cache,
@@ -90,7 +100,8 @@ int pa_paged_attention_decode(void* out, const void* query, const void* key_cach
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
       (reinterpret_cast<uintptr_t>(block_tables) & 3u))
     return PA_ERR_INVALID_ARG;
-  const int part = pa::resolve_partition(partition_size);
+  const int part =
+      pa::resolve_partition(partition_size, num_seqs, num_heads, num_kv_heads, max_seq_len);
   pa::DecodeArgs a{};
   a.ws = pa::workspace_layout(num_seqs, num_heads, head_dim, max_seq_len, part);
   if (a.ws.total > 0 && (!workspace || workspace_bytes < a.ws.total || !aligned16(workspace)))

@@ -23,7 +23,11 @@
 // Scores are kept in log2 units (q is pre-multiplied by scale * log2(e) and, for
 // FP8 caches, by k_scale), so exponentials are exp2.
 
+#include <cuda.h>  // CUtensorMap and its enums (types only; no driver library link)
 #include <math.h>
+#include <string.h>
+
+#include <type_traits>
 
 #include "pa_common.cuh"
 #include "pa_internal.h"
@@ -35,7 +39,20 @@ __device__ unsigned int g_decode_err;
 
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = 8;
+// Ring depths.  Block i goes to stage i % stages and to consumer warp i % 4, so a
+// stage count that is a multiple of the warp count gives every stage a single
+// owning warp.  That matters: a parity wait cannot tell phase k from phase k - 2,
+// so a warp must never wait on a stage whose previous phase another warp is still
+// filling or reading.
+#ifndef PA_MMA16_STAGES
+#define PA_MMA16_STAGES 4
+#endif
+constexpr int kStagesSimt = 8;                  // 8 KB K+V per stage at D = 128, 16-bit
+constexpr int kStagesMma16 = PA_MMA16_STAGES;   // 8 KB per stage; 4 CTAs per SM
+constexpr int kStagesMmaFp8 = 8;                // 4 KB per stage
+static_assert(kStagesSimt % kConsumerWarps == 0 && kStagesMma16 % kConsumerWarps == 0 &&
+                  kStagesMmaFp8 % kConsumerWarps == 0,
+              "each ring stage must belong to one consumer warp");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -156,19 +173,57 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, float v, int d
     static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
 }
 
-template <int D, int GT, typename CT>
+// Merge the consumer warps' softmax states (cm: max in log2 units, cl: sum,
+// cacc: unnormalised accumulators, all in shared memory) and store the result:
+// the output itself when the sequence has one partition, else this partition's
+// (m, l, o) for the log-sum-exp reduce.
+template <int D, int GT>
+__device__ __forceinline__ void combine_and_store(const float* cm, const float* cl,
+                                                  const float* cacc, const Params& p, int seq,
+                                                  int part, int head0, int nparts) {
+  for (int e = threadIdx.x; e < GT * D; e += kThreads) {
+    const int g = e / D, d = e - g * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * GT + g]);
+    float Ls = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float mw = cm[w * GT + g];
+      if (mw == -INFINITY) continue;  // warp saw no block
+      const float f = exp2f(mw - M);
+      Ls += cl[w * GT + g] * f;
+      O += cacc[(w * GT + g) * D + d] * f;
+    }
+    const float o = O / Ls * p.v_mult;
+    const int64_t row = int64_t(seq) * p.num_heads + head0 + g;
+    if (nparts == 1) {
+      store_out(p.out, row * D + d, o, p.out_dtype);
+    } else {
+      const int64_t r = row * p.max_parts + part;
+      p.ws_o[r * D + d] = o;
+      if (d == 0) {
+        p.ws_m[r] = M * kLn2;
+        p.ws_l[r] = Ls;
+      }
+    }
+  }
+}
+
+template <int D, int GT, typename CT, int S>
 constexpr size_t smem_bytes() {
   constexpr size_t tile = size_t(kBlockSize) * D * CacheTraits<CT>::bytes;
-  constexpr size_t pipe = 2 * kStages * tile;
+  constexpr size_t pipe = 2 * S * tile;
   constexpr size_t combine = size_t(kConsumerWarps) * GT * (D + 2) * sizeof(float);
   constexpr size_t body = pipe > combine ? pipe : combine;
-  return body + 2 * kStages * sizeof(uint64_t) + size_t(kConsumerWarps) * GT * 16 * sizeof(float);
+  return body + 2 * S * sizeof(uint64_t) + size_t(kConsumerWarps) * GT * 16 * sizeof(float);
 }
 
 // GT: query heads served by one CTA (a divisor of the GQA group, at most 8).
-template <int D, int GT, typename CT, typename QT>
+template <int D, int GT, typename CT, typename QT, int kStages>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(kStages % kConsumerWarps == 0, "each ring stage must belong to one warp");
   constexpr int DPL = D / 32;
   constexpr int TILE = kBlockSize * D * CacheTraits<CT>::bytes;
   constexpr int TC = GT >= 2 ? 32 / GT : 16;  // tokens per reduction chunk
@@ -194,6 +249,13 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   const int hsub = blockIdx.y - kvh * p.head_groups;
   const int head0 = kvh * p.group + hsub * GT;  // first query head of this CTA
 
+  // The producer starts the first block-table read before anything else; the row
+  // has max_blocks_per_seq entries, so the speculative read stays inside it.
+  const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
+  const int blk_begin = part * (p.partition / kBlockSize);
+  int32_t phys_first = 0;
+  if (warp == kConsumerWarps && blk_begin + lane < p.max_blocks_per_seq)
+    phys_first = table_row[blk_begin + lane];
   // Sequence length, range-checked against the launch bound and the table width.
   int L = p.seq_lens[seq];
   const int cap = min(p.max_seq_len, p.max_blocks_per_seq * kBlockSize);
@@ -211,7 +273,6 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   }
   const int tok_begin = part * p.partition;
   const int tok_end = min(L, tok_begin + p.partition);
-  const int blk_begin = tok_begin / kBlockSize;
   const int nblk = (tok_end - tok_begin + kBlockSize - 1) / kBlockSize;
 
   if (tid == 0) {
@@ -228,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
 
   if (warp == kConsumerWarps) {
     // ---------------- producer: block table -> bulk copies ----------------
-    const int32_t* table = p.block_tables + int64_t(seq) * p.max_blocks_per_seq + blk_begin;
+    const int32_t* table = table_row + blk_begin;
     const uint64_t policy = l2_policy_evict_first();
     const size_t head_off = size_t(kvh) * TILE;
     const size_t block_stride = size_t(p.num_kv_heads) * TILE;
@@ -237,7 +298,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
     for (int base = 0; base < nblk && ok; base += 32) {
       int32_t phys = 0;
       if (base + lane < nblk) {
-        phys = table[base + lane];
+        phys = base == 0 ? phys_first : table[base + lane];
         if (phys < 0 || phys >= p.num_blocks) {
           atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
           phys = 0;
@@ -378,68 +439,419 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
       for (int e = 0; e < DPL; ++e) cacc[(warp * GT + g) * D + lane * DPL + e] = acc[g][e];
   }
   __syncthreads();
-  for (int e = tid; e < GT * D; e += kThreads) {
-    const int g = e / D, d = e - g * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * GT + g]);
-    float Ls = 0.f, O = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const float mw = cm[w * GT + g];
-      if (mw == -INFINITY) continue;  // warp saw no block
-      const float f = exp2f(mw - M);
-      Ls += cl[w * GT + g] * f;
-      O += cacc[(w * GT + g) * D + d] * f;
+  combine_and_store<D, GT>(cm, cl, cacc, p, seq, part, head0, nparts);
+  // let the merge kernel (launched as a programmatic dependent) get scheduled
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core consumer for GQA groups of 4 or 8 query heads (head_dim 128).
+//
+// Per 16-token block the two contractions are warp-level MMAs (m16n8k16, fp32
+// accumulate):  S^T[16 tokens x 8 heads] = K[16 x 128] . Q^T[128 x 8]  and
+// O^T[128 x 8] += V^T[128 x 16] . P^T[16 x 8].  The GQA heads are the N side,
+// so a group of 8 fills the instruction; P^T comes from the S^T accumulator by
+// an in-register 8x8 transpose (movmatrix).  Softmax stays fp32.  K/V blocks are
+// staged by tiled TMA with the 128-byte swizzle so that every ldmatrix is free
+// of bank conflicts.  For bf16, P is split into bf16 hi + lo parts (two MMAs)
+// so the probabilities keep ~16 significant bits.  E4M3 caches are widened to
+// f16 exactly in registers; a bf16 query is then scaled by a power of two into
+// f16 range (undone in the score multiplier).
+// ---------------------------------------------------------------------------
+struct TmaParams {
+  CUtensorMap tmk;  // K pool as [rows = blocks * kv_heads * 16][128] elements
+  CUtensorMap tmv;  // V pool, same view
+  Params p;
+};
+
+template <typename CT, int kStages>
+constexpr size_t mma_smem_bytes() {
+  constexpr size_t tile = size_t(kBlockSize) * 128 * CacheTraits<CT>::bytes;
+  constexpr size_t pipe = 2 * kStages * tile;
+  constexpr size_t combine = size_t(kConsumerWarps) * 8 * (128 + 2) * sizeof(float);
+  constexpr size_t body = pipe > combine ? pipe : combine;
+  return 1024 + body + 2 * kStages * sizeof(uint64_t);
+}
+
+template <int GT, typename CT, typename QT, int kStages>
+__global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_constant__ TmaParams tp) {
+  constexpr int D = 128;
+  constexpr bool kFp8 = CacheTraits<CT>::bytes == 1;
+  constexpr int TILE = kBlockSize * D * CacheTraits<CT>::bytes;
+  using MT = typename std::conditional<kFp8, __half, CT>::type;  // MMA element type
+  constexpr bool kSplitP = std::is_same<MT, __nv_bfloat16>::value;
+  static_assert(GT == 4 || GT == 8, "heads per CTA");
+  static_assert(kStages % kConsumerWarps == 0, "each ring stage must belong to one warp");
+  const Params& p = tp.p;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  constexpr size_t tile_region = 2 * kStages * size_t(TILE);
+  constexpr size_t combine_region = size_t(kConsumerWarps) * GT * (D + 2) * sizeof(float);
+  constexpr size_t body = tile_region > combine_region ? tile_region : combine_region;
+  uint8_t* kbuf = smem;
+  uint8_t* vbuf = smem + kStages * TILE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + body);
+  uint64_t* empty = full + kStages;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int seq = blockIdx.x / p.max_parts;
+  const int part = blockIdx.x - seq * p.max_parts;
+  const int kvh = blockIdx.y / p.head_groups;
+  const int hsub = blockIdx.y - kvh * p.head_groups;
+  const int head0 = kvh * p.group + hsub * GT;
+
+  const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
+  const int blk_begin = part * (p.partition / kBlockSize);
+  int32_t phys_first = 0;
+  if (warp == kConsumerWarps && blk_begin + lane < p.max_blocks_per_seq)
+    phys_first = table_row[blk_begin + lane];
+  int L = p.seq_lens[seq];
+  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * kBlockSize);
+  if (L < 0 || L > cap) {
+    if (tid == 0 && part == 0 && blockIdx.y == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
+    L = L < 0 ? 0 : cap;
+  }
+  const int nparts = (L + p.partition - 1) / p.partition;
+  if (part >= (nparts > 0 ? nparts : 1)) return;
+  if (L == 0) {
+    for (int e = tid; e < GT * D; e += kThreads)
+      store_out(p.out, (int64_t(seq) * p.num_heads + head0 + e / D) * D + e % D, 0.f,
+                p.out_dtype);
+    return;
+  }
+  const int tok_begin = part * p.partition;
+  const int tok_end = min(L, tok_begin + p.partition);
+  const int nblk = (tok_end - tok_begin + kBlockSize - 1) / kBlockSize;
+
+  if (tid == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
     }
-    const float o = O / Ls * p.v_mult;
-    const int64_t row = int64_t(seq) * p.num_heads + head0 + g;
-    if (nparts == 1) {
-      store_out(p.out, row * D + d, o, p.out_dtype);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  float acc[8][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const int g = lane >> 2, c = lane & 3;   // fragment row group / column pair
+  const int mi = lane >> 3, r = lane & 7;  // ldmatrix: matrix index / row
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: block table -> tiled TMA loads ----------------
+    const int32_t* table = table_row + blk_begin;
+    const uint64_t policy = l2_policy_evict_first();
+    int issued = 0;
+    bool ok = true;
+    for (int base = 0; base < nblk && ok; base += 32) {
+      int32_t phys = 0;
+      if (base + lane < nblk) {
+        phys = base == 0 ? phys_first : table[base + lane];
+        if (phys < 0 || phys >= p.num_blocks) {
+          atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
+          phys = 0;
+        }
+      }
+      const int cnt = min(32, nblk - base);
+      for (int j = 0; j < cnt; ++j) {
+        const int32_t pb = __shfl_sync(kFullMask, phys, j);
+        const int i = base + j, stage = i % kStages;
+        if (lane == 0) {
+          if (i >= kStages && !mbar_wait_bounded(&empty[stage], ((i / kStages) - 1) & 1)) {
+            atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+            ok = false;
+          }
+          if (ok) {
+            const int row = (pb * p.num_kv_heads + kvh) * kBlockSize;
+            uint8_t* kd = kbuf + stage * TILE;
+            uint8_t* vd = vbuf + stage * TILE;
+            mbar_arrive_expect_tx(&full[stage], 2 * TILE);
+            if constexpr (kFp8) {
+              tma_load_2d(kd, &tp.tmk, 0, row, &full[stage], policy);
+              tma_load_2d(vd, &tp.tmv, 0, row, &full[stage], policy);
+            } else {
+              tma_load_2d(kd, &tp.tmk, 0, row, &full[stage], policy);
+              tma_load_2d(kd + TILE / 2, &tp.tmk, 64, row, &full[stage], policy);
+              tma_load_2d(vd, &tp.tmv, 0, row, &full[stage], policy);
+              tma_load_2d(vd + TILE / 2, &tp.tmv, 64, row, &full[stage], policy);
+            }
+            ++issued;
+          }
+        }
+        ok = __shfl_sync(kFullMask, ok, 0);
+        if (!ok) break;
+      }
+    }
+    if (lane == 0) {
+      const int first = issued > kStages ? issued - kStages : 0;
+      for (int i = first; i < issued; ++i)
+        if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1))
+          atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- consumers ----------------
+    // Q^T as the B operand, one fragment pair per 16-wide k-step.  Heads past
+    // the group (GT = 4) are zero columns.
+    uint32_t qb[8][2];
+    float mult = p.q_mult;
+    const uint8_t* qrow = p.query + (int64_t(seq) * p.num_heads + head0 + (g < GT ? g : 0)) * D * 2;
+    if constexpr (!kFp8) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        qb[ks][0] = g < GT ? *reinterpret_cast<const uint32_t*>(qrow + (16 * ks + 2 * c) * 2) : 0u;
+        qb[ks][1] = g < GT ? *reinterpret_cast<const uint32_t*>(qrow + (16 * ks + 2 * c + 8) * 2) : 0u;
+      }
     } else {
-      const int64_t r = row * p.max_parts + part;
-      p.ws_o[r * D + d] = o;
-      if (d == 0) {
-        p.ws_m[r] = M * kLn2;
-        p.ws_l[r] = Ls;
+      // k-step ks covers dims 16 ks + 4c .. 4c+3 for this thread (see the K loads)
+      uint2 raw[8];
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        raw[ks] = g < GT ? *reinterpret_cast<const uint2*>(qrow + (16 * ks + 4 * c) * 2)
+                         : make_uint2(0u, 0u);
+      if constexpr (std::is_same<QT, __half>::value) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          qb[ks][0] = raw[ks].x;
+          qb[ks][1] = raw[ks].y;
+        }
+      } else {
+        // bf16 -> f16: scale by 2^sq so that the largest |q| of the group lands in
+        // [2^14, 2^15); the scores are multiplied back by 2^-sq.
+        float qmax = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const float2 a = unpack2(raw[ks].x, QT{}), b = unpack2(raw[ks].y, QT{});
+          qmax = fmaxf(qmax, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y))));
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(kFullMask, qmax, o));
+        int e = 0;
+        if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &e);
+        const int sq = min(max(15 - e, -100), 100);
+        mult = ldexpf(mult, -sq);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const float2 a = unpack2(raw[ks].x, QT{}), b = unpack2(raw[ks].y, QT{});
+          qb[ks][0] = pack2(ldexpf(a.x, sq), ldexpf(a.y, sq), __half{});
+          qb[ks][1] = pack2(ldexpf(b.x, sq), ldexpf(b.y, sq), __half{});
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+
+    for (int i = warp; i < nblk; i += kConsumerWarps) {
+      const int stage = i % kStages;
+      if (!__all_sync(kFullMask, mbar_wait_bounded(&full[stage], (i / kStages) & 1))) {
+        if (lane == 0) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+        break;
+      }
+      const uint32_t kt = smem_u32(kbuf + stage * TILE);
+      const uint32_t vt = smem_u32(vbuf + stage * TILE);
+      const int nvalid = min(kBlockSize, tok_end - (blk_begin + i) * kBlockSize);
+
+      // ---- S^T = K . Q^T ----
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (!kFp8) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const int tok = r + 8 * (mi & 1), j = 2 * ks + (mi >> 1);
+          uint32_t a[4];
+          ldsm_x4(kt + (j >> 3) * (TILE / 2) + tok * 128 + (((j & 7) ^ r) << 4), a);
+          mma_16816(sc, a, qb[ks][0], qb[ks][1], MT{});
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tok = r + 8 * (mi & 1), j = 2 * u + (mi >> 1);
+          uint32_t R[4];
+          ldsm_x4(kt + tok * 128 + ((j ^ r) << 4), R);
+          const uint32_t a0[4] = {e4m3x2_to_f16x2(R[0]), e4m3x2_to_f16x2(R[1]),
+                                  e4m3x2_to_f16x2(R[0] >> 16), e4m3x2_to_f16x2(R[1] >> 16)};
+          const uint32_t a1[4] = {e4m3x2_to_f16x2(R[2]), e4m3x2_to_f16x2(R[3]),
+                                  e4m3x2_to_f16x2(R[2] >> 16), e4m3x2_to_f16x2(R[3] >> 16)};
+          mma_16816(sc, a0, qb[2 * u][0], qb[2 * u][1], MT{});
+          mma_16816(sc, a1, qb[2 * u + 1][0], qb[2 * u + 1][1], MT{});
+        }
+      }
+      // sc = {S(g, 2c), S(g, 2c+1), S(g+8, 2c), S(g+8, 2c+1)} in log2 units
+      const bool v0 = g < nvalid, v8 = g + 8 < nvalid;  // rows past the context -> -inf
+      sc[0] = v0 ? sc[0] * mult : -INFINITY;
+      sc[1] = v0 ? sc[1] * mult : -INFINITY;
+      sc[2] = v8 ? sc[2] * mult : -INFINITY;
+      sc[3] = v8 ? sc[3] * mult : -INFINITY;
+      float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+      for (int o = 4; o <= 16; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      const float p0 = exp2f(sc[0] - mn0), p1 = exp2f(sc[1] - mn1);
+      const float p2 = exp2f(sc[2] - mn0), p3 = exp2f(sc[3] - mn1);
+      l0 = l0 * al0 + (p0 + p2);
+      l1 = l1 * al1 + (p1 + p3);
+      // P^T fragments: the accumulator layout of S^T is an m8n8 fragment per 8
+      // tokens; its transpose is the B operand of the P.V product.
+      const uint32_t x0 = pack2(p0, p1, MT{}), x1 = pack2(p2, p3, MT{});
+      const uint32_t bh0 = movmatrix_trans(x0), bh1 = movmatrix_trans(x1);
+      uint32_t bl0 = 0, bl1 = 0;
+      if constexpr (kSplitP) {
+        const float2 h0 = unpack2(x0, MT{}), h1 = unpack2(x1, MT{});
+        bl0 = movmatrix_trans(pack2(p0 - h0.x, p1 - h0.y, MT{}));
+        bl1 = movmatrix_trans(pack2(p2 - h1.x, p3 - h1.y, MT{}));
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        acc[t][0] *= al0;
+        acc[t][1] *= al1;
+        acc[t][2] *= al0;
+        acc[t][3] *= al1;
+      }
+      // zero V rows past the context: they may hold anything, even NaN
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (nvalid < kBlockSize) {
+        mlo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+        mhi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+      }
+      // ---- O^T += V^T . P^T ----
+      if constexpr (!kFp8) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int tok = r + 8 * (mi >> 1), j = 2 * t + (mi & 1);
+          uint32_t a[4];
+          ldsm_x4_trans(vt + (j >> 3) * (TILE / 2) + tok * 128 + (((j & 7) ^ r) << 4), a);
+          a[0] &= mlo;
+          a[1] &= mlo;
+          a[2] &= mhi;
+          a[3] &= mhi;
+          mma_16816(acc[t], a, bh0, bh1, MT{});
+          if constexpr (kSplitP) mma_16816(acc[t], a, bl0, bl1, MT{});
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tok = r + 8 * (mi & 1), j = 2 * u + (mi >> 1);
+          uint32_t R[4];
+          ldsm_x4_trans(vt + tok * 128 + ((j ^ r) << 4), R);
+          // R[q] bytes: (token 2c, dim d), (2c, d+1), (2c+1, d), (2c+1, d+1), d = 16 chunk + 2g
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t lo = R[2 * h], hi8 = R[2 * h + 1];
+            uint32_t a[4] = {e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x20)) & mlo,
+                             e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x31)) & mlo,
+                             e4m3x2_to_f16x2(__byte_perm(hi8, 0, 0x20)) & mhi,
+                             e4m3x2_to_f16x2(__byte_perm(hi8, 0, 0x31)) & mhi};
+            mma_16816(acc[2 * u + h], a, bh0, bh1, MT{});
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+    }
+#pragma unroll
+    for (int o = 4; o <= 16; o <<= 1) {
+      l0 += __shfl_xor_sync(kFullMask, l0, o);
+      l1 += __shfl_xor_sync(kFullMask, l1, o);
+    }
+  }
+
+  __syncthreads();  // pipeline finished: the tile region becomes the combine region
+  float* cm = reinterpret_cast<float*>(smem);
+  float* cl = cm + kConsumerWarps * GT;
+  float* cacc = cl + kConsumerWarps * GT;
+  if (warp < kConsumerWarps) {
+    if (g == 0) {
+      if (2 * c < GT) {
+        cm[warp * GT + 2 * c] = m0;
+        cl[warp * GT + 2 * c] = l0;
+      }
+      if (2 * c + 1 < GT) {
+        cm[warp * GT + 2 * c + 1] = m1;
+        cl[warp * GT + 2 * c + 1] = l1;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      // rows of the O^T fragment -> head dims
+      const int d0 = kFp8 ? 16 * t + 2 * g : 16 * t + g;
+      const int d1 = kFp8 ? d0 + 1 : d0 + 8;
+      if (2 * c < GT) {
+        cacc[(warp * GT + 2 * c) * D + d0] = acc[t][0];
+        cacc[(warp * GT + 2 * c) * D + d1] = acc[t][2];
+      }
+      if (2 * c + 1 < GT) {
+        cacc[(warp * GT + 2 * c + 1) * D + d0] = acc[t][1];
+        cacc[(warp * GT + 2 * c + 1) * D + d1] = acc[t][3];
       }
     }
   }
+  __syncthreads();
+  combine_and_store<D, GT>(cm, cl, cacc, p, seq, part, head0, nparts);
+  // let the merge kernel (launched as a programmatic dependent) get scheduled
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Log-sum-exp merge of the partitions of sequences with more than one:
 // M = max m_p, w_p = l_p exp(m_p - M), out = sum w_p o_p / sum w_p.
-// grid = num_seqs * num_heads (one CTA per output row), one thread per element.
-__global__ void lse_reduce_kernel(void* out, const float* __restrict__ ws_m,
-                                  const float* __restrict__ ws_l, const float* __restrict__ ws_o,
-                                  const int32_t* __restrict__ seq_lens, int num_heads,
-                                  int head_dim, int max_parts, int partition, int cap,
-                                  int out_dtype) {
-  const int seq = blockIdx.x / num_heads, h = blockIdx.x - seq * num_heads;
-  int L = seq_lens[seq];
+// One warp per (sequence, head) row, 8 rows per CTA; lanes own D/32 dims.
+// Launched as a programmatic dependent of the decode kernel: it waits for that
+// grid's results before reading the workspace.
+template <int D>
+__global__ void __launch_bounds__(256) lse_reduce_kernel(void* out, const float* __restrict__ ws_m,
+                                                         const float* __restrict__ ws_l,
+                                                         const float* __restrict__ ws_o,
+                                                         const int32_t* __restrict__ seq_lens,
+                                                         int num_rows, int num_heads,
+                                                         int max_parts, int partition, int cap,
+                                                         int out_dtype) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int DPL = D / 32;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= num_rows) return;
+  int L = seq_lens[row / num_heads];
   L = L < 0 ? 0 : (L > cap ? cap : L);
   const int nparts = (L + partition - 1) / partition;
   if (nparts <= 1) return;  // written by the decode kernel
-  const int64_t row = int64_t(seq) * num_heads + h;
-  const float* m = ws_m + row * max_parts;
-  const float* l = ws_l + row * max_parts;
+  const float* m = ws_m + int64_t(row) * max_parts;
+  const float* l = ws_l + int64_t(row) * max_parts;
+  const float* o = ws_o + int64_t(row) * max_parts * D + lane * DPL;
   float M = -INFINITY;
-  for (int q = 0; q < nparts; ++q) M = fmaxf(M, m[q]);
-  for (int d = threadIdx.x; d < head_dim; d += blockDim.x) {
-    float W = 0.f, O = 0.f;
-    for (int q = 0; q < nparts; ++q) {
-      const float w = l[q] * exp2f((m[q] - M) * kLog2e);
-      W += w;
-      O += w * ws_o[(row * max_parts + q) * head_dim + d];
+  for (int q = lane; q < nparts; q += 32) M = fmaxf(M, m[q]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
+  float acc[DPL] = {};
+  float W = 0.f;
+  for (int q = 0; q < nparts; ++q) {
+    const float w = l[q] * exp2f((m[q] - M) * kLog2e);
+    W += w;
+    if constexpr (DPL == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(o + int64_t(q) * D);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+      acc[2] = fmaf(w, v.z, acc[2]);
+      acc[3] = fmaf(w, v.w, acc[3]);
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(o + int64_t(q) * D);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
     }
-    store_out(out, row * head_dim + d, O / W, out_dtype);
   }
+  const float inv = 1.f / W;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e)
+    store_out(out, int64_t(row) * D + lane * DPL + e, acc[e] * inv, out_dtype);
 }
 
 template <int D, int GT, typename CT, typename QT>
 int launch_typed(const Params& p, int num_seqs, cudaStream_t stream) {
-  constexpr size_t smem = smem_bytes<D, GT, CT>();
-  auto kern = decode_kernel<D, GT, CT, QT>;
+  constexpr size_t smem = smem_bytes<D, GT, CT, kStagesSimt>();
+  auto kern = decode_kernel<D, GT, CT, QT, kStagesSimt>;
   // The shared-memory opt-in is set once per device and instantiation; a race
   // only repeats an idempotent call.
   static unsigned long long attr_set_mask = 0;
@@ -476,6 +888,75 @@ int dispatch_d(const Params& p, int d, int gt, int num_seqs, cudaStream_t s) {
   return PA_ERR_UNSUPPORTED;
 }
 
+// ---- tensor maps for the tensor-core kernel ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, fetched once through the runtime.
+EncodeTiledFn encode_fn() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// A pool [blocks][kv_heads][16][128] viewed as rows x 128 elements; boxes of 16 rows
+// and 128 bytes (64 16-bit or 128 E4M3 elements), 128-byte swizzle.
+bool encode_pool_map(CUtensorMap* m, const void* base, int64_t rows, bool fp8) {
+  const cuuint64_t dims[2] = {128, cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {fp8 ? 128u : 256u};
+  const cuuint32_t box[2] = {fp8 ? 128u : 64u, 16u};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                     const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int GT, typename CT, typename QT>
+int launch_mma_typed(const Params& p, const void* kc, const void* vc, int64_t rows, int num_seqs,
+                     cudaStream_t stream) {
+  constexpr bool fp8 = CacheTraits<CT>::bytes == 1;
+  constexpr int stages = fp8 ? kStagesMmaFp8 : kStagesMma16;
+  constexpr size_t smem = mma_smem_bytes<CT, stages>();
+  auto kern = decode_mma_kernel<GT, CT, QT, stages>;
+  static unsigned long long attr_set_mask = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set_mask & bit)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    attr_set_mask |= bit;
+  }
+  TmaParams tp;
+  memset(&tp, 0, sizeof tp);
+  tp.p = p;
+  if (!encode_pool_map(&tp.tmk, kc, rows, fp8) || !encode_pool_map(&tp.tmv, vc, rows, fp8))
+    return PA_ERR_CUDA;
+  const dim3 grid(unsigned(num_seqs) * unsigned(p.max_parts),
+                  unsigned(p.num_kv_heads * p.head_groups));
+  kern<<<grid, kThreads, smem, stream>>>(tp);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename CT, typename QT>
+int dispatch_mma(const Params& p, int gt, const void* kc, const void* vc, int64_t rows,
+                 int num_seqs, cudaStream_t s) {
+  if (gt == 8) return launch_mma_typed<8, CT, QT>(p, kc, vc, rows, num_seqs, s);
+  return launch_mma_typed<4, CT, QT>(p, kc, vc, rows, num_seqs, s);
+}
+
 }  // namespace
 
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
@@ -508,7 +989,23 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     p.ws_o = reinterpret_cast<float*>(w + a.ws.o_off);
   }
   int rc;
-  if (a.cache_dtype == PA_F16 && a.q_dtype == PA_F16)
+  const int64_t rows = a.num_blocks * a.num_kv_heads * kBlockSize;
+  const bool use_mma = a.head_dim == 128 && (gt == 4 || gt == 8) && rows < (int64_t(1) << 31) &&
+                       encode_fn() != nullptr;
+  if (use_mma) {
+    const void* kc = a.key_cache;
+    const void* vc = a.value_cache;
+    if (a.cache_dtype == PA_F16 && a.q_dtype == PA_F16)
+      rc = dispatch_mma<__half, __half>(p, gt, kc, vc, rows, a.num_seqs, stream);
+    else if (a.cache_dtype == PA_BF16 && a.q_dtype == PA_BF16)
+      rc = dispatch_mma<__nv_bfloat16, __nv_bfloat16>(p, gt, kc, vc, rows, a.num_seqs, stream);
+    else if (fp8 && a.q_dtype == PA_F16)
+      rc = dispatch_mma<fp8_e4m3, __half>(p, gt, kc, vc, rows, a.num_seqs, stream);
+    else if (fp8 && a.q_dtype == PA_BF16)
+      rc = dispatch_mma<fp8_e4m3, __nv_bfloat16>(p, gt, kc, vc, rows, a.num_seqs, stream);
+    else
+      rc = PA_ERR_UNSUPPORTED;
+  } else if (a.cache_dtype == PA_F16 && a.q_dtype == PA_F16)
     rc = dispatch_d<__half, __half>(p, a.head_dim, gt, a.num_seqs, stream);
   else if (a.cache_dtype == PA_BF16 && a.q_dtype == PA_BF16)
     rc = dispatch_d<__nv_bfloat16, __nv_bfloat16>(p, a.head_dim, gt, a.num_seqs, stream);
@@ -522,10 +1019,28 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int cap = a.max_seq_len < a.max_blocks_per_seq * kBlockSize
                       ? a.max_seq_len
                       : a.max_blocks_per_seq * kBlockSize;
-  lse_reduce_kernel<<<unsigned(a.num_seqs) * unsigned(a.num_heads), a.head_dim, 0, stream>>>(
-      a.out, p.ws_m, p.ws_l, p.ws_o, a.seq_lens, a.num_heads, a.head_dim, p.max_parts,
-      a.partition, cap, a.out_dtype);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const int out_rows = a.num_seqs * a.num_heads;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned((out_rows + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* wm = p.ws_m;
+  const float* wl = p.ws_l;
+  const float* wo = p.ws_o;
+  cudaError_t e;
+  if (a.head_dim == 128)
+    e = cudaLaunchKernelEx(&cfg, lse_reduce_kernel<128>, a.out, wm, wl, wo, a.seq_lens, out_rows,
+                           a.num_heads, p.max_parts, a.partition, cap, int(a.out_dtype));
+  else
+    e = cudaLaunchKernelEx(&cfg, lse_reduce_kernel<64>, a.out, wm, wl, wo, a.seq_lens, out_rows,
+                           a.num_heads, p.max_parts, a.partition, cap, int(a.out_dtype));
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 cudaError_t read_and_clear_decode_errors(unsigned* bits, cudaStream_t stream) {

@@ -57,8 +57,8 @@ extern "C" int pa_paged_attention_decode_static_workspace(
     int max_seq_len, int num_heads, int num_kv_heads, int head_dim, int block_size,
     int64_t num_blocks, float scale, pa_dtype q_dtype, pa_dtype cache_dtype, pa_dtype out_dtype,
     float k_scale, float v_scale, int partition_size, void* stream) {
-  const size_t need = pa_paged_attention_workspace_size(num_seqs, num_heads, head_dim,
-                                                        max_seq_len, partition_size);
+  const size_t need = pa_paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads,
+                                                        head_dim, max_seq_len, partition_size);
   if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_WORKSPACE;  // beyond the fixed maximum
   void* scratch = nullptr;
   if (need > 0) {

@@ -19,9 +19,30 @@ struct WorkspaceLayout {
   int max_parts;                           // partitions of the longest sequence
 };
 
-// Partition size in tokens for a requested value (0 = default).
-inline int resolve_partition(int requested) {
-  return requested > 0 ? requested : kDefaultPartition;
+constexpr int kAutoTargetCtas = 2048;   // work units that keep a B200's 148 SMs streaming
+constexpr int kAutoMinPartition = 256;  // smallest partition the default ever picks
+
+// Query heads served by one CTA: the largest of 8, 4, 2, 1 dividing the group.
+inline int heads_per_cta(int group) {
+  return group % 8 == 0 ? 8 : group % 4 == 0 ? 4 : group % 2 == 0 ? 2 : 1;
+}
+
+// Partition size in tokens.  A positive request is taken as is.  The default (0)
+// splits a sequence only when there are fewer than kAutoTargetCtas (sequence,
+// head group) units to spread over the GPU: then into enough partitions of at
+// least kAutoMinPartition tokens to reach that count.  Longer partitions amortise
+// each CTA's pipeline fill and epilogue and avoid the merge pass.
+inline int resolve_partition(int requested, int num_seqs, int num_heads, int num_kv_heads,
+                             int max_seq_len) {
+  if (requested > 0) return requested;
+  const int whole = max_seq_len > 16 ? (max_seq_len + 15) / 16 * 16 : 16;
+  const int64_t units =
+      int64_t(num_seqs) * num_heads / heads_per_cta(num_kv_heads > 0 ? num_heads / num_kv_heads : 1);
+  if (units >= kAutoTargetCtas) return whole;
+  const int64_t splits = (kAutoTargetCtas + units - 1) / (units > 0 ? units : 1);
+  int part = int((max_seq_len + splits - 1) / splits + 15) / 16 * 16;
+  if (part < kAutoMinPartition) part = kAutoMinPartition;
+  return part < whole ? part : whole;
 }
 
 inline WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim,

@@ -59,8 +59,8 @@ def gpu_prepare(wl: W.Workload, d: Dev) -> None:
 
 def workspace_for(wl: W.Workload, partition_size: int, dev: str = "cuda"):
     n = pa.pa_paged_attention_workspace_size(wl.cfg.num_seqs * max(1, wl.cfg.beam_width),
-                                             wl.cfg.num_heads, wl.cfg.head_dim,
-                                             max_seq_len(wl), partition_size)
+                                             wl.cfg.num_heads, wl.cfg.num_kv_heads,
+                                             wl.cfg.head_dim, max_seq_len(wl), partition_size)
     return torch.empty(n, dtype=torch.uint8, device=dev) if n else None
 
 

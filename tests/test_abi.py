@@ -46,17 +46,34 @@ def test_status_strings(lib):
 
 
 def test_workspace_size_host_function(lib):
-    # one partition: no workspace
-    assert pa.pa_paged_attention_workspace_size(64, 32, 128, 512, 0) == 0
-    assert pa.pa_paged_attention_workspace_size(64, 32, 128, 512, 512) == 0
-    # 8 x 32 heads x 64 partitions: m, l (256-byte aligned) and o
-    rows = 8 * 32 * 64
+    ws = pa.pa_paged_attention_workspace_size
     up = lambda x: (x + 255) // 256 * 256
-    assert pa.pa_paged_attention_workspace_size(8, 32, 128, 32768, 512) == \
-        up(rows * 4) * 2 + up(rows * 128 * 4)
-    assert pa.pa_paged_attention_workspace_size(8, 32, 128, 32768, 0) == \
-        pa.pa_paged_attention_workspace_size(8, 32, 128, 32768, 512)
-    assert pa.pa_paged_attention_workspace_size(8, 32, 128, 1000, 24) == 0  # not a multiple of 16
+    # explicit partitions: one partition needs no workspace
+    assert ws(64, 32, 32, 128, 512, 512) == 0
+    # 8 seqs x 32 heads x 64 partitions of 512: m, l (256-byte aligned) and o
+    rows = 8 * 32 * 64
+    assert ws(8, 32, 8, 128, 32768, 512) == up(rows * 4) * 2 + up(rows * 128 * 4)
+    # default: >= 2048 (sequence, head group) units keep sequences whole
+    assert ws(64, 32, 32, 128, 2048, 0) == 0          # MHA: 64 x 32 units
+    assert ws(256, 64, 8, 128, 768, 0) == 0           # GQA-8: 256 x 8 units
+    # default: 8 x 32 / 4 = 64 units -> 32 partitions of 1024 tokens
+    rows = 8 * 32 * 32
+    assert ws(8, 32, 8, 128, 32768, 0) == up(rows * 4) * 2 + up(rows * 128 * 4)
+    # default never goes below 256-token partitions
+    rows = 4 * 4 * 4
+    assert ws(4, 4, 4, 64, 1000, 0) == up(rows * 4) * 2 + up(rows * 64 * 4)
+    assert ws(4, 4, 4, 64, 100, 0) == 0
+    assert ws(8, 32, 8, 128, 1000, 24) == 0           # not a multiple of 16
+    assert ws(8, 30, 8, 128, 1000, 0) == 0            # heads not a multiple of kv heads
+    part = pa.pa_paged_attention_partition_size
+    assert part(64, 32, 32, 2048, 0) == 2048
+    assert part(256, 64, 8, 768, 0) == 768
+    assert part(256, 32, 8, 1036, 0) == 1040            # whole, rounded up to a block
+    assert part(8, 32, 8, 32768, 0) == 1024
+    assert part(8, 32, 8, 32768, 512) == 512
+    assert part(4, 4, 4, 1000, 0) == 256
+    assert part(4, 4, 4, 100, 0) == 112
+    assert part(4, 4, 4, 100, 8) == 0
 
 
 def test_host_validation_without_gpu(lib):

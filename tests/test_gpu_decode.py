@@ -154,7 +154,7 @@ def test_workspace_errors():
     wl = W.make_workload("tiny")
     d = flow.to_device(wl)
     out = torch.empty(d.query.shape, dtype=torch.float16, device="cuda")
-    need = pa.pa_paged_attention_workspace_size(4, 4, 64, 100, 16)
+    need = pa.pa_paged_attention_workspace_size(4, 4, 4, 64, 100, 16)
     assert need > 0
     small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(pa.PaError, match="WORKSPACE"):

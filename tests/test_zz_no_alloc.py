@@ -35,7 +35,8 @@ def test_static_workspace_matches_workspace_entry_point(name, over, part, out_dt
     ref = flow.gpu_step(wl, d, out_dtype, part)        # existing entry point, own workspace
     max_len = flow.max_seq_len(wl)
     need = pa.pa_paged_attention_workspace_size(d.query.shape[0], wl.cfg.num_heads,
-                                                wl.cfg.head_dim, max_len, part)
+                                                wl.cfg.num_kv_heads, wl.cfg.head_dim, max_len,
+                                                part)
     assert 0 < need <= pa.binding.PA_STATIC_WORKSPACE_BYTES
     outs = []
     for call in range(2):
@@ -63,7 +64,7 @@ def test_static_workspace_rejects_sizes_beyond_the_maximum():
     # 4 seqs x 4 heads x 8192 partitions of 16 tokens x (64 + 2) floats: ~34.6 MB of scratch
     max_len = 16 * 8192
     bt = torch.zeros(4, 8192, dtype=torch.int32, device="cuda")
-    assert pa.pa_paged_attention_workspace_size(4, 4, 64, max_len, 16) > \
+    assert pa.pa_paged_attention_workspace_size(4, 4, 4, 64, max_len, 16) > \
         pa.binding.PA_STATIC_WORKSPACE_BYTES
     with pytest.raises(pa.PaError, match="static scratch"):
         pa.pa_paged_attention_decode_static_workspace(
