@@ -103,6 +103,20 @@ def copy_bytes(wl: W.Workload) -> int:
 
 
 # ---------------------------------------------------------------- helpers
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    if world <= 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_gbs(step_bytes: int, world: int, steps: int, elapsed_ms: float) -> float:
+    """Replicas: every rank processes its own batch, so the job moves world x the bytes."""
+    return step_bytes * world * steps / (elapsed_ms * 1e-3) / 1e9
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -298,16 +312,13 @@ def run_ours(args, rank, world, local_rank):
         sampler.__exit__(None, None, None)
     elapsed_ms = t0.elapsed_time(t1)
     decode_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    if world > 1:
-        t = torch.tensor([elapsed_ms, decode_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms, decode_ms = t.tolist()
+    elapsed_ms, decode_ms = max_over_ranks([elapsed_ms, decode_ms], world, dev)
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error bits set during the timed steps")
 
     step_bytes = decode_bytes(wl, out_dtype) + cache_write_bytes(wl) + copy_bytes(wl)
     ms_per_step = elapsed_ms / args.steps
-    value = step_bytes * world * args.steps / (elapsed_ms * 1e-3) / 1e9
+    value = whole_job_gbs(step_bytes, world, args.steps, elapsed_ms)
 
     # ---- end to end through the public API with host buffers
     pin = lambda t: None if t is None else t.pin_memory()
@@ -340,12 +351,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     a1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = a0.elapsed_time(a1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = t.item()
-    e2e_value = step_bytes * world * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks([a0.elapsed_time(a1)], world, dev)[0]
+    e2e_value = whole_job_gbs(step_bytes, world, e2e_steps, e2e_ms)
 
     if rank != 0:
         return None

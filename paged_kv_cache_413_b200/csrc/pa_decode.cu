@@ -173,40 +173,65 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, float v, int d
     static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
 }
 
+// Combine region layout: per warp and head the max (log2 units) and the sum, then
+// the unnormalised accumulators with rows padded to D + 4 floats, which keeps the
+// fragment-order writes of the four column groups on distinct banks.
+template <int D>
+constexpr int combine_row() {
+  return D + 4;
+}
+template <int D, int GT>
+constexpr size_t combine_bytes() {
+  return (size_t(kConsumerWarps) * GT * 2 + size_t(kConsumerWarps) * GT * combine_row<D>() +
+          size_t(GT) * (kConsumerWarps + 1)) *
+         sizeof(float);
+}
+
 // Merge the consumer warps' softmax states (cm: max in log2 units, cl: sum,
 // cacc: unnormalised accumulators, all in shared memory) and store the result:
 // the output itself when the sequence has one partition, else this partition's
-// (m, l, o) for the log-sum-exp reduce.
+// (m, l, o) for the log-sum-exp reduce.  The per-head factors are computed once
+// (cf: the weight of each warp divided by the total) before the element loop.
 template <int D, int GT>
 __device__ __forceinline__ void combine_and_store(const float* cm, const float* cl,
-                                                  const float* cacc, const Params& p, int seq,
-                                                  int part, int head0, int nparts) {
-  for (int e = threadIdx.x; e < GT * D; e += kThreads) {
-    const int g = e / D, d = e - g * D;
+                                                  const float* cacc, float* cf, const Params& p,
+                                                  int seq, int part, int head0, int nparts) {
+  constexpr int R = combine_row<D>();
+  if (threadIdx.x < GT) {
+    const int g = threadIdx.x;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * GT + g]);
-    float Ls = 0.f, O = 0.f;
+    float f[kConsumerWarps];
+    float Ls = 0.f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
       const float mw = cm[w * GT + g];
-      if (mw == -INFINITY) continue;  // warp saw no block
-      const float f = exp2f(mw - M);
-      Ls += cl[w * GT + g] * f;
-      O += cacc[(w * GT + g) * D + d] * f;
+      f[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);  // a warp that saw no block weighs 0
+      Ls += cl[w * GT + g] * f[w];
     }
-    const float o = O / Ls * p.v_mult;
+    const float inv = p.v_mult / Ls;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) cf[g * (kConsumerWarps + 1) + w] = f[w] * inv;
+    cf[g * (kConsumerWarps + 1) + kConsumerWarps] = Ls;
+    if (nparts > 1) {
+      const int64_t r = (int64_t(seq) * p.num_heads + head0 + g) * p.max_parts + part;
+      p.ws_m[r] = M * kLn2;
+      p.ws_l[r] = Ls;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < GT * D; e += kThreads) {
+    const int g = e / D, d = e - g * D;
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w)
+      o = fmaf(cacc[(w * GT + g) * R + d], cf[g * (kConsumerWarps + 1) + w], o);
     const int64_t row = int64_t(seq) * p.num_heads + head0 + g;
-    if (nparts == 1) {
+    if (nparts == 1)
       store_out(p.out, row * D + d, o, p.out_dtype);
-    } else {
-      const int64_t r = row * p.max_parts + part;
-      p.ws_o[r * D + d] = o;
-      if (d == 0) {
-        p.ws_m[r] = M * kLn2;
-        p.ws_l[r] = Ls;
-      }
-    }
+    else
+      p.ws_o[(row * p.max_parts + part) * D + d] = o;
   }
 }
 
@@ -214,7 +239,7 @@ template <int D, int GT, typename CT, int S>
 constexpr size_t smem_bytes() {
   constexpr size_t tile = size_t(kBlockSize) * D * CacheTraits<CT>::bytes;
   constexpr size_t pipe = 2 * S * tile;
-  constexpr size_t combine = size_t(kConsumerWarps) * GT * (D + 2) * sizeof(float);
+  constexpr size_t combine = combine_bytes<D, GT>();
   constexpr size_t body = pipe > combine ? pipe : combine;
   return body + 2 * S * sizeof(uint64_t) + size_t(kConsumerWarps) * GT * 16 * sizeof(float);
 }
@@ -234,7 +259,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
 
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr size_t tile_region = 2 * kStages * size_t(TILE);
-  constexpr size_t combine_region = size_t(kConsumerWarps) * GT * (D + 2) * sizeof(float);
+  constexpr size_t combine_region = combine_bytes<D, GT>();
   constexpr size_t body = tile_region > combine_region ? tile_region : combine_region;
   uint8_t* kbuf = smem;
   uint8_t* vbuf = smem + kStages * TILE;
@@ -424,9 +449,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   }
 
   __syncthreads();  // pipeline finished: the tile region becomes the combine region
+  constexpr int R = combine_row<D>();
   float* cm = reinterpret_cast<float*>(smem);             // [warps][GT]
   float* cl = cm + kConsumerWarps * GT;                    // [warps][GT]
-  float* cacc = cl + kConsumerWarps * GT;                  // [warps][GT][D]
+  float* cacc = cl + kConsumerWarps * GT;                  // [warps][GT][R]
+  float* cf = cacc + kConsumerWarps * GT * R;              // [GT][warps + 1]
   if (warp < kConsumerWarps) {
     if ((lane % GROUP_LANES) == 0) {
       const int g = lane / GROUP_LANES;
@@ -436,10 +463,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
 #pragma unroll
     for (int g = 0; g < GT; ++g)
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) cacc[(warp * GT + g) * D + lane * DPL + e] = acc[g][e];
+      for (int e = 0; e < DPL; ++e) cacc[(warp * GT + g) * R + lane * DPL + e] = acc[g][e];
   }
   __syncthreads();
-  combine_and_store<D, GT>(cm, cl, cacc, p, seq, part, head0, nparts);
+  combine_and_store<D, GT>(cm, cl, cacc, cf, p, seq, part, head0, nparts);
   // let the merge kernel (launched as a programmatic dependent) get scheduled
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -468,7 +495,7 @@ template <typename CT, int kStages>
 constexpr size_t mma_smem_bytes() {
   constexpr size_t tile = size_t(kBlockSize) * 128 * CacheTraits<CT>::bytes;
   constexpr size_t pipe = 2 * kStages * tile;
-  constexpr size_t combine = size_t(kConsumerWarps) * 8 * (128 + 2) * sizeof(float);
+  constexpr size_t combine = combine_bytes<128, 8>();
   constexpr size_t body = pipe > combine ? pipe : combine;
   return 1024 + body + 2 * kStages * sizeof(uint64_t);
 }
@@ -487,7 +514,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   constexpr size_t tile_region = 2 * kStages * size_t(TILE);
-  constexpr size_t combine_region = size_t(kConsumerWarps) * GT * (D + 2) * sizeof(float);
+  constexpr size_t combine_region = combine_bytes<D, GT>();
   constexpr size_t body = tile_region > combine_region ? tile_region : combine_region;
   uint8_t* kbuf = smem;
   uint8_t* vbuf = smem + kStages * TILE;
@@ -762,9 +789,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
   }
 
   __syncthreads();  // pipeline finished: the tile region becomes the combine region
+  constexpr int R = combine_row<D>();
   float* cm = reinterpret_cast<float*>(smem);
   float* cl = cm + kConsumerWarps * GT;
   float* cacc = cl + kConsumerWarps * GT;
+  float* cf = cacc + kConsumerWarps * GT * R;
   if (warp < kConsumerWarps) {
     if (g == 0) {
       if (2 * c < GT) {
@@ -782,17 +811,17 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
       const int d0 = kFp8 ? 16 * t + 2 * g : 16 * t + g;
       const int d1 = kFp8 ? d0 + 1 : d0 + 8;
       if (2 * c < GT) {
-        cacc[(warp * GT + 2 * c) * D + d0] = acc[t][0];
-        cacc[(warp * GT + 2 * c) * D + d1] = acc[t][2];
+        cacc[(warp * GT + 2 * c) * R + d0] = acc[t][0];
+        cacc[(warp * GT + 2 * c) * R + d1] = acc[t][2];
       }
       if (2 * c + 1 < GT) {
-        cacc[(warp * GT + 2 * c + 1) * D + d0] = acc[t][1];
-        cacc[(warp * GT + 2 * c + 1) * D + d1] = acc[t][3];
+        cacc[(warp * GT + 2 * c + 1) * R + d0] = acc[t][1];
+        cacc[(warp * GT + 2 * c + 1) * R + d1] = acc[t][3];
       }
     }
   }
   __syncthreads();
-  combine_and_store<D, GT>(cm, cl, cacc, p, seq, part, head0, nparts);
+  combine_and_store<D, GT>(cm, cl, cacc, cf, p, seq, part, head0, nparts);
   // let the merge kernel (launched as a programmatic dependent) get scheduled
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
