@@ -69,6 +69,17 @@ def decode_bytes(wl: W.Workload, out_dtype: str) -> int:
     return kv + qo + tables
 
 
+def shared_decode_bytes(wl: W.Workload, out_dtype: str) -> int:
+    """Shared-prefix decode: each distinct K/V block once, plus Q, out, tables, lengths."""
+    cfg = wl.cfg
+    L = wl.seq_lens.numpy().astype(np.int64)
+    qo = len(L) * cfg.num_heads * cfg.head_dim * (W.ELT_BYTES[cfg.q_dtype] +
+                                                   W.ELT_BYTES[out_dtype])
+    tables = int(np.ceil(L / cfg.block_size).sum()) * 4 + 4 * len(L)
+    groups = 4 * (2 * wl.prefix_lens.numel() + 1)
+    return unique_kv_bytes(wl) + qo + tables + groups
+
+
 def unique_kv_bytes(wl: W.Workload) -> int:
     """K/V bytes of distinct physical blocks the decode reads (shared prefixes once)."""
     cfg = wl.cfg
@@ -270,7 +281,22 @@ def run_ours(args, rank, world, local_rank):
     reduce_runs = max_len > part_eff
     launches = 1 + 1 + (1 if reduce_runs else 0) + (1 if bm is not None else 0)
 
+    shared = wl.group_starts is not None and args.decode in ("auto", "shared")
+    if shared:
+        gs, pl = f(wl.group_starts), f(wl.prefix_lens)
+        max_group = int((wl.group_starts[1:] - wl.group_starts[:-1]).max())
+        launches -= 1 if reduce_runs else 0  # the shared-prefix decode needs no merge
     ev = []
+
+    def decode():
+        if shared:
+            pa.pa_paged_attention_decode_shared_prefix(
+                out, q, kc, vc, bt, sl, gs, pl, max_seq_len=max_len, max_group_size=max_group,
+                scale=wl.scale, k_scale=wl.k_scale, v_scale=wl.v_scale)
+        else:
+            pa.pa_paged_attention_decode(out, q, kc, vc, bt, sl, max_seq_len=max_len,
+                                         scale=wl.scale, k_scale=wl.k_scale, v_scale=wl.v_scale,
+                                         partition_size=part, workspace=ws)
 
     def step(timed: bool):
         if bm is not None:
@@ -280,9 +306,7 @@ def run_ours(args, rank, world, local_rank):
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        pa.pa_paged_attention_decode(out, q, kc, vc, bt, sl, max_seq_len=max_len, scale=wl.scale,
-                                     k_scale=wl.k_scale, v_scale=wl.v_scale,
-                                     partition_size=part, workspace=ws)
+        decode()
         if timed:
             e1.record(stream)
             ev.append((e0, e1))
@@ -316,7 +340,8 @@ def run_ours(args, rank, world, local_rank):
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error bits set during the timed steps")
 
-    step_bytes = decode_bytes(wl, out_dtype) + cache_write_bytes(wl) + copy_bytes(wl)
+    dec_b = shared_decode_bytes(wl, out_dtype) if shared else decode_bytes(wl, out_dtype)
+    step_bytes = dec_b + cache_write_bytes(wl) + copy_bytes(wl)
     ms_per_step = elapsed_ms / args.steps
     value = whole_job_gbs(step_bytes, world, args.steps, elapsed_ms)
 
@@ -357,7 +382,6 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
     peak, peak_kind = measured_peak()
-    dec_b = decode_bytes(wl, out_dtype)
     achieved = dec_b / (decode_ms * 1e-3) / 1e9
     traffic = recorded_traffic(args.config)
     L = wl.seq_lens.numpy().astype(np.int64)
@@ -375,7 +399,9 @@ def run_ours(args, rank, world, local_rank):
         "pct_of_peak": round(100.0 * value / peak, 2),
         "decode_tokens_per_s_per_layer": round(n_seqs * world / (ms_per_step * 1e-3), 1),
         "context_tokens_per_s_per_layer": round(int(L.sum()) * world / (ms_per_step * 1e-3), 1),
-        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (+ LSE reduce)",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("paged_attention_decode_shared_prefix" if shared else
+                                "paged_attention_decode (+ LSE reduce)"),
                      "achieved": round(achieved, 2), "peak": peak,
                      "peak_kind": f"{peak_kind} (hbm_gbs, copy burst)", "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -388,7 +414,11 @@ def run_ours(args, rank, world, local_rank):
         "clocks": sampler.summary() if sampler else None,
     }
     if wl.prefix_key is not None:
-        line["unique_kv_bytes_per_step"] = unique_kv_bytes(wl)
+        logical = decode_bytes(wl, out_dtype)
+        line["decode_bytes"] = {"distinct": dec_b if shared else shared_decode_bytes(wl, out_dtype),
+                                "per_sequence": logical,
+                                "per_sequence_gbs": round(logical / (decode_ms * 1e-3) / 1e9, 2)}
+        line["config"]["decode"] = "shared-prefix" if shared else "per-sequence"
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, out_dtype)
     return line
@@ -434,6 +464,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--decode", default="auto", choices=["auto", "shared", "standard"],
+                    help="copy-on-write workloads: shared-prefix decode (auto) or per sequence")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))

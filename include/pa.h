@@ -66,6 +66,7 @@ typedef enum {
 #define PA_DEVERR_SEQ_LEN 0x4u       /* decode: seq_len < 0, > max_seq_len or > table capacity */
 #define PA_DEVERR_PIPE_TIMEOUT 0x8u  /* decode: a pipeline wait gave up after ~1 s */
 #define PA_DEVERR_COPY_RANGE 0x10u   /* copy_blocks: block id outside [0, num_blocks) */
+#define PA_DEVERR_PREFIX 0x20u       /* shared-prefix decode: prefix_len or tables break the promise */
 
 /*
  * pa_reshape_and_cache -- write the new tokens' keys and values into their cache
@@ -155,6 +156,36 @@ int pa_paged_attention_decode(void* out, const void* query, const void* key_cach
                               pa_dtype cache_dtype, pa_dtype out_dtype, float k_scale,
                               float v_scale, int partition_size, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/*
+ * pa_paged_attention_decode_shared_prefix -- decode attention for groups of
+ * sequences whose block tables share their first blocks: the beams of one prompt,
+ * or parallel samples, after copy-on-write forking ("vLLM推理引擎PagedAttention原理
+ * 与性能优化实战" sec 3.2: sharers' block tables point at the same physical blocks;
+ * "vLLM 是什么…" sec 2: branches share the prompt's blocks).  The result is the
+ * same as pa_paged_attention_decode on the same arguments; each shared block is
+ * read from HBM, staged and widened once per group instead of once per sequence.
+ *
+ *   group_starts  [num_groups + 1] int32 (device): group g is the consecutive
+ *                 sequences group_starts[g] .. group_starts[g+1] - 1
+ *   prefix_lens   [num_groups] int32 (device): the group's shared prefix in tokens,
+ *                 a multiple of block_size, at most its shortest seq_len; every
+ *                 sequence of the group has the same block-table entries there
+ *   max_group_size  host-side bound on the group sizes (sizes the launch)
+ *   other arguments as for pa_paged_attention_decode (no partitions, no workspace)
+ * A broken promise (prefix not block-aligned or too long, tables differing in the
+ * prefix, a group larger than max_group_size) sets PA_DEVERR_PREFIX; the affected
+ * outputs are then unspecified, and nothing faults.
+ * Supported: block_size 16; head_dim 128; num_heads / num_kv_heads <= 16; the same
+ * dtype pairs as pa_paged_attention_decode.
+ */
+int pa_paged_attention_decode_shared_prefix(
+    void* out, const void* query, const void* key_cache, const void* value_cache,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+    int max_seq_len, const int32_t* group_starts, const int32_t* prefix_lens, int num_groups,
+    int max_group_size, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int64_t num_blocks, float scale, pa_dtype q_dtype, pa_dtype cache_dtype, pa_dtype out_dtype,
+    float k_scale, float v_scale, void* stream);
 
 /*
  * pa_copy_blocks -- the copy step of copy-on-write ("vLLM推理引擎PagedAttention原理

@@ -22,11 +22,12 @@ PA_F16, PA_BF16, PA_F32, PA_FP8_E4M3 = 0, 1, 2, 3
 STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED",
           -3: "PA_ERR_WORKSPACE", -4: "PA_ERR_CUDA"}
 DEVERR = {0x1: "SLOT_RANGE", 0x2: "BLOCK_RANGE", 0x4: "SEQ_LEN", 0x8: "PIPE_TIMEOUT",
-          0x10: "COPY_RANGE"}
+          0x10: "COPY_RANGE", 0x20: "PREFIX"}
 EXPORTS = ("pa_reshape_and_cache", "pa_paged_attention_workspace_size",
            "pa_paged_attention_partition_size",
            "pa_paged_attention_decode", "pa_copy_blocks", "pa_status_string",
-           "pa_get_device_error", "pa_paged_attention_decode_static_workspace")
+           "pa_get_device_error", "pa_paged_attention_decode_static_workspace",
+           "pa_paged_attention_decode_shared_prefix")
 PA_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 _DTYPE = {torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.float32: PA_F32,
@@ -69,6 +70,9 @@ def library() -> ctypes.CDLL:
             lib.pa_paged_attention_decode_static_workspace.argtypes = [
                 P, P, P, P, P, I, P, I, I, I, I, I, I, L, F, I, I, I, F, F, I, P]
             lib.pa_paged_attention_decode_static_workspace.restype = I
+            lib.pa_paged_attention_decode_shared_prefix.argtypes = [
+                P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, I, I, L, F, I, I, I, F, F, P]
+            lib.pa_paged_attention_decode_shared_prefix.restype = I
             lib.pa_copy_blocks.argtypes = [P, P, I, P, I, S, L, P]
             lib.pa_copy_blocks.restype = I
             lib.pa_status_string.argtypes = [I]
@@ -189,6 +193,38 @@ def pa_paged_attention_decode_static_workspace(out: torch.Tensor, query: torch.T
         raise PaError("pa_paged_attention_decode_static_workspace (needs more than the "
                       f"{PA_STATIC_WORKSPACE_BYTES} bytes of static scratch)", status)
     _check("pa_paged_attention_decode_static_workspace", status)
+
+
+def pa_paged_attention_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor,
+                                            key_cache: torch.Tensor, value_cache: torch.Tensor,
+                                            block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                                            group_starts: torch.Tensor,
+                                            prefix_lens: torch.Tensor, *, max_seq_len: int,
+                                            max_group_size: int, scale: float,
+                                            k_scale: float = 1.0, v_scale: float = 1.0,
+                                            stream=None) -> None:
+    """Decode for groups sharing the blocks of a prefix (beams, parallel samples).
+    group_starts [G + 1] int32, prefix_lens [G] int32 (tokens, block multiples)."""
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens"),
+                    (group_starts, "group_starts"), (prefix_lens, "prefix_lens")):
+        if t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+    b, h, d = query.shape
+    nb, hkv, bs, d2 = key_cache.shape
+    ng = prefix_lens.shape[0]
+    if out.shape != query.shape or d2 != d or value_cache.shape != key_cache.shape or \
+            block_tables.dim() != 2 or block_tables.shape[0] != b or seq_lens.shape != (b,) or \
+            group_starts.shape != (ng + 1,):
+        raise ValueError("shape mismatch")
+    _check("pa_paged_attention_decode_shared_prefix",
+           library().pa_paged_attention_decode_shared_prefix(
+               _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
+               _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+               block_tables.shape[1], _dev(seq_lens, "seq_lens"), b, int(max_seq_len),
+               _dev(group_starts, "group_starts"), _dev(prefix_lens, "prefix_lens"), ng,
+               int(max_group_size), h, hkv, d, bs, nb, float(scale), _dt(query, "query"),
+               _dt(key_cache, "key_cache"), _dt(out, "out"), float(k_scale), float(v_scale),
+               _stream(stream)))
 
 
 def pa_copy_blocks(key_caches: list, value_caches: list, block_mapping: torch.Tensor, *,

@@ -133,6 +133,65 @@ int pa_paged_attention_decode(void* out, const void* query, const void* key_cach
   return pa::launch_decode(a, static_cast<cudaStream_t>(stream));
 }
 
+int pa_paged_attention_decode_shared_prefix(
+    void* out, const void* query, const void* key_cache, const void* value_cache,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+    int max_seq_len, const int32_t* group_starts, const int32_t* prefix_lens, int num_groups,
+    int max_group_size, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int64_t num_blocks, float scale, pa_dtype q_dtype, pa_dtype cache_dtype, pa_dtype out_dtype,
+    float k_scale, float v_scale, void* stream) {
+  if (num_seqs < 0 || num_groups < 0 || max_group_size < 0 || max_seq_len < 0 ||
+      num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0 || max_blocks_per_seq < 0 || !valid_dtype(q_dtype) ||
+      !valid_dtype(cache_dtype) || !valid_dtype(out_dtype) || !isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (block_size != pa::kBlockSize || head_dim != 128 || num_heads / num_kv_heads > 16 ||
+      num_heads > 65535)
+    return PA_ERR_UNSUPPORTED;
+  if (out_dtype == PA_FP8_E4M3 || q_dtype == PA_FP8_E4M3 || q_dtype == PA_F32 ||
+      cache_dtype == PA_F32 || (cache_dtype != PA_FP8_E4M3 && cache_dtype != q_dtype))
+    return PA_ERR_UNSUPPORTED;
+  if (cache_dtype == PA_FP8_E4M3 &&
+      !(isfinite(k_scale) && k_scale > 0.f && isfinite(v_scale) && v_scale > 0.f))
+    return PA_ERR_INVALID_ARG;
+  if (int64_t(max_blocks_per_seq) * pa::kBlockSize < int64_t(max_seq_len))
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || num_groups == 0) return PA_OK;
+  if (max_group_size == 0) return PA_ERR_INVALID_ARG;
+  if (!out || !query || !key_cache || !value_cache || !seq_lens || !group_starts ||
+      !prefix_lens || (max_seq_len > 0 && !block_tables))
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(group_starts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(prefix_lens) & 3u))
+    return PA_ERR_INVALID_ARG;
+  pa::DecodeArgs a{};
+  a.out = out;
+  a.query = query;
+  a.key_cache = key_cache;
+  a.value_cache = value_cache;
+  a.block_tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.max_seq_len = max_seq_len;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.num_blocks = num_blocks;
+  a.scale = scale;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.q_dtype = q_dtype;
+  a.cache_dtype = cache_dtype;
+  a.out_dtype = out_dtype;
+  return pa::launch_decode_shared_prefix(a, group_starts, prefix_lens, num_groups, max_group_size,
+                                         static_cast<cudaStream_t>(stream));
+}
+
 int pa_copy_blocks(void* const* key_caches, void* const* value_caches, int num_layers,
                    const int64_t* block_mapping, int num_pairs, size_t block_bytes,
                    int64_t num_blocks, void* stream) {

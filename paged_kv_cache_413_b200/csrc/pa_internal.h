@@ -89,6 +89,11 @@ struct DecodeArgs {
 // PA_OK, PA_ERR_UNSUPPORTED (no kernel for the combination) or PA_ERR_CUDA.
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
+// Shared-prefix decode (groups of sequences sharing their first blocks).
+int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts,
+                                const int32_t* prefix_lens, int num_groups, int max_group_size,
+                                cudaStream_t stream);
+
 // Read and clear the device error words of the kernel files (synchronises stream).
 cudaError_t read_and_clear_cache_errors(unsigned* bits, cudaStream_t stream);
 cudaError_t read_and_clear_decode_errors(unsigned* bits, cudaStream_t stream);

@@ -157,6 +157,9 @@ class Workload:
     prefix_slot_mapping: torch.Tensor | None = None
     block_mapping: torch.Tensor | None = None   # [NP, 2] int64 (src, dst)
     refs: dict = field(default_factory=dict)
+    # sequences sharing the physical blocks of a prefix (copy-on-write groups)
+    group_starts: torch.Tensor | None = None    # [num_groups + 1] int32
+    prefix_lens: torch.Tensor | None = None     # [num_groups] int32, tokens
 
     @property
     def num_blocks(self) -> int:
@@ -312,6 +315,7 @@ def _make_beam_workload(cfg: DecodeConfig) -> Workload:
         k_scale = v_scale = 1.0
     kc = _fill_nan((nb, Hkv, bs, D), cfg.cache_dtype)
     vc = _fill_nan((nb, Hkv, bs, D), cfg.cache_dtype)
+    starts, prefixes = _shared_prefixes(tables, [W] * P, [L] * B, bs)
     return Workload(cfg=cfg, query=q, key_cache=kc, value_cache=vc,
                     block_tables=_table_tensor(tables, -(-L // bs)),
                     seq_lens=torch.full((B,), L, dtype=torch.int32),
@@ -323,4 +327,84 @@ def _make_beam_workload(cfg: DecodeConfig) -> Workload:
                     prefix_value=_to_storage(pv.reshape(P * S, Hkv, D), src),
                     prefix_slot_mapping=torch.from_numpy(prefix_slots),
                     block_mapping=torch.tensor(pairs, dtype=torch.int64).reshape(-1, 2),
-                    refs=dict(pool.refs))
+                    refs=dict(pool.refs), group_starts=starts, prefix_lens=prefixes)
+
+
+def _shared_prefixes(tables, group_sizes, lens, bs):
+    """group_starts and, per group, the tokens of the leading full blocks whose
+    block-table entries every member shares (what the block manager knows from
+    its forks)."""
+    starts, prefixes, s = [0], [], 0
+    for n in group_sizes:
+        members = tables[s:s + n]
+        full = min(int(L) for L in lens[s:s + n]) // bs
+        k = 0
+        while k < full and len({t[k] for t in members}) == 1:
+            k += 1
+        prefixes.append(k * bs)
+        s += n
+        starts.append(s)
+    return (torch.tensor(starts, dtype=torch.int32), torch.tensor(prefixes, dtype=torch.int32))
+
+
+def make_group_workload(num_groups: int, group_size: tuple, prefix_blocks: tuple,
+                        own_len: tuple, *, num_heads: int, num_kv_heads: int,
+                        head_dim: int = 128, dtype: str = "bf16", seed: int = 0,
+                        pool_factor: float = 1.3) -> Workload:
+    """Groups of sequences forked from a shared prompt prefix (16-bit caches).
+
+    Each group draws a size in ``group_size`` and a number of shared full blocks
+    in ``prefix_blocks`` (inclusive ranges); every member then owns
+    ``own_len`` tokens (at least 1: its last token is the new one) in blocks of
+    its own.  Draw order: group sizes, prefix blocks, own lengths, block
+    permutation, Q, K pool, V pool, new-token K, new-token V.
+    """
+    bs = BLOCK_SIZE
+    rng = np.random.default_rng(seed)
+    sizes = rng.integers(group_size[0], group_size[1] + 1, size=num_groups)
+    pblks = rng.integers(prefix_blocks[0], prefix_blocks[1] + 1, size=num_groups)
+    B = int(sizes.sum())
+    own = rng.integers(max(1, own_len[0]), own_len[1] + 1, size=B)
+    lens = np.concatenate([[pblks[g] * bs] * sizes[g] for g in range(num_groups)]).astype(np.int64) + own
+    need = int(pblks.sum()) + int(sum(-(-int(o) // bs) for o in own))
+    nb = max(1, math.ceil(pool_factor * need))
+    pool = BlockPool(rng.permutation(nb))
+    tables, i = [], 0
+    for g in range(num_groups):
+        shared = [pool.allocate() for _ in range(int(pblks[g]))]
+        for _ in range(int(sizes[g])):
+            tables.append(pool.fork(shared) + pool.allocate_for(int(own[i]), bs))
+            i += 1
+        for b in shared:
+            pool.refs[b] -= 1
+    Hkv, D = num_kv_heads, head_dim
+    q = _to_storage(_draw(rng, (B, num_heads, D), "normal"), dtype)
+    kpool = _draw(rng, (nb, Hkv, bs, D), "normal")
+    vpool = _draw(rng, (nb, Hkv, bs, D), "normal")
+    nk = _draw(rng, (B, Hkv, D), "normal")
+    nv = _draw(rng, (B, Hkv, D), "normal")
+    owned = np.zeros((nb, bs), dtype=bool)
+    slots = np.empty(B, dtype=np.int64)
+    for i, L in enumerate(lens):
+        L = int(L)
+        for j, b in enumerate(tables[i]):
+            owned[b, :min(bs, L - j * bs)] = True
+        s = _slot(tables[i], L - 1, bs)
+        slots[i] = s
+    for i, L in enumerate(lens):  # the new tokens' slots stay poisoned until written
+        s = int(slots[i])
+        owned[s // bs, s % bs] = False
+    for b in np.nonzero(~owned.all(axis=1))[0]:
+        kpool[b][:, ~owned[b], :] = np.nan
+        vpool[b][:, ~owned[b], :] = np.nan
+    cfg = DecodeConfig("groups", num_seqs=B, num_heads=num_heads, num_kv_heads=Hkv, head_dim=D,
+                       seq_lens=tuple(int(x) for x in lens), num_blocks=nb, q_dtype=dtype,
+                       cache_dtype=dtype, out_dtype=dtype, seed=seed)
+    starts, prefixes = _shared_prefixes(tables, [int(x) for x in sizes], lens, bs)
+    width = max(len(t) for t in tables)
+    return Workload(cfg=cfg, query=q, key_cache=_to_storage(kpool, dtype),
+                    value_cache=_to_storage(vpool, dtype), block_tables=_table_tensor(tables, width),
+                    seq_lens=torch.from_numpy(lens.astype(np.int32)),
+                    new_key=_to_storage(nk, dtype), new_value=_to_storage(nv, dtype),
+                    slot_mapping=torch.from_numpy(slots), scale=_scale(D), src_dtype=dtype,
+                    refs=dict(pool.refs), group_starts=starts, prefix_lens=prefixes)
