@@ -258,6 +258,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cfg = W.CONFIGS[args.config]
+    if args.block_size:
+        cfg = cfg.scaled(block_size=args.block_size)
     wl = W.make_workload(cfg, seed=cfg.seed + 1000 * rank) if rank else W.make_workload(cfg)
     out_dtype = cfg.out_dtype
     f = lambda t: None if t is None else t.to(dev)
@@ -392,6 +394,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "kv_dtype": cfg.cache_dtype, "data": "synthetic",
         "config": {"workload": f"{args.config}: {DESCR[args.config]}",
+                   "block_size": cfg.block_size,
                    "partition_tokens": part_eff, "out_dtype": out_dtype,
                    "l2": "no flush: inputs larger than L2 (%.2f GB read per step vs 126 MB L2)"
                          % (dec_b / 1e9),
@@ -464,6 +467,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--block-size", type=int, default=0,
+                    help="tokens per physical block (default: the workload's, 16)")
     ap.add_argument("--decode", default="auto", choices=["auto", "shared", "standard"],
                     help="copy-on-write workloads: shared-prefix decode (auto) or per sequence")
     ap.add_argument("--no-cpu-baseline", action="store_true")

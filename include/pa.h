@@ -84,7 +84,7 @@ typedef enum {
  *                     k_scale / v_scale, which must then be finite and > 0)
  * Two tokens naming the same slot give an unspecified winner.  A slot at or past
  * num_blocks * block_size is skipped and sets PA_DEVERR_SLOT_RANGE.
- * Supported: block_size 16; head_dim a multiple of 8 up to 256.
+ * Supported: block_size 16, 32, 64 or 128; head_dim a multiple of 8 up to 256.
  * num_tokens == 0 is a no-op returning PA_OK.
  */
 int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
@@ -96,8 +96,8 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
  * pa_paged_attention_workspace_size -- bytes of device workspace that
  * pa_paged_attention_decode needs for these sizes (0 when every sequence fits in
  * one partition, i.e. max_seq_len <= the partition size).
- * partition_size: 0 = the library's default, else a positive multiple of the
- * block size.  The default keeps a sequence whole when the batch has at least
+ * partition_size: 0 = the library's default, else a positive multiple of 16
+ * tokens.  The default keeps a sequence whole when the batch has at least
  * 2048 (sequence, head group) units, a head group being the largest of 8, 4, 2, 1
  * query heads dividing num_heads / num_kv_heads; otherwise it splits sequences
  * into enough partitions of at least 256 tokens to reach 2048 units.
@@ -141,11 +141,13 @@ int pa_paged_attention_partition_size(int num_seqs, int num_heads, int num_kv_he
  *   k_scale,
  *   v_scale       FP8 dequantisation scales; ignored for F16/BF16 caches
  *   partition_size  0 = default (see the size function), else a positive
- *                 multiple of block_size
+ *                 multiple of 16 tokens
  *   workspace     device buffer of at least pa_paged_attention_workspace_size()
  *                 bytes (may be NULL when that size is 0); contents on entry are
  *                 ignored, on exit unspecified
- * Supported: block_size 16; head_dim 64 or 128; num_heads % num_kv_heads == 0;
+ * Supported: block_size 16, 32, 64 or 128 (the kernels stream 16-token tiles, so a
+ * block is read as block_size / 16 contiguous tiles); head_dim 64 or 128;
+ * num_heads % num_kv_heads == 0;
  * (q_dtype, cache_dtype) in {(F16,F16), (BF16,BF16), (F16,FP8), (BF16,FP8)}.
  */
 int pa_paged_attention_decode(void* out, const void* query, const void* key_cache,
@@ -176,8 +178,8 @@ int pa_paged_attention_decode(void* out, const void* query, const void* key_cach
  * A broken promise (prefix not block-aligned or too long, tables differing in the
  * prefix, a group larger than max_group_size) sets PA_DEVERR_PREFIX; the affected
  * outputs are then unspecified, and nothing faults.
- * Supported: block_size 16; head_dim 128; num_heads / num_kv_heads <= 16; the same
- * dtype pairs as pa_paged_attention_decode.
+ * Supported: block_size 16, 32, 64 or 128; head_dim 128; num_heads / num_kv_heads
+ * <= 16; the same dtype pairs as pa_paged_attention_decode.
  */
 int pa_paged_attention_decode_shared_prefix(
     void* out, const void* query, const void* key_cache, const void* value_cache,
@@ -240,6 +242,33 @@ int pa_paged_attention_decode_static_workspace(
     int max_seq_len, int num_heads, int num_kv_heads, int head_dim, int block_size,
     int64_t num_blocks, float scale, pa_dtype q_dtype, pa_dtype cache_dtype, pa_dtype out_dtype,
     float k_scale, float v_scale, int partition_size, void* stream);
+
+/*
+ * pa_swap_blocks -- move whole blocks between two pools, e.g. out of GPU memory into
+ * page-locked host memory when the pool runs out, and back when a preempted
+ * sequence resumes ("vLLM 是什么…" sec 5, misconception 3: blocks are swapped to
+ * CPU memory, or requests preempted).  One launch moves every pair of every layer:
+ * the kernel reads and writes host memory through its device mapping, so scattered
+ * blocks cost no per-block copy call.
+ *
+ *   dst_key_caches, dst_value_caches,
+ *   src_key_caches, src_value_caches
+ *                  HOST arrays of num_layers pointers; each pool is device memory or
+ *                  page-locked host memory the device addresses at the same pointer
+ *                  (cudaHostAlloc / cudaMallocHost / torch pin_memory);
+ *                  [src_num_blocks or dst_num_blocks][block_bytes] bytes per layer
+ *   block_mapping  [num_pairs][2] int64 (src block, dst block), device memory or
+ *                  page-locked host memory
+ *   block_bytes    bytes of one block of one layer; a multiple of 16
+ * Pairs run concurrently: a dst must not repeat.  An id out of range skips the pair
+ * and sets PA_DEVERR_COPY_RANGE.  Pageable (unregistered) host memory is rejected
+ * with PA_ERR_INVALID_ARG.  num_pairs == 0 or num_layers == 0 is a no-op.
+ */
+int pa_swap_blocks(void* const* dst_key_caches, void* const* dst_value_caches,
+                   const void* const* src_key_caches, const void* const* src_value_caches,
+                   int num_layers, const int64_t* block_mapping, int num_pairs,
+                   size_t block_bytes, int64_t src_num_blocks, int64_t dst_num_blocks,
+                   void* stream);
 
 /* Human-readable name of a pa_status value (static storage). */
 const char* pa_status_string(int status);

@@ -15,6 +15,8 @@ What each function computes, and the passage it follows:
   ("vLLM 推理优化技术深度调研报告" sec 2, memory flow; "vLLM 是什么…" sec 2).
 * ``copy_blocks`` -- whole-block copies, the copy step of copy-on-write
   ("vLLM推理引擎PagedAttention原理与性能优化实战" sec 3.2).
+* ``swap_blocks`` -- whole-block moves between two pools (swapping to CPU memory,
+  "vLLM 是什么…" sec 5 misconception 3).
 * ``paged_attention_decode`` -- explicit gather through the block table, then
   textbook softmax(scale * q K^T) V ("vLLM 推理优化技术深度调研报告" sec 3
   formulas 3 and 4; dim. 1 sec 1 misconception 2).
@@ -76,6 +78,8 @@ def _load():
             lib.oracle_reshape_and_cache.restype = I
             lib.oracle_copy_blocks.argtypes = [P, P, I, P, L, L]
             lib.oracle_copy_blocks.restype = I
+            lib.oracle_swap_blocks.argtypes = [P, P, P, P, I, P, L, L, L, L]
+            lib.oracle_swap_blocks.restype = I
             lib.oracle_paged_attention_decode.argtypes = [
                 P, P, P, P, P, I, P, I, I, I, I, I, L, D, I, I, D, D]
             lib.oracle_paged_attention_decode.restype = I
@@ -207,6 +211,28 @@ def copy_blocks(key_caches, value_caches, block_mapping, *, dtype: str):
     if rc != 0:
         raise ValueError("oracle_copy_blocks rejected its arguments")
     return kcs, vcs
+
+
+def swap_blocks(dst_key_caches, dst_value_caches, src_key_caches, src_value_caches,
+                block_mapping, *, dtype: str):
+    """Return copies of the destination pools with every (src, dst) block moved in."""
+    dk = [_raw(x, dtype).copy() for x in dst_key_caches]
+    dv = [_raw(x, dtype).copy() for x in dst_value_caches]
+    sk = [_raw(x, dtype) for x in src_key_caches]
+    sv = [_raw(x, dtype) for x in src_value_caches]
+    bm = np.ascontiguousarray(np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2))
+    if not dk:
+        return dk, dv
+    block_bytes = dk[0].nbytes // dk[0].shape[0]
+    if sk[0].nbytes // sk[0].shape[0] != block_bytes:
+        raise ValueError("source and destination blocks differ in size")
+    arr = lambda xs: ctypes.cast((ctypes.c_void_p * len(xs))(*[_ptr(x) for x in xs]),
+                                 ctypes.c_void_p)
+    rc = _load().oracle_swap_blocks(arr(dk), arr(dv), arr(sk), arr(sv), len(dk), _ptr(bm),
+                                    bm.shape[0], block_bytes, sk[0].shape[0], dk[0].shape[0])
+    if rc != 0:
+        raise ValueError("oracle_swap_blocks rejected its arguments")
+    return dk, dv
 
 
 def _decode_args(query, key_cache, value_cache, block_tables, seq_lens, q_dtype, cache_dtype):

@@ -11,7 +11,8 @@
  *        sec 5.2 (FP8 KV cache).
  *   [P2] "vLLM 是什么：PagedAttention 让大模型推理快 2-4 倍，还能撑起更长思维链"
  *        sec 2 (logically contiguous, physically scattered blocks; a new block only
- *        when the current one is full).
+ *        when the current one is full), sec 5 misconception 3 (block swapping to
+ *        CPU memory when GPU memory runs out).
  *   [P3] "vLLM 推理优化技术深度调研报告"
  *        dim. 1 sec 1 misconception 2 (attention is the standard Softmax(QK^T/sqrt d)V),
  *        sec 3 formula 3 (logical -> physical page mapping through BlockTable[s]),
@@ -208,6 +209,30 @@ int oracle_copy_blocks(void* const* key_caches, void* const* value_caches, int n
              (size_t)block_bytes);
       memcpy((char*)value_caches[l] + dst * block_bytes,
              (char*)value_caches[l] + src * block_bytes, (size_t)block_bytes);
+    }
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * swap_blocks: whole blocks moved between two pools (device <-> host memory when
+ * GPU memory runs out: [P2] sec 5 misconception 3, block swapping to CPU memory):
+ * for each (src, dst) pair in order, block src of the source pool is copied to
+ * block dst of the destination pool, K and V, every layer.
+ * ------------------------------------------------------------------------- */
+int oracle_swap_blocks(void* const* dst_key_caches, void* const* dst_value_caches,
+                       void* const* src_key_caches, void* const* src_value_caches,
+                       int num_layers, const int64_t* block_mapping, int64_t num_pairs,
+                       int64_t block_bytes, int64_t src_num_blocks, int64_t dst_num_blocks) {
+  if (num_layers < 0 || num_pairs < 0 || block_bytes <= 0) return -1;
+  for (int64_t p = 0; p < num_pairs; ++p) {
+    int64_t src = block_mapping[2 * p], dst = block_mapping[2 * p + 1];
+    if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return -1;
+    for (int l = 0; l < num_layers; ++l) {
+      memcpy((char*)dst_key_caches[l] + dst * block_bytes,
+             (const char*)src_key_caches[l] + src * block_bytes, (size_t)block_bytes);
+      memcpy((char*)dst_value_caches[l] + dst * block_bytes,
+             (const char*)src_value_caches[l] + src * block_bytes, (size_t)block_bytes);
     }
   }
   return 0;

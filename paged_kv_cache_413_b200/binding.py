@@ -27,7 +27,7 @@ EXPORTS = ("pa_reshape_and_cache", "pa_paged_attention_workspace_size",
            "pa_paged_attention_partition_size",
            "pa_paged_attention_decode", "pa_copy_blocks", "pa_status_string",
            "pa_get_device_error", "pa_paged_attention_decode_static_workspace",
-           "pa_paged_attention_decode_shared_prefix")
+           "pa_paged_attention_decode_shared_prefix", "pa_swap_blocks")
 PA_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 _DTYPE = {torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.float32: PA_F32,
@@ -74,6 +74,8 @@ def library() -> ctypes.CDLL:
                 P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, I, I, L, F, I, I, I, F, F, P]
             lib.pa_paged_attention_decode_shared_prefix.restype = I
             lib.pa_copy_blocks.argtypes = [P, P, I, P, I, S, L, P]
+            lib.pa_swap_blocks.argtypes = [P, P, P, P, I, P, I, S, L, L, P]
+            lib.pa_swap_blocks.restype = I
             lib.pa_copy_blocks.restype = I
             lib.pa_status_string.argtypes = [I]
             lib.pa_status_string.restype = ctypes.c_char_p
@@ -248,6 +250,43 @@ def pa_copy_blocks(key_caches: list, value_caches: list, block_mapping: torch.Te
         ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), n,
         _dev(block_mapping, "block_mapping"), block_mapping.shape[0], block_bytes, nb,
         _stream(stream)))
+
+
+def _dev_or_pinned(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous tensor")
+    if t.device.type == "cuda" or (t.device.type == "cpu" and t.is_pinned()):
+        return t.data_ptr()
+    raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+
+
+def pa_swap_blocks(dst_key_caches: list, dst_value_caches: list, src_key_caches: list,
+                   src_value_caches: list, block_mapping: torch.Tensor, *, stream=None) -> None:
+    """Move blocks between pools (device <-> pinned host); block_mapping [NP, 2] int64."""
+    if block_mapping.dtype != torch.int64:
+        raise ValueError("block_mapping must be int64")
+    n = len(dst_key_caches)
+    if n == 0 or block_mapping.numel() == 0:
+        return
+    if not (len(dst_value_caches) == len(src_key_caches) == len(src_value_caches) == n):
+        raise ValueError("all four pool lists need one entry per layer")
+    d0, s0 = dst_key_caches[0], src_key_caches[0]
+    block_bytes = d0.numel() * d0.element_size() // d0.shape[0]
+    if s0.numel() * s0.element_size() // s0.shape[0] != block_bytes:
+        raise ValueError("source and destination blocks differ in size")
+    for c in list(dst_key_caches) + list(dst_value_caches):
+        if c.shape != d0.shape or c.dtype != d0.dtype:
+            raise ValueError("destination layers must share one shape and dtype")
+    for c in list(src_key_caches) + list(src_value_caches):
+        if c.shape != s0.shape or c.dtype != s0.dtype:
+            raise ValueError("source layers must share one shape and dtype")
+    arr = lambda xs, nm: ctypes.cast((ctypes.c_void_p * n)(*[_dev_or_pinned(c, nm) for c in xs]),
+                                     ctypes.c_void_p)
+    _check("pa_swap_blocks", library().pa_swap_blocks(
+        arr(dst_key_caches, "dst_key_caches[i]"), arr(dst_value_caches, "dst_value_caches[i]"),
+        arr(src_key_caches, "src_key_caches[i]"), arr(src_value_caches, "src_value_caches[i]"),
+        n, _dev_or_pinned(block_mapping, "block_mapping"), block_mapping.shape[0], block_bytes,
+        s0.shape[0], d0.shape[0], _stream(stream)))
 
 
 def pa_status_string(status: int) -> str:

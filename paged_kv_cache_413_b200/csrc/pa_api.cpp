@@ -30,7 +30,7 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
   if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
       num_blocks <= 0 || !valid_dtype(src_dtype) || !valid_dtype(cache_dtype))
     return PA_ERR_INVALID_ARG;
-  if (block_size != pa::kBlockSize || head_dim % 8 != 0 || head_dim > 256)
+  if (!pa::valid_block_size(block_size) || head_dim % 8 != 0 || head_dim > 256)
     return PA_ERR_UNSUPPORTED;
   if (src_dtype != PA_F16 && src_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
   const bool quant = cache_dtype == PA_FP8_E4M3;
@@ -44,7 +44,8 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
     return PA_ERR_INVALID_ARG;
   return cuda_status(pa::launch_reshape_and_cache(
       key, value, key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
-      num_blocks, src_dtype, cache_dtype, k_scale, v_scale, static_cast<cudaStream_t>(stream)));
+      block_size, num_blocks, src_dtype, cache_dtype, k_scale, v_scale,
+      static_cast<cudaStream_t>(stream)));
 }
 
 size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
@@ -81,7 +82,7 @@ int pa_paged_attention_decode(void* out, const void* query, const void* key_cach
     return PA_ERR_INVALID_ARG;
   if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
   if (partition_size % pa::kBlockSize != 0) return PA_ERR_INVALID_ARG;
-  if (block_size != pa::kBlockSize || (head_dim != 64 && head_dim != 128))
+  if (!pa::valid_block_size(block_size) || (head_dim != 64 && head_dim != 128))
     return PA_ERR_UNSUPPORTED;
   if (out_dtype == PA_FP8_E4M3 || q_dtype == PA_FP8_E4M3 || q_dtype == PA_F32)
     return PA_ERR_UNSUPPORTED;
@@ -90,7 +91,7 @@ int pa_paged_attention_decode(void* out, const void* query, const void* key_cach
   if (cache_dtype == PA_FP8_E4M3 &&
       !(isfinite(k_scale) && k_scale > 0.f && isfinite(v_scale) && v_scale > 0.f))
     return PA_ERR_INVALID_ARG;
-  if (int64_t(max_blocks_per_seq) * pa::kBlockSize < int64_t(max_seq_len))
+  if (int64_t(max_blocks_per_seq) * block_size < int64_t(max_seq_len))
     return PA_ERR_INVALID_ARG;  // the tables cannot hold the longest context
   if (num_seqs == 0) return PA_OK;
   if (!out || !query || !key_cache || !value_cache || !seq_lens ||
@@ -121,6 +122,7 @@ int pa_paged_attention_decode(void* out, const void* query, const void* key_cach
   a.num_heads = num_heads;
   a.num_kv_heads = num_kv_heads;
   a.head_dim = head_dim;
+  a.block_size = block_size;
   a.num_blocks = num_blocks;
   a.scale = scale;
   a.k_scale = k_scale;
@@ -146,7 +148,7 @@ int pa_paged_attention_decode_shared_prefix(
       !valid_dtype(cache_dtype) || !valid_dtype(out_dtype) || !isfinite(scale))
     return PA_ERR_INVALID_ARG;
   if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
-  if (block_size != pa::kBlockSize || head_dim != 128 || num_heads / num_kv_heads > 16 ||
+  if (!pa::valid_block_size(block_size) || head_dim != 128 || num_heads / num_kv_heads > 16 ||
       num_heads > 65535)
     return PA_ERR_UNSUPPORTED;
   if (out_dtype == PA_FP8_E4M3 || q_dtype == PA_FP8_E4M3 || q_dtype == PA_F32 ||
@@ -155,7 +157,7 @@ int pa_paged_attention_decode_shared_prefix(
   if (cache_dtype == PA_FP8_E4M3 &&
       !(isfinite(k_scale) && k_scale > 0.f && isfinite(v_scale) && v_scale > 0.f))
     return PA_ERR_INVALID_ARG;
-  if (int64_t(max_blocks_per_seq) * pa::kBlockSize < int64_t(max_seq_len))
+  if (int64_t(max_blocks_per_seq) * block_size < int64_t(max_seq_len))
     return PA_ERR_INVALID_ARG;
   if (num_seqs == 0 || num_groups == 0) return PA_OK;
   if (max_group_size == 0) return PA_ERR_INVALID_ARG;
@@ -181,6 +183,7 @@ int pa_paged_attention_decode_shared_prefix(
   a.num_heads = num_heads;
   a.num_kv_heads = num_kv_heads;
   a.head_dim = head_dim;
+  a.block_size = block_size;
   a.num_blocks = num_blocks;
   a.scale = scale;
   a.k_scale = k_scale;
@@ -208,6 +211,43 @@ int pa_copy_blocks(void* const* key_caches, void* const* value_caches, int num_l
   return cuda_status(pa::launch_copy_blocks(key_caches, value_caches, num_layers, block_mapping,
                                             num_pairs, block_bytes, num_blocks,
                                             static_cast<cudaStream_t>(stream)));
+}
+
+// Device memory, or page-locked host memory that the device can address directly
+// at the same pointer (all cudaHostAlloc / pinned allocations under unified addressing).
+static bool device_addressable(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return true;
+  return a.type == cudaMemoryTypeHost && a.devicePointer == p;
+}
+
+int pa_swap_blocks(void* const* dst_key_caches, void* const* dst_value_caches,
+                   const void* const* src_key_caches, const void* const* src_value_caches,
+                   int num_layers, const int64_t* block_mapping, int num_pairs,
+                   size_t block_bytes, int64_t src_num_blocks, int64_t dst_num_blocks,
+                   void* stream) {
+  if (num_layers < 0 || num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_layers == 0 || num_pairs == 0) return PA_OK;
+  if (!dst_key_caches || !dst_value_caches || !src_key_caches || !src_value_caches ||
+      !block_mapping || block_bytes == 0 || block_bytes % 16)
+    return PA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_mapping) & 7u) || !device_addressable(block_mapping))
+    return PA_ERR_INVALID_ARG;
+  for (int l = 0; l < num_layers; ++l) {
+    const void* ptrs[4] = {dst_key_caches[l], dst_value_caches[l], src_key_caches[l],
+                           src_value_caches[l]};
+    for (const void* q : ptrs)
+      if (!q || !aligned16(q) || !device_addressable(q)) return PA_ERR_INVALID_ARG;
+  }
+  return cuda_status(pa::launch_swap_blocks(dst_key_caches, dst_value_caches, src_key_caches,
+                                            src_value_caches, num_layers, block_mapping,
+                                            num_pairs, block_bytes, src_num_blocks,
+                                            dst_num_blocks, static_cast<cudaStream_t>(stream)));
 }
 
 const char* pa_status_string(int status) {

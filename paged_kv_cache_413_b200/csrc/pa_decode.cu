@@ -67,6 +67,8 @@ struct Params {
   float* ws_l;
   float* ws_o;
   int max_blocks_per_seq;
+  int block_size;       // tokens per physical block (a multiple of 16)
+  int tiles_per_block;  // block_size / 16
   int max_seq_len;
   int num_heads;
   int num_kv_heads;
@@ -279,11 +281,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
   const int blk_begin = part * (p.partition / kBlockSize);
   int32_t phys_first = 0;
-  if (warp == kConsumerWarps && blk_begin + lane < p.max_blocks_per_seq)
-    phys_first = table_row[blk_begin + lane];
+  if (warp == kConsumerWarps && (blk_begin + lane) / p.tiles_per_block < p.max_blocks_per_seq)
+    phys_first = table_row[(blk_begin + lane) / p.tiles_per_block];
   // Sequence length, range-checked against the launch bound and the table width.
   int L = p.seq_lens[seq];
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * kBlockSize);
+  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
   if (L < 0 || L > cap) {
     if (tid == 0 && part == 0 && blockIdx.y == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
     L = L < 0 ? 0 : cap;
@@ -314,24 +316,25 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
 
   if (warp == kConsumerWarps) {
     // ---------------- producer: block table -> bulk copies ----------------
-    const int32_t* table = table_row + blk_begin;
     const uint64_t policy = l2_policy_evict_first();
-    const size_t head_off = size_t(kvh) * TILE;
-    const size_t block_stride = size_t(p.num_kv_heads) * TILE;
     int issued = 0;
     bool ok = true;
     for (int base = 0; base < nblk && ok; base += 32) {
-      int32_t phys = 0;
+      // 16-token tile t of the sequence lives in block table_row[t / R] at sub-tile
+      // t % R; its index in the pool viewed as [blocks][kv_heads][R] tiles:
+      int tile = 0;
       if (base + lane < nblk) {
-        phys = base == 0 ? phys_first : table[base + lane];
+        const int t = blk_begin + base + lane, e = t / p.tiles_per_block;
+        int32_t phys = base == 0 ? phys_first : table_row[e];
         if (phys < 0 || phys >= p.num_blocks) {
           atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
           phys = 0;
         }
+        tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
       }
       const int cnt = min(32, nblk - base);
       for (int j = 0; j < cnt; ++j) {
-        const int32_t pb = __shfl_sync(kFullMask, phys, j);
+        const int tl = __shfl_sync(kFullMask, tile, j);
         const int i = base + j, stage = i % kStages;
         if (lane == 0) {
           if (i >= kStages && !mbar_wait_bounded(&empty[stage], ((i / kStages) - 1) & 1)) {
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
           }
           if (ok) {
             mbar_arrive_expect_tx(&full[stage], 2 * TILE);
-            const size_t off = size_t(pb) * block_stride + head_off;
+            const size_t off = size_t(tl) * TILE;
             bulk_copy_g2s(kbuf + stage * TILE, p.key_cache + off, TILE, &full[stage], policy);
             bulk_copy_g2s(vbuf + stage * TILE, p.value_cache + off, TILE, &full[stage], policy);
             ++issued;
@@ -531,10 +534,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
   const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
   const int blk_begin = part * (p.partition / kBlockSize);
   int32_t phys_first = 0;
-  if (warp == kConsumerWarps && blk_begin + lane < p.max_blocks_per_seq)
-    phys_first = table_row[blk_begin + lane];
+  if (warp == kConsumerWarps && (blk_begin + lane) / p.tiles_per_block < p.max_blocks_per_seq)
+    phys_first = table_row[(blk_begin + lane) / p.tiles_per_block];
   int L = p.seq_lens[seq];
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * kBlockSize);
+  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
   if (L < 0 || L > cap) {
     if (tid == 0 && part == 0 && blockIdx.y == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
     L = L < 0 ? 0 : cap;
@@ -567,22 +570,25 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
 
   if (warp == kConsumerWarps) {
     // ---------------- producer: block table -> tiled TMA loads ----------------
-    const int32_t* table = table_row + blk_begin;
     const uint64_t policy = l2_policy_evict_first();
     int issued = 0;
     bool ok = true;
     for (int base = 0; base < nblk && ok; base += 32) {
-      int32_t phys = 0;
+      // 16-token tile t of the sequence lives in block table_row[t / R] at sub-tile
+      // t % R; its index in the pool viewed as [blocks][kv_heads][R] tiles:
+      int tile = 0;
       if (base + lane < nblk) {
-        phys = base == 0 ? phys_first : table[base + lane];
+        const int t = blk_begin + base + lane, e = t / p.tiles_per_block;
+        int32_t phys = base == 0 ? phys_first : table_row[e];
         if (phys < 0 || phys >= p.num_blocks) {
           atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
           phys = 0;
         }
+        tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
       }
       const int cnt = min(32, nblk - base);
       for (int j = 0; j < cnt; ++j) {
-        const int32_t pb = __shfl_sync(kFullMask, phys, j);
+        const int tl = __shfl_sync(kFullMask, tile, j);
         const int i = base + j, stage = i % kStages;
         if (lane == 0) {
           if (i >= kStages && !mbar_wait_bounded(&empty[stage], ((i / kStages) - 1) & 1)) {
@@ -590,7 +596,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             ok = false;
           }
           if (ok) {
-            const int row = (pb * p.num_kv_heads + kvh) * kBlockSize;
+            const int row = tl * kBlockSize;
             uint8_t* kd = kbuf + stage * TILE;
             uint8_t* vd = vbuf + stage * TILE;
             mbar_arrive_expect_tx(&full[stage], 2 * TILE);
@@ -912,7 +918,7 @@ __global__ void __launch_bounds__(kThreads) decode_shared_prefix_kernel(
   if (nseq <= 0) return;
 
   // lengths of the CTA's sequences and the shared prefix (device data: checked)
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * kBlockSize);
+  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
   int Lmin = cap;
   int Ls[kSharedCols];
 #pragma unroll
@@ -926,9 +932,9 @@ __global__ void __launch_bounds__(kThreads) decode_shared_prefix_kernel(
     if (j < nseq) Lmin = min(Lmin, L);
   }
   int P = sp.prefix_lens[grp];
-  if (P < 0 || P % kBlockSize != 0 || P > Lmin) {
+  if (P < 0 || P % p.block_size != 0 || P > Lmin) {
     if (tid == 0 && sub == 0 && kvh == 0) atomicOr(&g_decode_err, PA_DEVERR_PREFIX);
-    P = P < 0 ? 0 : (min(P, Lmin) / kBlockSize) * kBlockSize;
+    P = P < 0 ? 0 : (min(P, Lmin) / p.block_size) * p.block_size;
   }
   const int pblk = P / kBlockSize;
   int ntotal = pblk;
@@ -971,22 +977,24 @@ __global__ void __launch_bounds__(kThreads) decode_shared_prefix_kernel(
       const int b0 = s_b0 + max(0, lo - gpos), b1 = s_b0 + min(s_b1 - s_b0, hi - gpos);
       gpos += s_b1 - s_b0;
       for (int base = b0; base < b1 && ok; base += 32) {
-        int32_t phys = 0;
+        int tile = 0;
         if (base + lane < b1) {
-          phys = row[base + lane];
+          const int t = base + lane, e = t / p.tiles_per_block;
+          int32_t phys = row[e];
           if (owner < 0) {  // the promise: every sequence of the group has these blocks
             for (int j = 1; j < nseq; ++j)
-              if (p.block_tables[int64_t(s0 + j) * p.max_blocks_per_seq + base + lane] != phys)
+              if (p.block_tables[int64_t(s0 + j) * p.max_blocks_per_seq + e] != phys)
                 atomicOr(&g_decode_err, PA_DEVERR_PREFIX);
           }
           if (phys < 0 || phys >= p.num_blocks) {
             atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
             phys = 0;
           }
+          tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
         }
         const int cnt = min(32, b1 - base);
         for (int jj = 0; jj < cnt; ++jj) {
-          const int32_t pb = __shfl_sync(kFullMask, phys, jj);
+          const int tl = __shfl_sync(kFullMask, tile, jj);
           const int i = issued, stage = i % kStages;
           if (lane == 0) {
             if (i >= kStages && !mbar_wait_bounded(&empty[stage], ((i / kStages) - 1) & 1)) {
@@ -996,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads) decode_shared_prefix_kernel(
             if (ok) {
               const int nvalid = min(kBlockSize, Lown - (base + jj) * kBlockSize);
               info[stage] = ((owner + 1) << 8) | nvalid;
-              const int trow = (pb * p.num_kv_heads + kvh) * kBlockSize;
+              const int trow = tl * kBlockSize;
               uint8_t* kd = kbuf + stage * TILE;
               uint8_t* vd = vbuf + stage * TILE;
               mbar_arrive_expect_tx(&full[stage], 2 * TILE);
@@ -1560,7 +1568,7 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
                                 const int32_t* prefix_lens, int num_groups, int max_group_size,
                                 cudaStream_t stream) {
   const int group = a.num_heads / a.num_kv_heads;
-  const int64_t rows = a.num_blocks * a.num_kv_heads * kBlockSize;
+  const int64_t rows = a.num_blocks * a.num_kv_heads * a.block_size;
   if (a.head_dim != 128 || group > kSharedCols || rows >= (int64_t(1) << 31) ||
       encode_fn() == nullptr)
     return PA_ERR_UNSUPPORTED;
@@ -1572,6 +1580,8 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
   p.block_tables = a.block_tables;
   p.seq_lens = a.seq_lens;
   p.max_blocks_per_seq = a.max_blocks_per_seq;
+  p.block_size = a.block_size;
+  p.tiles_per_block = a.block_size / kBlockSize;
   p.max_seq_len = a.max_seq_len;
   p.num_heads = a.num_heads;
   p.num_kv_heads = a.num_kv_heads;
@@ -1623,6 +1633,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.block_tables = a.block_tables;
   p.seq_lens = a.seq_lens;
   p.max_blocks_per_seq = a.max_blocks_per_seq;
+  p.block_size = a.block_size;
+  p.tiles_per_block = a.block_size / kBlockSize;
   p.max_seq_len = a.max_seq_len;
   p.num_heads = a.num_heads;
   p.num_kv_heads = a.num_kv_heads;
@@ -1642,7 +1654,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     p.ws_o = reinterpret_cast<float*>(w + a.ws.o_off);
   }
   int rc;
-  const int64_t rows = a.num_blocks * a.num_kv_heads * kBlockSize;
+  const int64_t rows = a.num_blocks * a.num_kv_heads * a.block_size;
   const bool use_mma = a.head_dim == 128 && (gt == 4 || gt == 8) && rows < (int64_t(1) << 31) &&
                        encode_fn() != nullptr;
   if (use_mma) {
@@ -1669,9 +1681,9 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   else
     rc = PA_ERR_UNSUPPORTED;
   if (rc != PA_OK || a.ws.max_parts <= 1) return rc;
-  const int cap = a.max_seq_len < a.max_blocks_per_seq * kBlockSize
+  const int cap = a.max_seq_len < a.max_blocks_per_seq * a.block_size
                       ? a.max_seq_len
-                      : a.max_blocks_per_seq * kBlockSize;
+                      : a.max_blocks_per_seq * a.block_size;
   const int out_rows = a.num_seqs * a.num_heads;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned((out_rows + 7) / 8));

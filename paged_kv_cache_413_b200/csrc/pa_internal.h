@@ -10,7 +10,10 @@
 
 namespace pa {
 
-constexpr int kBlockSize = 16;            // tokens per physical block
+constexpr int kBlockSize = 16;            // tokens per streamed tile (and the smallest block)
+
+// Physical block sizes the kernels take: multiples of the 16-token tile.
+inline bool valid_block_size(int bs) { return bs == 16 || bs == 32 || bs == 64 || bs == 128; }
 constexpr int kDefaultPartition = 512;     // tokens per split-K partition
 constexpr int kMaxLayersPerLaunch = 64;    // copy_blocks: layer pointers per launch
 
@@ -62,13 +65,20 @@ inline WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_di
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
                                      void* value_cache, const int64_t* slot_mapping,
                                      int num_tokens, int num_kv_heads, int head_dim,
-                                     int64_t num_blocks, pa_dtype src_dtype,
+                                     int block_size, int64_t num_blocks, pa_dtype src_dtype,
                                      pa_dtype cache_dtype, float k_scale, float v_scale,
                                      cudaStream_t stream);
 
 cudaError_t launch_copy_blocks(void* const* key_caches, void* const* value_caches,
                                int num_layers, const int64_t* block_mapping, int num_pairs,
                                size_t block_bytes, int64_t num_blocks, cudaStream_t stream);
+
+cudaError_t launch_swap_blocks(void* const* dst_key_caches, void* const* dst_value_caches,
+                               const void* const* src_key_caches,
+                               const void* const* src_value_caches, int num_layers,
+                               const int64_t* block_mapping, int num_pairs, size_t block_bytes,
+                               int64_t src_num_blocks, int64_t dst_num_blocks,
+                               cudaStream_t stream);
 
 struct DecodeArgs {
   void* out;
@@ -78,6 +88,7 @@ struct DecodeArgs {
   const int32_t* block_tables;
   const int32_t* seq_lens;
   int max_blocks_per_seq, num_seqs, max_seq_len, num_heads, num_kv_heads, head_dim;
+  int block_size;
   int64_t num_blocks;
   float scale, k_scale, v_scale;
   pa_dtype q_dtype, cache_dtype, out_dtype;

@@ -350,7 +350,7 @@ def _shared_prefixes(tables, group_sizes, lens, bs):
 def make_group_workload(num_groups: int, group_size: tuple, prefix_blocks: tuple,
                         own_len: tuple, *, num_heads: int, num_kv_heads: int,
                         head_dim: int = 128, dtype: str = "bf16", seed: int = 0,
-                        pool_factor: float = 1.3) -> Workload:
+                        pool_factor: float = 1.3, block_size: int = BLOCK_SIZE) -> Workload:
     """Groups of sequences forked from a shared prompt prefix (16-bit caches).
 
     Each group draws a size in ``group_size`` and a number of shared full blocks
@@ -359,7 +359,7 @@ def make_group_workload(num_groups: int, group_size: tuple, prefix_blocks: tuple
     its own.  Draw order: group sizes, prefix blocks, own lengths, block
     permutation, Q, K pool, V pool, new-token K, new-token V.
     """
-    bs = BLOCK_SIZE
+    bs = block_size
     rng = np.random.default_rng(seed)
     sizes = rng.integers(group_size[0], group_size[1] + 1, size=num_groups)
     pblks = rng.integers(prefix_blocks[0], prefix_blocks[1] + 1, size=num_groups)
@@ -399,7 +399,7 @@ def make_group_workload(num_groups: int, group_size: tuple, prefix_blocks: tuple
         vpool[b][:, ~owned[b], :] = np.nan
     cfg = DecodeConfig("groups", num_seqs=B, num_heads=num_heads, num_kv_heads=Hkv, head_dim=D,
                        seq_lens=tuple(int(x) for x in lens), num_blocks=nb, q_dtype=dtype,
-                       cache_dtype=dtype, out_dtype=dtype, seed=seed)
+                       cache_dtype=dtype, out_dtype=dtype, seed=seed, block_size=bs)
     starts, prefixes = _shared_prefixes(tables, [int(x) for x in sizes], lens, bs)
     width = max(len(t) for t in tables)
     return Workload(cfg=cfg, query=q, key_cache=_to_storage(kpool, dtype),

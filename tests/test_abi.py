@@ -81,8 +81,8 @@ def test_host_validation_without_gpu(lib):
     # reshape: bad sizes / unsupported block size / scale
     assert lib.pa_reshape_and_cache(nullp, nullp, nullp, nullp, nullp, 4, 0, 64, 16, 8, 0, 0,
                                     1.0, 1.0, nullp) == -1
-    assert lib.pa_reshape_and_cache(nullp, nullp, nullp, nullp, nullp, 4, 2, 64, 32, 8, 0, 0,
-                                    1.0, 1.0, nullp) == -2
+    assert lib.pa_reshape_and_cache(nullp, nullp, nullp, nullp, nullp, 4, 2, 64, 24, 8, 0, 0,
+                                    1.0, 1.0, nullp) == -2          # block size 24
     assert lib.pa_reshape_and_cache(nullp, nullp, nullp, nullp, nullp, 4, 2, 64, 16, 8, 1, 3,
                                     0.0, 1.0, nullp) == -1
     assert lib.pa_reshape_and_cache(nullp, nullp, nullp, nullp, nullp, 4, 2, 64, 16, 8, 0, 1,
@@ -105,7 +105,7 @@ def test_host_validation_without_gpu(lib):
 
     assert dec(h=6, hkv=4) == -1                 # heads not a multiple of kv heads
     assert dec(d=96) == -2                       # head_dim
-    assert dec(bs=32) == -2                      # block size
+    assert dec(bs=24) == -2                      # block size (16, 32, 64, 128 only)
     assert dec(qd=0, cd=1) == -2                 # f16 q with bf16 cache
     assert dec(od=3) == -2                       # fp8 output
     assert dec(part=24) == -1                    # partition not a multiple of 16

@@ -196,3 +196,23 @@ def test_full_beam_cow_fp8():
     prompts = [0, 37, 63]
     seqs = [p * 4 + w for p in prompts for w in range(4)]
     _check(wl, "bf16", wl.cfg.partition_size, seqs=seqs, prompts=prompts)
+
+
+@pytest.mark.parametrize("bs", [32, 64, 128])
+@pytest.mark.parametrize("name,over,part,out_dtype", [
+    ("llama2_7b", dict(num_seqs=5), 0, "f32"),
+    ("llama2_70b_gqa", dict(num_seqs=6), 48, "bf16"),
+    ("tiny", {}, 16, "f32"),
+])
+def test_block_sizes(bs, name, over, part, out_dtype):
+    """Blocks of 32, 64 and 128 tokens (read as 16-token tiles), partitions that
+    cut blocks in the middle included."""
+    wl = W.make_workload(name, block_size=bs, num_blocks=None, **over)
+    _check(wl, out_dtype, part)
+
+
+@pytest.mark.parametrize("bs", [32, 64])
+def test_block_sizes_fp8_beam(bs):
+    wl = W.make_workload("beam_cow_fp8", num_seqs=2, shared_len=bs * 3 + 5, block_size=bs,
+                         seed=bs)
+    _check(wl, "f32", 0)

@@ -109,3 +109,10 @@ def test_full_beam_cow_fp8_shared():
     prompts = [0, 21, 63]
     seqs = [p * 4 + w for p in prompts for w in range(4)]
     _check(wl, "bf16", seqs=seqs, prompts=prompts)
+
+
+@pytest.mark.parametrize("bs", [32, 64])
+def test_groups_block_sizes(bs):
+    wl = W.make_group_workload(5, (1, 6), (0, 3), (1, 90), num_heads=32, num_kv_heads=8,
+                               dtype="bf16", seed=bs, block_size=bs)
+    _check(wl, "f32")

@@ -167,3 +167,27 @@ def test_generated_new_token_slot_is_last_position():
             used[bt[i, pos // 16], pos % 16] = True
     assert not np.isnan(kc64.transpose(0, 2, 1, 3)[used]).any()
     assert np.isnan(kc64.transpose(0, 2, 1, 3)[~used]).all()
+
+
+def test_swap_blocks_moves_bytes_between_pools():
+    rng = np.random.default_rng(4)
+    gpu_k = [rng.integers(0, 255, (10, 2, 16, 8), dtype=np.uint8) for _ in range(2)]
+    gpu_v = [rng.integers(0, 255, (10, 2, 16, 8), dtype=np.uint8) for _ in range(2)]
+    cpu_k = [np.zeros((6, 2, 16, 8), dtype=np.uint8) for _ in range(2)]
+    cpu_v = [np.zeros((6, 2, 16, 8), dtype=np.uint8) for _ in range(2)]
+    pairs = np.array([[9, 0], [3, 5], [4, 1]], dtype=np.int64)  # gpu block -> cpu block
+    out_k, out_v = oracle.swap_blocks(cpu_k, cpu_v, gpu_k, gpu_v, pairs, dtype="e4m3")
+    for dst, src in list(zip(out_k, gpu_k)) + list(zip(out_v, gpu_v)):
+        assert np.array_equal(dst[0], src[9]) and np.array_equal(dst[5], src[3])
+        assert np.array_equal(dst[1], src[4])
+        assert not dst[[2, 3, 4]].any()
+    # and back into other gpu blocks
+    back_k, back_v = oracle.swap_blocks(gpu_k, gpu_v, out_k, out_v, [[0, 2], [5, 7]],
+                                        dtype="e4m3")
+    assert np.array_equal(back_k[1][2], gpu_k[1][9]) and np.array_equal(back_v[0][7], gpu_v[0][3])
+    try:
+        oracle.swap_blocks(cpu_k, cpu_v, gpu_k, gpu_v, [[10, 0]], dtype="e4m3")
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("out-of-range source block accepted")

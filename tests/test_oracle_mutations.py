@@ -30,6 +30,7 @@ MUTANTS = {
     "merge_unweighted": ("double w = lp * exp(m[r * max_parts + p] - M);", "double w = exp(m[r * max_parts + p] - M);"),
     "f16_subnormal": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
     "dequant_scale_dropped": ("        k *= k_scale;\n", "\n"),
+    "swap_wrong_pool": ("(const char*)src_key_caches[l] + src * block_bytes", "(const char*)dst_key_caches[l] + src * block_bytes"),
     "copy_wrong_direction": ("memcpy((char*)key_caches[l] + dst * block_bytes, (char*)key_caches[l] + src * block_bytes,",
                              "memcpy((char*)key_caches[l] + src * block_bytes, (char*)key_caches[l] + dst * block_bytes,"),
 }
