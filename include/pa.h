@@ -190,6 +190,33 @@ int pa_paged_attention_decode_shared_prefix(
     float k_scale, float v_scale, void* stream);
 
 /*
+ * pa_paged_attention_prefill -- several query tokens per sequence attending
+ * causally over the paged cache: a chunk of a long prompt processed between
+ * decode steps ("vLLM推理引擎PagedAttention原理与性能优化实战" sec 6, chunked
+ * prefill), or draft tokens checked in one pass.  The chunk's K/V are written by
+ * pa_reshape_and_cache first; seq_lens count them.
+ *
+ *   out, query    [total_queries][num_heads][head_dim]; sequence i's rows are
+ *                 query_start[i] .. query_start[i+1] - 1 (q_i rows)
+ *   query_start   [num_seqs + 1] int32 (device), non-decreasing, query_start[0] = 0
+ *   seq_lens      [num_seqs] int32: context lengths L_i including the chunk; row j of
+ *                 sequence i sits at position L_i - q_i + j and attends to positions
+ *                 0 .. L_i - q_i + j; q_i <= L_i (else PA_DEVERR_SEQ_LEN)
+ *   max_query_len host-side bound on q_i (sizes the launch)
+ *   other arguments as for pa_paged_attention_decode
+ * Supported: head_dim 128; (q_dtype, cache_dtype) (F16, F16) or (BF16, BF16); out
+ * F16, BF16 or F32; block_size 16, 32, 64 or 128.
+ */
+int pa_paged_attention_prefill(void* out, const void* query, const void* key_cache,
+                               const void* value_cache, const int32_t* block_tables,
+                               int max_blocks_per_seq, const int32_t* seq_lens,
+                               const int32_t* query_start, int num_seqs, int max_query_len,
+                               int max_seq_len, int num_heads, int num_kv_heads, int head_dim,
+                               int block_size, int64_t num_blocks, float scale,
+                               pa_dtype q_dtype, pa_dtype cache_dtype, pa_dtype out_dtype,
+                               void* stream);
+
+/*
  * pa_copy_blocks -- the copy step of copy-on-write ("vLLM推理引擎PagedAttention原理
  * 与性能优化实战" sec 3.2): when a block shared by several sequences (e.g. beams
  * with a common prefix) must be written by one of them, the block manager gives

@@ -20,6 +20,9 @@ What each function computes, and the passage it follows:
 * ``paged_attention_decode`` -- explicit gather through the block table, then
   textbook softmax(scale * q K^T) V ("vLLM 推理优化技术深度调研报告" sec 3
   formulas 3 and 4; dim. 1 sec 1 misconception 2).
+* ``paged_attention_prefill`` -- several query tokens per sequence, each attending
+  causally over the gathered context ("vLLM推理引擎PagedAttention原理与性能优化实战"
+  sec 6, chunked prefill).
 * ``decode_partition_stats`` / ``lse_merge`` -- the same definition applied to
   token ranges, and the log-sum-exp merge of those ranges.
 * ``e4m3_encode`` / ``e4m3_decode`` / ``f16_decode`` / ``bf16_decode`` -- the
@@ -83,6 +86,9 @@ def _load():
             lib.oracle_paged_attention_decode.argtypes = [
                 P, P, P, P, P, I, P, I, I, I, I, I, L, D, I, I, D, D]
             lib.oracle_paged_attention_decode.restype = I
+            lib.oracle_paged_attention_prefill.argtypes = [
+                P, P, P, P, P, I, P, P, I, I, I, I, I, L, D, I, I, D, D]
+            lib.oracle_paged_attention_prefill.restype = I
             lib.oracle_decode_partition_stats.argtypes = [
                 P, P, P, I, I, P, P, P, P, I, P, I, I, I, I, I, L, D, I, I, D, D]
             lib.oracle_decode_partition_stats.restype = I
@@ -263,6 +269,33 @@ def paged_attention_decode(query, key_cache, value_cache, block_tables, seq_lens
                                                float(v_scale))
     if rc != 0:
         raise ValueError("oracle_paged_attention_decode rejected its arguments")
+    return out
+
+
+def paged_attention_prefill(query, key_cache, value_cache, block_tables, seq_lens,
+                            query_start, *, scale: float, q_dtype: str, cache_dtype: str,
+                            k_scale: float = 1.0, v_scale: float = 1.0) -> np.ndarray:
+    """fp64 [total_queries, H, D]: causal multi-query attention over the paged cache."""
+    q = _raw(query, q_dtype)
+    kc = _raw(key_cache, cache_dtype)
+    vc = _raw(value_cache, cache_dtype)
+    bt = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    qs = np.ascontiguousarray(np.asarray(query_start, dtype=np.int32))
+    tq, h, d = q.shape
+    nb, hkv, bs, d2 = kc.shape
+    b = sl.shape[0]
+    if d2 != d or vc.shape != kc.shape or bt.shape[0] != b or qs.shape != (b + 1,) or \
+            qs[-1] != tq:
+        raise ValueError("shape mismatch")
+    out = np.zeros((tq, h, d), dtype=np.float64)
+    rc = _load().oracle_paged_attention_prefill(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(bt),
+                                                bt.shape[1], _ptr(sl), _ptr(qs), b, h, hkv, d,
+                                                bs, nb, float(scale), DTYPES[q_dtype],
+                                                DTYPES[cache_dtype], float(k_scale),
+                                                float(v_scale))
+    if rc != 0:
+        raise ValueError("oracle_paged_attention_prefill rejected its arguments")
     return out
 
 

@@ -8,7 +8,7 @@
  * Sources (page title, then the passage):
  *   [P1] "vLLM推理引擎PagedAttention原理与性能优化实战"
  *        sec 2.2 (16-token blocks, per-request block table), sec 3.2 (copy-on-write),
- *        sec 5.2 (FP8 KV cache).
+ *        sec 5.2 (FP8 KV cache), sec 6 (chunked prefill).
  *   [P2] "vLLM 是什么：PagedAttention 让大模型推理快 2-4 倍，还能撑起更长思维链"
  *        sec 2 (logically contiguous, physically scattered blocks; a new block only
  *        when the current one is full), sec 5 misconception 3 (block swapping to
@@ -344,6 +344,68 @@ int oracle_paged_attention_decode(double* out, const void* query, const void* ke
         int64_t qrow = ((int64_t)i * num_heads + h) * head_dim;
         for (int d = 0; d < head_dim; ++d) q[d] = load_elt(query, qrow + d, q_dtype);
         attend_rows(out + qrow, NULL, NULL, q, K, V, 0, L, head_dim, scale, sc);
+      }
+    }
+    free(K);
+    free(V);
+    free(sc);
+    free(q);
+  }
+  return failed ? -1 : 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Multi-query attention over the paged cache (chunked prefill, [P1] sec 6: a
+ * long prompt is processed in chunks interleaved with decode steps; several
+ * query tokens per sequence).  Sequence i has q_i = query_start[i+1] -
+ * query_start[i] query tokens, the last q_i positions of its context (their K/V
+ * already in the cache); query token j sits at position L_i - q_i + j and attends
+ * to positions 0 .. its own (causal).  Each query row is the textbook attention
+ * of attend_rows over that prefix of the gathered K, V.
+ * out: fp64 [total_queries][num_heads][head_dim].
+ * ------------------------------------------------------------------------- */
+int oracle_paged_attention_prefill(double* out, const void* query, const void* key_cache,
+                                   const void* value_cache, const int32_t* block_tables,
+                                   int max_blocks_per_seq, const int32_t* seq_lens,
+                                   const int32_t* query_start, int num_seqs, int num_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int64_t num_blocks, double scale, int q_dtype, int cache_dtype,
+                                   double k_scale, double v_scale) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+    return -1;
+  if (num_heads % num_kv_heads != 0) return -1;
+  if (!elt_size(q_dtype) || !elt_size(cache_dtype)) return -1;
+  int group = num_heads / num_kv_heads;
+  int failed = 0;
+  int64_t npairs = (int64_t)num_seqs * num_kv_heads;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
+  for (int64_t pr = 0; pr < npairs; ++pr) {
+    int i = (int)(pr / num_kv_heads), kvh = (int)(pr % num_kv_heads);
+    int L = seq_lens[i];
+    int q0 = query_start[i], nq = query_start[i + 1] - query_start[i];
+    if (L < 0 || nq < 0 || nq > L || (int64_t)L > (int64_t)max_blocks_per_seq * block_size) {
+      failed = 1;
+      continue;
+    }
+    int Lc = L > 0 ? L : 1;
+    double* K = (double*)malloc(sizeof(double) * (size_t)Lc * head_dim);
+    double* V = (double*)malloc(sizeof(double) * (size_t)Lc * head_dim);
+    double* sc = (double*)malloc(sizeof(double) * (size_t)Lc);
+    double* q = (double*)malloc(sizeof(double) * (size_t)head_dim);
+    if (!K || !V || !sc || !q ||
+        gather_kv(K, V, key_cache, value_cache, block_tables + (int64_t)i * max_blocks_per_seq,
+                  L, kvh, num_kv_heads, head_dim, block_size, num_blocks, cache_dtype, k_scale,
+                  v_scale) != 0) {
+      failed = 1;
+    } else {
+      for (int j = 0; j < nq; ++j) {
+        int pos = L - nq + j; /* this query token's position */
+        for (int g = 0; g < group; ++g) {
+          int h = kvh * group + g;
+          int64_t row = ((int64_t)(q0 + j) * num_heads + h) * head_dim;
+          for (int d = 0; d < head_dim; ++d) q[d] = load_elt(query, row + d, q_dtype);
+          attend_rows(out + row, NULL, NULL, q, K, V, 0, pos + 1, head_dim, scale, sc);
+        }
       }
     }
     free(K);

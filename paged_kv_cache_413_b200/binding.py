@@ -27,7 +27,8 @@ EXPORTS = ("pa_reshape_and_cache", "pa_paged_attention_workspace_size",
            "pa_paged_attention_partition_size",
            "pa_paged_attention_decode", "pa_copy_blocks", "pa_status_string",
            "pa_get_device_error", "pa_paged_attention_decode_static_workspace",
-           "pa_paged_attention_decode_shared_prefix", "pa_swap_blocks")
+           "pa_paged_attention_decode_shared_prefix", "pa_swap_blocks",
+           "pa_paged_attention_prefill")
 PA_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 _DTYPE = {torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.float32: PA_F32,
@@ -74,6 +75,9 @@ def library() -> ctypes.CDLL:
                 P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, I, I, L, F, I, I, I, F, F, P]
             lib.pa_paged_attention_decode_shared_prefix.restype = I
             lib.pa_copy_blocks.argtypes = [P, P, I, P, I, S, L, P]
+            lib.pa_paged_attention_prefill.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I,
+                                                       I, I, L, F, I, I, I, P]
+            lib.pa_paged_attention_prefill.restype = I
             lib.pa_swap_blocks.argtypes = [P, P, P, P, I, P, I, S, L, L, P]
             lib.pa_swap_blocks.restype = I
             lib.pa_copy_blocks.restype = I
@@ -227,6 +231,32 @@ def pa_paged_attention_decode_shared_prefix(out: torch.Tensor, query: torch.Tens
                int(max_group_size), h, hkv, d, bs, nb, float(scale), _dt(query, "query"),
                _dt(key_cache, "key_cache"), _dt(out, "out"), float(k_scale), float(v_scale),
                _stream(stream)))
+
+
+def pa_paged_attention_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                               value_cache: torch.Tensor, block_tables: torch.Tensor,
+                               seq_lens: torch.Tensor, query_start: torch.Tensor, *,
+                               max_query_len: int, max_seq_len: int, scale: float,
+                               stream=None) -> None:
+    """Causal multi-query attention (chunked prefill); query/out [total_q, H, D],
+    query_start [B + 1] int32."""
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens"),
+                    (query_start, "query_start")):
+        if t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+    tq, h, d = query.shape
+    nb, hkv, bs, d2 = key_cache.shape
+    b = seq_lens.shape[0]
+    if out.shape != query.shape or d2 != d or value_cache.shape != key_cache.shape or \
+            block_tables.dim() != 2 or block_tables.shape[0] != b or \
+            query_start.shape != (b + 1,):
+        raise ValueError("shape mismatch")
+    _check("pa_paged_attention_prefill", library().pa_paged_attention_prefill(
+        _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
+        _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+        block_tables.shape[1], _dev(seq_lens, "seq_lens"), _dev(query_start, "query_start"), b,
+        int(max_query_len), int(max_seq_len), h, hkv, d, bs, nb, float(scale),
+        _dt(query, "query"), _dt(key_cache, "key_cache"), _dt(out, "out"), _stream(stream)))
 
 
 def pa_copy_blocks(key_caches: list, value_caches: list, block_mapping: torch.Tensor, *,

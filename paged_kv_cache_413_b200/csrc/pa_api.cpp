@@ -195,6 +195,57 @@ int pa_paged_attention_decode_shared_prefix(
                                          static_cast<cudaStream_t>(stream));
 }
 
+int pa_paged_attention_prefill(void* out, const void* query, const void* key_cache,
+                               const void* value_cache, const int32_t* block_tables,
+                               int max_blocks_per_seq, const int32_t* seq_lens,
+                               const int32_t* query_start, int num_seqs, int max_query_len,
+                               int max_seq_len, int num_heads, int num_kv_heads, int head_dim,
+                               int block_size, int64_t num_blocks, float scale,
+                               pa_dtype q_dtype, pa_dtype cache_dtype, pa_dtype out_dtype,
+                               void* stream) {
+  if (num_seqs < 0 || max_query_len < 0 || max_seq_len < 0 || num_heads <= 0 ||
+      num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq < 0 || !valid_dtype(q_dtype) || !valid_dtype(cache_dtype) ||
+      !valid_dtype(out_dtype) || !isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (!pa::valid_block_size(block_size) || head_dim != 128 || num_heads > 65535 ||
+      (q_dtype != PA_F16 && q_dtype != PA_BF16) || cache_dtype != q_dtype ||
+      out_dtype == PA_FP8_E4M3)
+    return PA_ERR_UNSUPPORTED;
+  if (int64_t(max_blocks_per_seq) * block_size < int64_t(max_seq_len) ||
+      max_query_len > max_seq_len)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !seq_lens || !query_start || !block_tables)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(query_start) & 3u))
+    return PA_ERR_INVALID_ARG;
+  pa::DecodeArgs a{};
+  a.out = out;
+  a.query = query;
+  a.key_cache = key_cache;
+  a.value_cache = value_cache;
+  a.block_tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.max_seq_len = max_seq_len;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.scale = scale;
+  a.q_dtype = q_dtype;
+  a.cache_dtype = cache_dtype;
+  a.out_dtype = out_dtype;
+  return pa::launch_prefill(a, query_start, max_query_len, static_cast<cudaStream_t>(stream));
+}
+
 int pa_copy_blocks(void* const* key_caches, void* const* value_caches, int num_layers,
                    const int64_t* block_mapping, int num_pairs, size_t block_bytes,
                    int64_t num_blocks, void* stream) {

@@ -93,6 +93,13 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_s
       : "memory");
 }
 
+// L2 policy for data other CTAs will read again soon: evict last.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // L2 policy for data read exactly once (streamed K/V): evict first.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;

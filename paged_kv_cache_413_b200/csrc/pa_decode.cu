@@ -1370,6 +1370,282 @@ __global__ void __launch_bounds__(kThreads) decode_shared_prefix_kernel(
   cluster_sync();  // keep every CTA's shared memory alive until all reads are done
 }
 
+// ---------------------------------------------------------------------------
+// Multi-query attention over the paged cache (chunked prefill: several query
+// tokens per sequence, each attending causally; "vLLM推理引擎PagedAttention原理与
+// 性能优化实战" sec 6).  Sequence i's query rows are query_start[i] .. [i+1] - 1;
+// row j sits at position L - q + j.  One CTA serves 64 (query token, head) rows of
+// one kv head: row r is token r / G, head r % G of the group.  Each of the four
+// consumer warps owns 16 rows for the whole pass (FlashAttention-2 layout over
+// paged tiles): S = Q K^T and O += P V as mma.sync m16n8k16 per 16-token tile, P
+// going straight from the S accumulator into the A operand, fp32 online softmax
+// per row, causal and context masks.  Every staged tile is read by all four warps.
+// ---------------------------------------------------------------------------
+struct PrefillParams {
+  CUtensorMap tmk;
+  CUtensorMap tmv;
+  Params p;
+  const int32_t* query_start;  // [num_seqs + 1]
+  int row_blocks;              // CTAs per (sequence, kv head): ceil(max rows / 64)
+};
+
+constexpr int kPrefillRows = kConsumerWarps * 16;
+
+template <typename CT, int kStages>
+constexpr size_t prefill_smem_bytes() {
+  return 1024 + 2 * kStages * size_t(kBlockSize) * 128 * CacheTraits<CT>::bytes +
+         2 * kStages * sizeof(uint64_t);
+}
+
+template <typename CT, int kStages>
+__global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant__ PrefillParams pp) {
+  constexpr int D = 128;
+  constexpr int TILE = kBlockSize * D * CacheTraits<CT>::bytes;
+  static_assert(CacheTraits<CT>::bytes == 2, "16-bit caches");
+  using MT = CT;
+  constexpr bool kSplitP = std::is_same<MT, __nv_bfloat16>::value;
+  const Params& p = pp.p;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* kbuf = smem;
+  uint8_t* vbuf = smem + kStages * TILE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * kStages * TILE);
+  uint64_t* empty = full + kStages;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int seq = blockIdx.x / pp.row_blocks;
+  const int rblk = blockIdx.x - seq * pp.row_blocks;
+  const int kvh = blockIdx.y;
+  const int G = p.group;
+  const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
+
+  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+  int L = p.seq_lens[seq];
+  const int q0 = pp.query_start[seq];
+  int nq = pp.query_start[seq + 1] - q0;
+  if (L < 0 || L > cap || nq < 0 || nq > L) {
+    if (tid == 0 && rblk == 0 && kvh == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
+    L = L < 0 ? 0 : (L > cap ? cap : L);
+    nq = nq < 0 ? 0 : (nq > L ? L : nq);
+  }
+  const int rows = nq * G;
+  const int row0 = rblk * kPrefillRows;
+  if (row0 >= rows) return;
+  // positions: row r -> token r / G at L - nq + r / G; tiles up to the CTA's last row
+  const int pos_last = L - nq + (min(rows, row0 + kPrefillRows) - 1) / G;
+  const int nblk = pos_last / kBlockSize + 1;
+
+  if (tid == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kConsumerWarps);  // every consumer warp reads every tile
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int g = lane >> 2, c = lane & 3;
+  const int mi = lane >> 3, r = lane & 7;
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: tiles 0 .. nblk-1 of the sequence ----------------
+    const uint64_t policy = l2_policy_evict_last();  // re-read by the other row blocks
+    int issued = 0;
+    bool ok = true;
+    for (int base = 0; base < nblk && ok; base += 32) {
+      int tile = 0;
+      if (base + lane < nblk) {
+        const int t = base + lane, e = t / p.tiles_per_block;
+        int32_t phys = table_row[e];
+        if (phys < 0 || phys >= p.num_blocks) {
+          atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
+          phys = 0;
+        }
+        tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
+      }
+      const int cnt = min(32, nblk - base);
+      for (int j = 0; j < cnt; ++j) {
+        const int tl = __shfl_sync(kFullMask, tile, j);
+        const int i = base + j, stage = i % kStages;
+        if (lane == 0) {
+          if (i >= kStages && !mbar_wait_bounded(&empty[stage], ((i / kStages) - 1) & 1)) {
+            atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+            ok = false;
+          }
+          if (ok) {
+            const int row = tl * kBlockSize;
+            uint8_t* kd = kbuf + stage * TILE;
+            uint8_t* vd = vbuf + stage * TILE;
+            mbar_arrive_expect_tx(&full[stage], 2 * TILE);
+            tma_load_2d(kd, &pp.tmk, 0, row, &full[stage], policy);
+            tma_load_2d(kd + TILE / 2, &pp.tmk, 64, row, &full[stage], policy);
+            tma_load_2d(vd, &pp.tmv, 0, row, &full[stage], policy);
+            tma_load_2d(vd + TILE / 2, &pp.tmv, 64, row, &full[stage], policy);
+            ++issued;
+          }
+        }
+        ok = __shfl_sync(kFullMask, ok, 0);
+        if (!ok) break;
+      }
+    }
+    if (lane == 0) {
+      const int first = issued > kStages ? issued - kStages : 0;
+      for (int i = first; i < issued; ++i)
+        if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1))
+          atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+    }
+    return;
+  }
+
+  // ---------------- consumers: 16 rows per warp ----------------
+  const int ra = row0 + warp * 16 + g, rb = ra + 8;  // this thread's two rows
+  const bool va = ra < rows, vb = rb < rows;
+  const int pa_pos = L - nq + ra / G, pb_pos = L - nq + rb / G;
+  const int wlast = min(rows, row0 + warp * 16 + 16) - 1;  // the warp's last row
+  const int wpos = wlast >= row0 + warp * 16 ? L - nq + wlast / G : -1;
+  auto qrow = [&](int rr) {
+    return p.query + (int64_t(q0 + rr / G) * p.num_heads + kvh * G + rr % G) * D * 2;
+  };
+  uint32_t qa[8][4];
+  {
+    const uint8_t* ya = qrow(va ? ra : row0);
+    const uint8_t* yb = qrow(vb ? rb : row0);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qa[ks][0] = va ? *reinterpret_cast<const uint32_t*>(ya + (16 * ks + 2 * c) * 2) : 0u;
+      qa[ks][1] = vb ? *reinterpret_cast<const uint32_t*>(yb + (16 * ks + 2 * c) * 2) : 0u;
+      qa[ks][2] = va ? *reinterpret_cast<const uint32_t*>(ya + (16 * ks + 2 * c + 8) * 2) : 0u;
+      qa[ks][3] = vb ? *reinterpret_cast<const uint32_t*>(yb + (16 * ks + 2 * c + 8) * 2) : 0u;
+    }
+  }
+  const float mult = p.q_mult;
+  float acc[16][4];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+
+  for (int i = 0; i < nblk; ++i) {
+    const int stage = i % kStages;
+    if (!__all_sync(kFullMask, mbar_wait_bounded(&full[stage], (i / kStages) & 1))) {
+      if (lane == 0) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+      break;
+    }
+    if (i * kBlockSize <= wpos) {  // some row of this warp sees part of this tile
+      const uint32_t kt = smem_u32(kbuf + stage * TILE);
+      const uint32_t vt = smem_u32(vbuf + stage * TILE);
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int tok = r + 8 * (mi >> 1), j = 2 * ks + (mi & 1);
+        uint32_t b[4];
+        ldsm_x4(kt + (j >> 3) * (TILE / 2) + tok * 128 + (((j & 7) ^ r) << 4), b);
+        mma_16816(sc[0], qa[ks], b[0], b[1], MT{});
+        mma_16816(sc[1], qa[ks], b[2], b[3], MT{});
+      }
+      // causal and context masks: token position tp is visible to a row at pos if tp <= pos
+      float mxa = -INFINITY, mxb = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tp = i * kBlockSize + nt * 8 + 2 * c + e;
+          sc[nt][e] = (va && tp <= pa_pos) ? sc[nt][e] * mult : -INFINITY;
+          sc[nt][2 + e] = (vb && tp <= pb_pos) ? sc[nt][2 + e] * mult : -INFINITY;
+          mxa = fmaxf(mxa, sc[nt][e]);
+          mxb = fmaxf(mxb, sc[nt][2 + e]);
+        }
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        mxa = fmaxf(mxa, __shfl_xor_sync(kFullMask, mxa, o));
+        mxb = fmaxf(mxb, __shfl_xor_sync(kFullMask, mxb, o));
+      }
+      const float mna = fmaxf(ma, mxa), mnb = fmaxf(mb, mxb);
+      const float ala = mna == -INFINITY ? 1.f : exp2f(ma - mna);
+      const float alb = mnb == -INFINITY ? 1.f : exp2f(mb - mnb);
+      ma = mna;
+      mb = mnb;
+      float pr[2][4];
+      float suma = 0.f, sumb = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          pr[nt][e] = mna == -INFINITY ? 0.f : exp2f(sc[nt][e] - mna);
+          pr[nt][2 + e] = mnb == -INFINITY ? 0.f : exp2f(sc[nt][2 + e] - mnb);
+          suma += pr[nt][e];
+          sumb += pr[nt][2 + e];
+        }
+      la = la * ala + suma;
+      lb = lb * alb + sumb;
+      // P as the A operand (rows x 16 tokens): the S accumulator layout, repacked
+      uint32_t ph[4] = {pack2(pr[0][0], pr[0][1], MT{}), pack2(pr[0][2], pr[0][3], MT{}),
+                        pack2(pr[1][0], pr[1][1], MT{}), pack2(pr[1][2], pr[1][3], MT{})};
+      uint32_t pl[4] = {0u, 0u, 0u, 0u};
+      if constexpr (kSplitP) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int nt = q >> 1, hr = (q & 1) * 2;
+          const float2 h = unpack2(ph[q], MT{});
+          pl[q] = pack2(pr[nt][hr] - h.x, pr[nt][hr + 1] - h.y, MT{});
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        acc[t][0] *= ala;
+        acc[t][1] *= ala;
+        acc[t][2] *= alb;
+        acc[t][3] *= alb;
+      }
+      // V rows past the context may hold anything (NaN): zero them in the B operand
+      const int nvalid = min(kBlockSize, L - i * kBlockSize);
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (nvalid < kBlockSize) {
+        mlo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+        mhi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+      }
+#pragma unroll
+      for (int dt = 0; dt < 8; ++dt) {
+        const int tok = r + 8 * (mi & 1), j = 2 * dt + (mi >> 1);
+        uint32_t b[4];
+        ldsm_x4_trans(vt + (j >> 3) * (TILE / 2) + tok * 128 + (((j & 7) ^ r) << 4), b);
+        b[0] &= mlo;
+        b[1] &= mhi;
+        b[2] &= mlo;
+        b[3] &= mhi;
+        mma_16816(acc[2 * dt], ph, b[0], b[1], MT{});
+        mma_16816(acc[2 * dt + 1], ph, b[2], b[3], MT{});
+        if constexpr (kSplitP) {
+          mma_16816(acc[2 * dt], pl, b[0], b[1], MT{});
+          mma_16816(acc[2 * dt + 1], pl, b[2], b[3], MT{});
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+  }
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    la += __shfl_xor_sync(kFullMask, la, o);
+    lb += __shfl_xor_sync(kFullMask, lb, o);
+  }
+  const float ia = la > 0.f ? p.v_mult / la : 0.f, ib = lb > 0.f ? p.v_mult / lb : 0.f;
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    const int d = 8 * t + 2 * c;
+    if (va) {
+      const int64_t o = (int64_t(q0 + ra / G) * p.num_heads + kvh * G + ra % G) * D + d;
+      store_out(p.out, o, acc[t][0] * ia, p.out_dtype);
+      store_out(p.out, o + 1, acc[t][1] * ia, p.out_dtype);
+    }
+    if (vb) {
+      const int64_t o = (int64_t(q0 + rb / G) * p.num_heads + kvh * G + rb % G) * D + d;
+      store_out(p.out, o, acc[t][2] * ib, p.out_dtype);
+      store_out(p.out, o + 1, acc[t][3] * ib, p.out_dtype);
+    }
+  }
+}
+
 // Log-sum-exp merge of the partitions of sequences with more than one:
 // M = max m_p, w_p = l_p exp(m_p - M), out = sum w_p o_p / sum w_p.
 // One warp per (sequence, head) row, 8 rows per CTA; lanes own D/32 dims.
@@ -1620,6 +1896,60 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
   if (fp8 && a.q_dtype == PA_BF16)
     return launch_shared_typed<fp8_e4m3, __nv_bfloat16>(sp, int(grid_x), stream);
   return PA_ERR_UNSUPPORTED;
+}
+
+int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_query_len,
+                   cudaStream_t stream) {
+  const int group = a.num_heads / a.num_kv_heads;
+  const int64_t rows = a.num_blocks * a.num_kv_heads * a.block_size;
+  if (a.head_dim != 128 || a.cache_dtype == PA_FP8_E4M3 || a.cache_dtype != a.q_dtype ||
+      rows >= (int64_t(1) << 31) || encode_fn() == nullptr)
+    return PA_ERR_UNSUPPORTED;
+  PrefillParams pp;
+  memset(&pp, 0, sizeof pp);
+  Params& p = pp.p;
+  p.out = a.out;
+  p.query = static_cast<const uint8_t*>(a.query);
+  p.block_tables = a.block_tables;
+  p.seq_lens = a.seq_lens;
+  p.max_blocks_per_seq = a.max_blocks_per_seq;
+  p.block_size = a.block_size;
+  p.tiles_per_block = a.block_size / kBlockSize;
+  p.max_seq_len = a.max_seq_len;
+  p.num_heads = a.num_heads;
+  p.num_kv_heads = a.num_kv_heads;
+  p.group = group;
+  p.out_dtype = a.out_dtype;
+  p.num_blocks = a.num_blocks;
+  p.q_mult = a.scale * kLog2e;
+  p.v_mult = 1.f;
+  pp.query_start = query_start;
+  pp.row_blocks = int((int64_t(max_query_len) * group + kPrefillRows - 1) / kPrefillRows);
+  const int64_t grid_x = int64_t(a.num_seqs) * pp.row_blocks;
+  if (pp.row_blocks == 0) return PA_OK;
+  if (grid_x > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (!encode_pool_map(&pp.tmk, a.key_cache, rows, false) ||
+      !encode_pool_map(&pp.tmv, a.value_cache, rows, false))
+    return PA_ERR_CUDA;
+  constexpr int stages = 4;
+  auto run = [&](auto kern, size_t smem, unsigned long long& mask) -> int {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(mask & bit)) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+          cudaSuccess)
+        return PA_ERR_CUDA;
+      mask |= bit;
+    }
+    kern<<<dim3(unsigned(grid_x), unsigned(a.num_kv_heads)), kThreads, smem, stream>>>(pp);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  };
+  static unsigned long long mask_h = 0, mask_b = 0;
+  if (a.cache_dtype == PA_F16)
+    return run(prefill_kernel<__half, stages>, prefill_smem_bytes<__half, stages>(), mask_h);
+  return run(prefill_kernel<__nv_bfloat16, stages>, prefill_smem_bytes<__nv_bfloat16, stages>(),
+             mask_b);
 }
 
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {

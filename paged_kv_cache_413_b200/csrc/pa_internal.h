@@ -100,6 +100,10 @@ struct DecodeArgs {
 // PA_OK, PA_ERR_UNSUPPORTED (no kernel for the combination) or PA_ERR_CUDA.
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
+// Multi-query (chunked prefill) attention.
+int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_query_len,
+                   cudaStream_t stream);
+
 // Shared-prefix decode (groups of sequences sharing their first blocks).
 int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts,
                                 const int32_t* prefix_lens, int num_groups, int max_group_size,

@@ -160,6 +160,9 @@ class Workload:
     # sequences sharing the physical blocks of a prefix (copy-on-write groups)
     group_starts: torch.Tensor | None = None    # [num_groups + 1] int32
     prefix_lens: torch.Tensor | None = None     # [num_groups] int32, tokens
+    # several query tokens per sequence (chunked prefill): query is then
+    # [total_queries, H, D] and sequence i's rows are query_start[i] .. query_start[i+1]-1
+    query_start: torch.Tensor | None = None     # [num_seqs + 1] int32
 
     @property
     def num_blocks(self) -> int:
@@ -408,3 +411,55 @@ def make_group_workload(num_groups: int, group_size: tuple, prefix_blocks: tuple
                     new_key=_to_storage(nk, dtype), new_value=_to_storage(nv, dtype),
                     slot_mapping=torch.from_numpy(slots), scale=_scale(D), src_dtype=dtype,
                     refs=dict(pool.refs), group_starts=starts, prefix_lens=prefixes)
+
+
+def make_prefill_workload(num_seqs: int, context: tuple, chunk: tuple, *, num_heads: int,
+                          num_kv_heads: int, head_dim: int = 128, dtype: str = "bf16",
+                          seed: int = 0, block_size: int = BLOCK_SIZE,
+                          pool_factor: float = 1.1) -> Workload:
+    """Chunked prefill: sequence i has L_i tokens (``context`` range, inclusive),
+    the last q_i of which (``chunk`` range, q_i <= L_i) are the chunk being
+    processed: their K/V are written by the step's cache write and their queries
+    attend causally.  Draw order: lengths, chunk sizes, block permutation, Q,
+    K pool, V pool, chunk K, chunk V.
+    """
+    bs = block_size
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(context[0], context[1] + 1, size=num_seqs).astype(np.int64)
+    nq = np.minimum(rng.integers(chunk[0], chunk[1] + 1, size=num_seqs), lens).astype(np.int64)
+    need = int(sum(-(-int(L) // bs) for L in lens))
+    nb = max(1, math.ceil(pool_factor * need))
+    pool = BlockPool(rng.permutation(nb))
+    tables = [pool.allocate_for(int(L), bs) for L in lens]
+    Hkv, D = num_kv_heads, head_dim
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    T = int(qs[-1])
+    q = _to_storage(_draw(rng, (T, num_heads, D), "normal"), dtype)
+    kpool = _draw(rng, (nb, Hkv, bs, D), "normal")
+    vpool = _draw(rng, (nb, Hkv, bs, D), "normal")
+    nk = _draw(rng, (T, Hkv, D), "normal")
+    nv = _draw(rng, (T, Hkv, D), "normal")
+    owned = np.zeros((nb, bs), dtype=bool)
+    slots = np.empty(T, dtype=np.int64)
+    for i, L in enumerate(lens):
+        L = int(L)
+        for j, b in enumerate(tables[i]):
+            owned[b, :min(bs, L - j * bs)] = True
+        for t in range(int(nq[i])):
+            slots[qs[i] + t] = _slot(tables[i], L - int(nq[i]) + t, bs)
+    for sl in slots:  # the chunk's slots stay poisoned until the cache write
+        owned[int(sl) // bs, int(sl) % bs] = False
+    for b in np.nonzero(~owned.all(axis=1))[0]:
+        kpool[b][:, ~owned[b], :] = np.nan
+        vpool[b][:, ~owned[b], :] = np.nan
+    cfg = DecodeConfig("prefill", num_seqs=num_seqs, num_heads=num_heads, num_kv_heads=Hkv,
+                       head_dim=D, seq_lens=tuple(int(x) for x in lens), num_blocks=nb,
+                       q_dtype=dtype, cache_dtype=dtype, out_dtype=dtype, seed=seed,
+                       block_size=bs, new_tokens_per_seq=0)
+    width = max(1, max(len(t) for t in tables))
+    return Workload(cfg=cfg, query=q, key_cache=_to_storage(kpool, dtype),
+                    value_cache=_to_storage(vpool, dtype), block_tables=_table_tensor(tables, width),
+                    seq_lens=torch.from_numpy(lens.astype(np.int32)),
+                    new_key=_to_storage(nk, dtype), new_value=_to_storage(nv, dtype),
+                    slot_mapping=torch.from_numpy(slots), scale=_scale(D), src_dtype=dtype,
+                    refs=dict(pool.refs), query_start=torch.from_numpy(qs))

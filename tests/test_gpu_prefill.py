@@ -1,0 +1,79 @@
+"""GPU parity of the multi-query (chunked prefill) attention against the oracle.
+
+Each sequence's chunk (its last q tokens) is written by reshape_and_cache, then
+every chunk token attends causally over its context.  Cases: GQA group sizes 1..8,
+chunks from 1 token (equal to decode) to whole prompts, chunks spanning several
+64-row blocks, block sizes 16..128, fp16/bf16, every output type.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_413_b200 as pa
+from paged_kv_cache_413_b200 import workloads as W
+
+import flow
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(wl, out_dtype):
+    d = flow.to_device(wl)
+    qs = wl.query_start.cuda()
+    pa.pa_reshape_and_cache(d.new_key, d.new_value, d.key_cache, d.value_cache, d.slot_mapping)
+    out = torch.full(d.query.shape, float("nan"), dtype=flow.TORCH_DT[out_dtype], device="cuda")
+    max_q = int((wl.query_start[1:] - wl.query_start[:-1]).max())
+    pa.pa_paged_attention_prefill(out, d.query, d.key_cache, d.value_cache, d.block_tables,
+                                  d.seq_lens, qs, max_query_len=max_q,
+                                  max_seq_len=flow.max_seq_len(wl), scale=wl.scale)
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error() == 0
+    return d, out
+
+
+def _check(wl, out_dtype):
+    d, out = _run(wl, out_dtype)
+    kc, vc = oracle.reshape_and_cache(wl.new_key, wl.new_value, wl.key_cache, wl.value_cache,
+                                      wl.slot_mapping, src_dtype=wl.src_dtype,
+                                      cache_dtype=wl.cfg.cache_dtype)
+    ref = oracle.paged_attention_prefill(wl.query, kc, vc, wl.block_tables, wl.seq_lens,
+                                         wl.query_start, scale=wl.scale, q_dtype=wl.cfg.q_dtype,
+                                         cache_dtype=wl.cfg.cache_dtype)
+    err = flow.max_abs_err(out, ref)
+    assert err <= flow.TOL[out_dtype], f"max abs error {err:.3e}"
+    return d, out
+
+
+@pytest.mark.parametrize("h,hkv", [(8, 8), (16, 4), (64, 8), (12, 4)])
+@pytest.mark.parametrize("dt,out_dtype", [("bf16", "f32"), ("f16", "f16"), ("bf16", "bf16")])
+def test_prefill_groups(h, hkv, dt, out_dtype):
+    wl = W.make_prefill_workload(4, (20, 300), (1, 60), num_heads=h, num_kv_heads=hkv, dtype=dt,
+                                 seed=h + hkv)
+    _check(wl, out_dtype)
+
+
+@pytest.mark.parametrize("bs", [16, 64, 128])
+def test_prefill_whole_prompts_and_block_sizes(bs):
+    # chunk = the whole context: the first query sees one token
+    wl = W.make_prefill_workload(3, (1, 130), (130, 130), num_heads=16, num_kv_heads=4,
+                                 dtype="bf16", seed=bs, block_size=bs)
+    _check(wl, "f32")
+
+
+def test_prefill_long_chunk_over_long_context():
+    wl = W.make_prefill_workload(2, (1500, 2100), (300, 520), num_heads=64, num_kv_heads=8,
+                                 dtype="bf16", seed=7)
+    _check(wl, "bf16")
+
+
+def test_prefill_single_token_equals_decode():
+    wl = W.make_prefill_workload(5, (1, 400), (1, 1), num_heads=32, num_kv_heads=8,
+                                 dtype="bf16", seed=3)
+    d, out = _run(wl, "f32")
+    dec = torch.empty_like(out)
+    pa.pa_paged_attention_decode(dec, d.query, d.key_cache, d.value_cache, d.block_tables,
+                                 d.seq_lens, max_seq_len=flow.max_seq_len(wl), scale=wl.scale,
+                                 partition_size=1024)
+    assert (out - dec).abs().max().item() <= 1e-3

@@ -232,3 +232,56 @@ def test_lse_merge_closed_form():
     l = np.array([[1.0, 1.0, 0.0]])
     o = np.array([[[2.0], [6.0], [1e300]]])
     np.testing.assert_allclose(oracle.lse_merge(m, l, o), [[5.0]], rtol=1e-15)
+
+
+def test_prefill_one_query_equals_decode():
+    rng = np.random.default_rng(13)
+    lens = [1, 9, 16, 33]
+    kc, vc, bt = _identity_layout(rng, lens, 2, 8)
+    q = rng.standard_normal((len(lens), 4, 8)).astype(np.float32)
+    dec = oracle.paged_attention_decode(q, kc, vc, bt, np.array(lens, np.int32), scale=0.4,
+                                        q_dtype="f32", cache_dtype="f32")
+    pre = oracle.paged_attention_prefill(q, kc, vc, bt, np.array(lens, np.int32),
+                                         np.arange(len(lens) + 1, dtype=np.int32), scale=0.4,
+                                         q_dtype="f32", cache_dtype="f32")
+    assert np.array_equal(pre, dec)
+
+
+@pytest.mark.parametrize("group", [1, 4])
+def test_prefill_matches_causal_sdpa(group):
+    rng = np.random.default_rng(14)
+    lens, nq = [20, 37, 5], [7, 37, 1]
+    hkv, d = 2, 16
+    kc, vc, bt = _identity_layout(rng, lens, hkv, d)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    q = rng.standard_normal((int(qs[-1]), hkv * group, d)).astype(np.float32)
+    out = oracle.paged_attention_prefill(q, kc, vc, bt, np.array(lens, np.int32), qs, scale=0.3,
+                                         q_dtype="f32", cache_dtype="f32")
+    for i, (L, n) in enumerate(zip(lens, nq)):
+        first = bt[i, 0]
+        k = kc[first:first + bt.shape[1]].transpose(1, 0, 2, 3).reshape(hkv, -1, d)[:, :L]
+        v = vc[first:first + bt.shape[1]].transpose(1, 0, 2, 3).reshape(hkv, -1, d)[:, :L]
+        qt = torch.from_numpy(q[qs[i]:qs[i + 1]].astype(np.float64)).permute(1, 0, 2)[None]
+        kt = torch.from_numpy(k.astype(np.float64)).repeat_interleave(group, 0)[None]
+        vt = torch.from_numpy(v.astype(np.float64)).repeat_interleave(group, 0)[None]
+        # query j sits at position L - n + j: it may see keys 0 .. L - n + j
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask,
+                                                               scale=0.3)[0].permute(1, 0, 2)
+        np.testing.assert_allclose(out[qs[i]:qs[i + 1]], ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_prefill_first_query_of_a_full_prompt_sees_one_token():
+    # a whole 3-token prompt as queries: query 0 sees only token 0 -> exactly V0
+    kc = np.zeros((1, 1, 16, 2), dtype=np.float32)
+    vc = np.zeros((1, 1, 16, 2), dtype=np.float32)
+    kc[0, 0, :3] = [[1, 0], [0, 1], [1, 1]]
+    vc[0, 0, :3] = [[3, -1], [5, 2], [-7, 4]]
+    q = np.array([[[1.0, 0.0]], [[0.0, 2.0]], [[1.0, 1.0]]], dtype=np.float32)
+    out = oracle.paged_attention_prefill(q, kc, vc, np.array([[0]], np.int32),
+                                         np.array([3], np.int32), np.array([0, 3], np.int32),
+                                         scale=1.0, q_dtype="f32", cache_dtype="f32")
+    assert np.array_equal(out[0, 0], [3.0, -1.0])
+    # query 1 (position 1): scores 0 and 2 over tokens 0, 1
+    w = np.exp([0.0, 2.0]) / np.exp([0.0, 2.0]).sum()
+    np.testing.assert_allclose(out[1, 0], w[0] * vc[0, 0, 0] + w[1] * vc[0, 0, 1], atol=1e-15)
