@@ -45,7 +45,12 @@ DEFAULT_CONFIG = "llama2_7b"
 FALLBACK_HBM_GBS = 6650.0
 TORCH_DT = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
 
+PREFILL = {"chunked_prefill_70b": dict(num_seqs=16, context=(2048, 4096), chunk=(512, 512),
+                                       num_heads=64, num_kv_heads=8, dtype="bf16", seed=6)}
+
 DESCR = {
+    "chunked_prefill_70b": "Llama-2-70B layer, chunked prefill: 16 seqs, context U[2048,4096], "
+                           "512-token chunks, 64 q / 8 kv heads, d128, bf16, causal",
     "tiny": "4 seqs L={1,17,33,100}, 4 heads MHA, d64, fp16, pool 64 blocks",
     "llama2_7b": "Llama-2-7B layer: 64 seqs, 32 heads MHA, d128, L~U[128,2048], fp16 KV, "
                  "block 16, shuffled pool 1.1x",
@@ -427,6 +432,107 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+def prefill_flops(wl: W.Workload) -> int:
+    """Causal attention FLOPs: 4 * D per (query head, visible key) pair (QK and PV)."""
+    cfg = wl.cfg
+    L = wl.seq_lens.numpy().astype(np.int64)
+    qs = wl.query_start.numpy().astype(np.int64)
+    pairs = 0
+    for i in range(len(L)):
+        n = qs[i + 1] - qs[i]
+        pos = L[i] - n + np.arange(n)
+        pairs += int((pos + 1).sum())
+    return pairs * cfg.num_heads * cfg.head_dim * 4
+
+
+def run_prefill(args, rank, world, local_rank):
+    """The multi-query (chunked prefill) step: cache write of the chunks + attention."""
+    import paged_kv_cache_413_b200 as pa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    spec = dict(PREFILL[args.config])
+    spec["seed"] += 1000 * rank
+    wl = W.make_prefill_workload(spec.pop("num_seqs"), spec.pop("context"), spec.pop("chunk"),
+                                 **spec)
+    f = lambda t: t.to(dev)
+    kc, vc, q, bt, sl = f(wl.key_cache), f(wl.value_cache), f(wl.query), f(wl.block_tables), \
+        f(wl.seq_lens)
+    nk, nv, sm, qs = f(wl.new_key), f(wl.new_value), f(wl.slot_mapping), f(wl.query_start)
+    out = torch.empty_like(q)
+    max_q = int((wl.query_start[1:] - wl.query_start[:-1]).max())
+    max_len = int(wl.seq_lens.max())
+    stream = torch.cuda.current_stream(dev)
+    ev = []
+
+    def step(timed):
+        pa.pa_reshape_and_cache(nk, nv, kc, vc, sm)
+        if timed:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        pa.pa_paged_attention_prefill(out, q, kc, vc, bt, sl, qs, max_query_len=max_q,
+                                      max_seq_len=max_len, scale=wl.scale)
+        if timed:
+            e1.record(stream)
+            ev.append((e0, e1))
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.__enter__()
+    if world > 1:
+        torch.distributed.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.__exit__(None, None, None)
+    elapsed_ms, kern_ms = max_over_ranks(
+        [t0.elapsed_time(t1), statistics.mean(a.elapsed_time(b) for a, b in ev)], world, dev)
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error bits set")
+    if rank != 0:
+        return None
+    flops = prefill_flops(wl)
+    cfg = wl.cfg
+    # the launcher's rule: 128-row tcgen05 tiles once a chunk fills one
+    kernel = ("prefill_tc_kernel (tcgen05.mma, TMEM accumulators)"
+              if max_q * (cfg.num_heads // cfg.num_kv_heads) >= 128
+              else "prefill_kernel (mma.sync m16n8k16)")
+    L = wl.seq_lens.numpy().astype(np.int64)
+    kv_bytes = int(L.sum()) * cfg.num_kv_heads * cfg.head_dim * 2 * 2
+    qo_bytes = 2 * q.numel() * 2
+    peak = 1686.0
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            peak = float(json.load(fh)["bf16_tflops"])
+        kind = "measured (bf16_tflops, cuBLAS burst)"
+    except Exception:
+        kind = "fallback"
+    tflops = flops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
+    achieved = flops / (kern_ms * 1e-3) / 1e12
+    return {"metric": "paged multi-query attention (chunked prefill): TFLOP/s", "value":
+            round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{args.config}: {DESCR[args.config]}",
+                       "query_tokens": int(wl.query_start[-1]), "flops_per_step": flops,
+                       "l2": f"KV read {kv_bytes / 1e6:.0f} MB per step, above the 126 MB L2"},
+            "roofline": {"bound": "tensor", "kernel": kernel,
+                         "achieved": round(achieved, 2), "peak": peak, "peak_kind": kind,
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "launch_ms": round(kern_ms, 5),
+                         "hbm_gbs": round((kv_bytes + qo_bytes) / (kern_ms * 1e-3) / 1e9, 1)},
+            "gpu_launches": 2 * args.steps,
+            "clocks": sampler.summary() if sampler else None}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm: each step a bounded sample (one sequence)."""
     if rank != 0:
@@ -464,7 +570,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.CONFIGS))
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.CONFIGS) + sorted(PREFILL))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=None)
     ap.add_argument("--block-size", type=int, default=0,
@@ -487,7 +593,10 @@ def main():
                 "nccl", timeout=datetime.timedelta(seconds=120),
                 device_id=torch.device("cuda", local_rank))
         try:
-            line = run_ours(args, rank, world, local_rank)
+            if args.config in PREFILL:
+                line = run_prefill(args, rank, world, local_rank)
+            else:
+                line = run_ours(args, rank, world, local_rank)
         finally:
             if world > 1:
                 torch.distributed.destroy_process_group()

@@ -47,7 +47,10 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 #ifndef PA_MMA16_STAGES
 #define PA_MMA16_STAGES 4
 #endif
-constexpr int kStagesSimt = 8;                  // 8 KB K+V per stage at D = 128, 16-bit
+#ifndef PA_SIMT_STAGES
+#define PA_SIMT_STAGES 8
+#endif
+constexpr int kStagesSimt = PA_SIMT_STAGES;     // 8 KB K+V per stage at D = 128, 16-bit
 constexpr int kStagesMma16 = PA_MMA16_STAGES;   // 8 KB per stage; 4 CTAs per SM
 constexpr int kStagesMmaFp8 = 8;                // 4 KB per stage
 static_assert(kStagesSimt % kConsumerWarps == 0 && kStagesMma16 % kConsumerWarps == 0 &&
@@ -1646,6 +1649,400 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
   }
 }
 
+// ---------------------------------------------------------------------------
+// Chunked prefill on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// For chunks with at least 128 (query token, head) rows per kv head the
+// contraction is large enough for the CTA-wide MMA: one CTA holds 128 rows (one
+// TMEM lane each) and walks the sequence's KV in stages of 64 tokens (four
+// 16-token tiles placed by TMA as one 128-byte-swizzled K-major operand):
+//   S[128 x 64]  = Q[128 x 128] . K^T         (tcgen05.mma, fp32 in TMEM, two buffers)
+//   O_blk[128 x 128] = P[128 x 64] . V[64 x 128]   (V read as an MN-major operand)
+// Four softmax warps own 32 rows each (a row per thread, so row statistics need
+// no shuffles): they read S from TMEM, apply the causal and context masks and the
+// online softmax in fp32, write P (16-bit) into swizzled shared memory for the
+// second MMA, and fold each O_blk into a register accumulator with the running
+// rescale.  One warp feeds the TMA ring; one thread issues every MMA and tracks
+// completion with tcgen05.commit on mbarriers.  All waits are bounded.
+// kSplitP (bf16 operands with an fp32 output): P is held as two bf16 terms, hi
+// and lo = P - hi, and P.V takes both, so the 16-bit rounding of P (relative
+// 2^-9 in bf16) does not reach a full-precision output.
+// ---------------------------------------------------------------------------
+constexpr int kTcRows = 128;                   // query rows per CTA = TMEM lanes
+constexpr int kTcKv = 64;                      // tokens per KV stage
+constexpr int kTcStages = 2;
+constexpr int kTcSoftmaxWarps = 4;
+constexpr int kTcThreads = (kTcSoftmaxWarps + 2) * 32;  // + TMA warp + MMA warp
+constexpr uint32_t kTcTmemCols = 256;          // S: 2 x 64 columns, O_blk: 128 columns
+constexpr int kTcQBytes = 2 * kTcRows * 128;   // [2 halves][128 rows][128 B]
+constexpr int kTcKvBytes = 2 * kTcKv * 128;    // K or V of one stage: [2][64][128 B]
+constexpr int kTcPBytes = kTcRows * 128;       // [128 rows][64 tokens x 2 B], per P term
+
+struct TcPrefillParams {
+  CUtensorMap tmk;
+  CUtensorMap tmv;
+  Params p;
+  const int32_t* query_start;
+  int row_blocks;
+};
+
+constexpr size_t tc_prefill_smem_bytes() {
+  return 1024 + size_t(kTcQBytes) + size_t(kTcStages) * 2 * kTcKvBytes + 2 * kTcPBytes +
+         (2 * kTcStages + 6) * sizeof(uint64_t) + 16;
+}
+
+template <typename CT, bool kSplitP>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ TcPrefillParams pp) {
+  constexpr int D = 128;
+  static_assert(CacheTraits<CT>::bytes == 2, "16-bit caches");
+  constexpr uint32_t kFmt = std::is_same<CT, __nv_bfloat16>::value ? 1u : 0u;
+  constexpr uint32_t kIdescS = umma_idesc_f16(kFmt, 0, kTcRows, kTcKv);
+  constexpr uint32_t kIdescPV = umma_idesc_f16(kFmt, 1, kTcRows, D);
+  const Params& p = pp.p;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* qs = smem;                                    // Q operand
+  uint8_t* kvs = qs + kTcQBytes;                         // stage s: K at s*2*KV, V after it
+  uint8_t* ps = kvs + kTcStages * 2 * kTcKvBytes;        // P operand (hi term)
+  uint8_t* ps_lo = ps + kTcPBytes;                       // P - hi, with kSplitP
+  uint64_t* kv_full = reinterpret_cast<uint64_t*>(ps + 2 * kTcPBytes);
+  uint64_t* kv_empty = kv_full + kTcStages;
+  uint64_t* s_full = kv_empty + kTcStages;               // [2]
+  uint64_t* o_full = s_full + 2;
+  uint64_t* p_ready = o_full + 1;
+  uint64_t* done = p_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int seq = blockIdx.x / pp.row_blocks;
+  const int rblk = blockIdx.x - seq * pp.row_blocks;
+  const int kvh = blockIdx.y;
+  const int G = p.group;
+  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+  int L = p.seq_lens[seq];
+  const int q0 = pp.query_start[seq];
+  int nq = pp.query_start[seq + 1] - q0;
+  if (L < 0 || L > cap || nq < 0 || nq > L) {
+    if (tid == 0 && rblk == 0 && kvh == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
+    L = L < 0 ? 0 : (L > cap ? cap : L);
+    nq = nq < 0 ? 0 : (nq > L ? L : nq);
+  }
+  const int rows = nq * G;
+  const int row0 = rblk * kTcRows;
+  if (row0 >= rows) return;  // uniform: before any barrier or TMEM allocation
+  const int pos_last = L - nq + (min(rows, row0 + kTcRows) - 1) / G;
+  const int ntiles = pos_last / kBlockSize + 1;
+  const int nkb = (pos_last + kTcKv) / kTcKv;  // KV stages to process
+
+  if (tid == 0) {
+    for (int st = 0; st < kTcStages; ++st) {
+      mbar_init(&kv_full[st], 1);
+      mbar_init(&kv_empty[st], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(o_full, 1);
+    mbar_init(p_ready, kTcSoftmaxWarps);
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == kTcSoftmaxWarps + 1) {  // the MMA warp owns the TMEM allocation
+    tmem_alloc(tmem_slot, kTcTmemCols);
+    tmem_relinquish();
+  }
+  // Q rows into the swizzled K-major operand: row r, 16-byte chunk c of 16.
+  if (warp < kTcSoftmaxWarps) {
+    const int r = tid;
+    const int gr = row0 + r;
+    const bool valid = gr < rows;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        p.query + (int64_t(q0 + (valid ? gr / G : 0)) * p.num_heads + kvh * G +
+                   (valid ? gr % G : 0)) * D * 2);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(qs + (c >> 3) * (kTcRows * 128) + r * 128 +
+                                (((c & 7) ^ (r & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  tcgen05_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTcSoftmaxWarps) {
+    // ---------------- TMA producer: stage jb = sequence tiles 4jb .. 4jb+3 ----------------
+    const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
+    const uint64_t policy = l2_policy_evict_last();  // other row blocks read it again
+    int issued = 0;
+    bool ok = true;
+    for (int jb = 0; jb < nkb && ok; ++jb) {
+      const int stage = jb % kTcStages;
+      const int ntl = min(4, ntiles - 4 * jb);
+      int tile = 0;
+      if (lane < ntl) {
+        const int t = 4 * jb + lane, e = t / p.tiles_per_block;
+        int32_t phys = table_row[e];
+        if (phys < 0 || phys >= p.num_blocks) {
+          atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
+          phys = 0;
+        }
+        tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
+      }
+      int tls[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) tls[t] = __shfl_sync(kFullMask, tile, t);
+      if (lane == 0) {
+        if (jb >= kTcStages && !mbar_wait_bounded(&kv_empty[stage], ((jb / kTcStages) - 1) & 1)) {
+          atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+          ok = false;
+        }
+        if (ok) {
+          uint8_t* kd = kvs + stage * 2 * kTcKvBytes;
+          uint8_t* vd = kd + kTcKvBytes;
+          mbar_arrive_expect_tx(&kv_full[stage], uint32_t(ntl) * 4 * 2048);
+          for (int t = 0; t < ntl; ++t) {
+            const int row = tls[t] * kBlockSize;
+            tma_load_2d(kd + t * 2048, &pp.tmk, 0, row, &kv_full[stage], policy);
+            tma_load_2d(kd + kTcKvBytes / 2 + t * 2048, &pp.tmk, 64, row, &kv_full[stage], policy);
+            tma_load_2d(vd + t * 2048, &pp.tmv, 0, row, &kv_full[stage], policy);
+            tma_load_2d(vd + kTcKvBytes / 2 + t * 2048, &pp.tmv, 64, row, &kv_full[stage], policy);
+          }
+          ++issued;
+        }
+      }
+      ok = __shfl_sync(kFullMask, ok, 0);
+    }
+    if (lane == 0) {
+      const int first = issued > kTcStages ? issued - kTcStages : 0;
+      for (int i = first; i < issued; ++i)
+        if (!mbar_wait_bounded(&kv_full[i % kTcStages], (i / kTcStages) & 1))
+          atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+    }
+  } else if (warp == kTcSoftmaxWarps + 1) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      const uint32_t qaddr = smem_u32(qs);
+      const uint32_t paddr = smem_u32(ps);
+      auto issue_s = [&](int jb) {  // S[jb % 2] = Q . K(stage of jb)^T
+        const uint32_t kaddr = smem_u32(kvs + (jb % kTcStages) * 2 * kTcKvBytes);
+        const uint32_t d = tmem + uint32_t(jb & 1) * kTcKv;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t a = umma_smem_desc(qaddr + (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32,
+                                            16, 1024, kUmmaSwizzle128B);
+          const uint64_t b = umma_smem_desc(kaddr + (ks >> 2) * (kTcKvBytes / 2) + (ks & 3) * 32,
+                                            16, 1024, kUmmaSwizzle128B);
+          umma_f16_ss(d, a, b, kIdescS, ks > 0);
+        }
+        umma_commit(&s_full[jb & 1]);
+      };
+      auto issue_pv = [&](int jb) {  // O_blk = P . V(stage of jb)
+        const uint32_t vaddr = smem_u32(kvs + (jb % kTcStages) * 2 * kTcKvBytes + kTcKvBytes);
+#pragma unroll
+        for (int ks = 0; ks < kTcKv / 16; ++ks) {
+          const uint64_t a = umma_smem_desc(paddr + ks * 32, 16, 1024, kUmmaSwizzle128B);
+          const uint64_t b =
+              umma_smem_desc(vaddr + ks * 2048, kTcKvBytes / 2, 1024, kUmmaSwizzle128B);
+          umma_f16_ss(tmem + 128, a, b, kIdescPV, ks > 0);
+        }
+        if constexpr (kSplitP) {
+#pragma unroll
+          for (int ks = 0; ks < kTcKv / 16; ++ks) {
+            const uint64_t a =
+                umma_smem_desc(paddr + kTcPBytes + ks * 32, 16, 1024, kUmmaSwizzle128B);
+            const uint64_t b =
+                umma_smem_desc(vaddr + ks * 2048, kTcKvBytes / 2, 1024, kUmmaSwizzle128B);
+            umma_f16_ss(tmem + 128, a, b, kIdescPV, 1u);
+          }
+        }
+        umma_commit(o_full);
+        umma_commit(&kv_empty[jb % kTcStages]);
+      };
+      bool ok = mbar_wait_bounded(&kv_full[0], 0);
+      if (ok) {
+        tcgen05_fence_after();
+        issue_s(0);
+      }
+      for (int jb = 0; jb < nkb && ok; ++jb) {
+        if (jb + 1 < nkb) {
+          ok = mbar_wait_bounded(&kv_full[(jb + 1) % kTcStages], ((jb + 1) / kTcStages) & 1);
+          if (!ok) break;
+          tcgen05_fence_after();
+          issue_s(jb + 1);
+        }
+        ok = mbar_wait_bounded(p_ready, jb & 1);
+        if (!ok) break;
+        tcgen05_fence_after();
+        issue_pv(jb);
+      }
+      if (!ok) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+      umma_commit(done);  // fires once every MMA issued above has completed
+    }
+    __syncwarp();
+  } else {
+    // ---------------- softmax warps: thread = row ----------------
+    const int r = tid;  // TMEM lane and Q row
+    const int gr = row0 + r;
+    const bool valid = gr < rows;
+    const int pos = valid ? L - nq + gr / G : -1;
+    const uint32_t tl = tmem + (uint32_t(32 * warp) << 16);  // this warp's lane quadrant
+    const float mult = p.q_mult;
+    float o[128];
+#pragma unroll
+    for (int d = 0; d < 128; ++d) o[d] = 0.f;
+    float m = -INFINITY, l = 0.f, alpha_pend = 1.f;
+    bool ok = true;
+    for (int jb = 0; jb < nkb; ++jb) {
+      if (!__all_sync(kFullMask, mbar_wait_bounded(&s_full[jb & 1], (jb >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tcgen05_fence_after();
+      float sv[64];
+      {
+        float a[32], b[32];
+        tmem_ld32(tl + uint32_t(jb & 1) * kTcKv, a);
+        tmem_ld32(tl + uint32_t(jb & 1) * kTcKv + 32, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = a[i];
+          sv[32 + i] = b[i];
+        }
+      }
+      const int t0 = jb * kTcKv;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        sv[i] = (t0 + i <= pos) ? sv[i] * mult : -INFINITY;  // causal, context and padding
+        mx = fmaxf(mx, sv[i]);
+      }
+      const float mn = fmaxf(m, mx);
+      const float alpha = mn == -INFINITY ? 1.f : exp2f(m - mn);
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        sv[i] = mn == -INFINITY ? 0.f : exp2f(sv[i] - mn);
+        sum += sv[i];
+      }
+      m = mn;
+      l = l * alpha + sum;
+      // P(jb) may overwrite the P operand once P.V(jb - 1) has completed
+      if (jb > 0) {
+        if (!__all_sync(kFullMask, mbar_wait_bounded(o_full, (jb - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tcgen05_fence_after();
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 w;
+        w.x = pack2(sv[8 * c + 0], sv[8 * c + 1], CT{});
+        w.y = pack2(sv[8 * c + 2], sv[8 * c + 3], CT{});
+        w.z = pack2(sv[8 * c + 4], sv[8 * c + 5], CT{});
+        w.w = pack2(sv[8 * c + 6], sv[8 * c + 7], CT{});
+        *reinterpret_cast<uint4*>(ps + r * 128 + ((c ^ (r & 7)) << 4)) = w;
+        if constexpr (kSplitP) {
+          const float2 h0 = unpack2(w.x, CT{}), h1 = unpack2(w.y, CT{}), h2 = unpack2(w.z, CT{}),
+                       h3 = unpack2(w.w, CT{});
+          uint4 lo;
+          lo.x = pack2(sv[8 * c + 0] - h0.x, sv[8 * c + 1] - h0.y, CT{});
+          lo.y = pack2(sv[8 * c + 2] - h1.x, sv[8 * c + 3] - h1.y, CT{});
+          lo.z = pack2(sv[8 * c + 4] - h2.x, sv[8 * c + 5] - h2.y, CT{});
+          lo.w = pack2(sv[8 * c + 6] - h3.x, sv[8 * c + 7] - h3.y, CT{});
+          *reinterpret_cast<uint4*>(ps_lo + r * 128 + ((c ^ (r & 7)) << 4)) = lo;
+        }
+      }
+      if (jb == nkb - 1) {
+        // V rows past the last visible token may be stale or NaN: zero them
+        if (!__all_sync(kFullMask, mbar_wait_bounded(&kv_full[jb % kTcStages], (jb / kTcStages) & 1))) {
+          ok = false;
+          break;
+        }
+        const int vr = r >> 1, half = r & 1;
+        if (t0 + vr > pos_last) {
+          uint8_t* vrow = kvs + (jb % kTcStages) * 2 * kTcKvBytes + kTcKvBytes +
+                          half * (kTcKvBytes / 2) + vr * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();
+      // fold O_blk(jb - 1) in before P.V(jb) may overwrite it
+      if (jb > 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float v[32];
+          tmem_ld32(tl + 128 + 32 * q, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[32 * q + i] = fmaf(o[32 * q + i], alpha_pend, v[i]);
+        }
+      }
+      alpha_pend = alpha;
+      tcgen05_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready);
+    }
+    if (ok && __all_sync(kFullMask, mbar_wait_bounded(o_full, (nkb - 1) & 1))) {
+      tcgen05_fence_after();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v[32];
+        tmem_ld32(tl + 128 + 32 * q, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[32 * q + i] = fmaf(o[32 * q + i], alpha_pend, v[i]);
+      }
+    } else {
+      ok = false;
+    }
+    if (!ok && lane == 0) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+    tcgen05_fence_before();
+    if (valid && ok) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint8_t* dst = static_cast<uint8_t*>(p.out);
+      const int64_t orow = (int64_t(q0 + gr / G) * p.num_heads + kvh * G + gr % G) * D;
+      if (p.out_dtype == PA_F32) {
+#pragma unroll
+        for (int d = 0; d < 128; d += 4)
+          *reinterpret_cast<float4*>(dst + (orow + d) * 4) =
+              make_float4(o[d] * inv, o[d + 1] * inv, o[d + 2] * inv, o[d + 3] * inv);
+      } else {
+#pragma unroll
+        for (int d = 0; d < 128; d += 8) {
+          uint4 w;
+          if (p.out_dtype == PA_F16) {
+            w = make_uint4(pack2(o[d] * inv, o[d + 1] * inv, __half{}),
+                           pack2(o[d + 2] * inv, o[d + 3] * inv, __half{}),
+                           pack2(o[d + 4] * inv, o[d + 5] * inv, __half{}),
+                           pack2(o[d + 6] * inv, o[d + 7] * inv, __half{}));
+          } else {
+            w = make_uint4(pack2(o[d] * inv, o[d + 1] * inv, __nv_bfloat16{}),
+                           pack2(o[d + 2] * inv, o[d + 3] * inv, __nv_bfloat16{}),
+                           pack2(o[d + 4] * inv, o[d + 5] * inv, __nv_bfloat16{}),
+                           pack2(o[d + 6] * inv, o[d + 7] * inv, __nv_bfloat16{}));
+          }
+          *reinterpret_cast<uint4*>(dst + (orow + d) * 2) = w;
+        }
+      }
+    }
+  }
+  // Free TMEM only after every MMA has completed and every TMEM read is done.
+  __syncthreads();
+  if (warp == kTcSoftmaxWarps + 1) {
+    if (!__all_sync(kFullMask, mbar_wait_bounded(done, 0)) && lane == 0)
+      atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+    tcgen05_fence_after();
+    tmem_dealloc(tmem, kTcTmemCols);
+  }
+}
+
 // Log-sum-exp merge of the partitions of sequences with more than one:
 // M = max m_p, w_p = l_p exp(m_p - M), out = sum w_p o_p / sum w_p.
 // One warp per (sequence, head) row, 8 rows per CTA; lanes own D/32 dims.
@@ -1946,6 +2343,36 @@ int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_quer
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   };
   static unsigned long long mask_h = 0, mask_b = 0;
+  if (int64_t(max_query_len) * group >= kTcRows) {
+    // 128-row tiles for the 5th-generation tensor cores
+    TcPrefillParams tp;
+    memset(&tp, 0, sizeof tp);
+    tp.tmk = pp.tmk;
+    tp.tmv = pp.tmv;
+    tp.p = pp.p;
+    tp.query_start = pp.query_start;
+    tp.row_blocks = int((int64_t(max_query_len) * group + kTcRows - 1) / kTcRows);
+    const int64_t gx = int64_t(a.num_seqs) * tp.row_blocks;
+    if (gx > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    constexpr size_t smem = tc_prefill_smem_bytes();
+    auto launch = [&](auto kern, unsigned long long& mask) -> int {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+      const unsigned long long bit = 1ull << (dev & 63);
+      if (!(mask & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+            cudaSuccess)
+          return PA_ERR_CUDA;
+        mask |= bit;
+      }
+      kern<<<dim3(unsigned(gx), unsigned(a.num_kv_heads)), kTcThreads, smem, stream>>>(tp);
+      return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    };
+    static unsigned long long tmask_h = 0, tmask_b = 0, tmask_bs = 0;
+    if (a.cache_dtype == PA_F16) return launch(prefill_tc_kernel<__half, false>, tmask_h);
+    if (a.out_dtype == PA_F32) return launch(prefill_tc_kernel<__nv_bfloat16, true>, tmask_bs);
+    return launch(prefill_tc_kernel<__nv_bfloat16, false>, tmask_b);
+  }
   if (a.cache_dtype == PA_F16)
     return run(prefill_kernel<__half, stages>, prefill_smem_bytes<__half, stages>(), mask_h);
   return run(prefill_kernel<__nv_bfloat16, stages>, prefill_smem_bytes<__nv_bfloat16, stages>(),

@@ -3,7 +3,9 @@
 Each sequence's chunk (its last q tokens) is written by reshape_and_cache, then
 every chunk token attends causally over its context.  Cases: GQA group sizes 1..8,
 chunks from 1 token (equal to decode) to whole prompts, chunks spanning several
-64-row blocks, block sizes 16..128, fp16/bf16, every output type.
+row blocks, block sizes 16..128, fp16/bf16, every output type.  Chunks with fewer
+than 128 (token, head) rows per kv head run on the 64-row mma.sync kernel, larger
+ones on the 128-row tcgen05 kernel: both sides of that edge are covered.
 """
 
 import numpy as np
@@ -77,3 +79,24 @@ def test_prefill_single_token_equals_decode():
                                  d.seq_lens, max_seq_len=flow.max_seq_len(wl), scale=wl.scale,
                                  partition_size=1024)
     assert (out - dec).abs().max().item() <= 1e-3
+
+
+@pytest.mark.parametrize("chunk", [15, 16, 17, 33])
+def test_prefill_row_block_edges(chunk):
+    # GQA-8: 120, 128, 136 and 264 rows per kv head around the 128-row tile
+    wl = W.make_prefill_workload(3, (chunk, 300), (chunk, chunk), num_heads=64, num_kv_heads=8,
+                                 dtype="bf16", seed=chunk)
+    _check(wl, "f32")
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_prefill_ragged_chunks_both_kernels(dt):
+    # chunks of 1..8 tokens (at most 32 rows per kv head): the 64-row kernel
+    wl = W.make_prefill_workload(6, (200, 900), (1, 8), num_heads=32, num_kv_heads=8,
+                                 dtype=dt, seed=11)
+    _check(wl, dt)
+    # chunks of 1..190 tokens (up to 6 row blocks of 128): CTAs past a short
+    # sequence's rows have nothing to do and leave before any barrier
+    wl2 = W.make_prefill_workload(6, (700, 900), (1, 190), num_heads=32, num_kv_heads=8,
+                                  dtype=dt, seed=12)
+    _check(wl2, dt)
