@@ -1670,7 +1670,11 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
 // ---------------------------------------------------------------------------
 constexpr int kTcRows = 128;                   // query rows per CTA = TMEM lanes
 constexpr int kTcKv = 64;                      // tokens per KV stage
-constexpr int kTcStages = 2;
+#ifndef PA_TC_STAGES
+#define PA_TC_STAGES 2
+#endif
+constexpr int kTcStages = PA_TC_STAGES;        // 32 KB of K+V per stage
+static_assert(kTcStages >= 2 && kTcStages <= 4, "Q, two P terms and the ring fit 227 KB");
 constexpr int kTcSoftmaxWarps = 4;
 constexpr int kTcThreads = (kTcSoftmaxWarps + 2) * 32;  // + TMA warp + MMA warp
 constexpr uint32_t kTcTmemCols = 256;          // S: 2 x 64 columns, O_blk: 128 columns
@@ -1760,9 +1764,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint4* src = reinterpret_cast<const uint4*>(
         p.query + (int64_t(q0 + (valid ? gr / G : 0)) * p.num_heads + kvh * G +
                    (valid ? gr % G : 0)) * D * 2);
+    // a negative scale is applied as |scale| to -Q (a sign flip is exact), so the
+    // softmax may take the row max before scaling
+    const uint32_t flip = p.q_mult < 0.f ? 0x80008000u : 0u;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-      const uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      v.x ^= flip;
+      v.y ^= flip;
+      v.z ^= flip;
+      v.w ^= flip;
       *reinterpret_cast<uint4*>(qs + (c >> 3) * (kTcRows * 128) + r * 128 +
                                 (((c & 7) ^ (r & 7)) << 4)) = v;
     }
@@ -1890,7 +1901,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const bool valid = gr < rows;
     const int pos = valid ? L - nq + gr / G : -1;
     const uint32_t tl = tmem + (uint32_t(32 * warp) << 16);  // this warp's lane quadrant
-    const float mult = p.q_mult;
+    const float mult = fabsf(p.q_mult);  // Q carries the sign
     float o[128];
 #pragma unroll
     for (int d = 0; d < 128; ++d) o[d] = 0.f;
@@ -1914,21 +1925,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           sv[32 + i] = b[i];
         }
       }
-      const int t0 = jb * kTcKv;
-      float mx = -INFINITY;
+      // causal, context and padding mask: only stages that cross this row's last
+      // visible position pay for it
+      const int nvis = pos - jb * kTcKv + 1;
+      float me = mult;  // multiplier still to apply to sv
+      if (nvis < kTcKv) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) sv[i] = i < nvis ? sv[i] * mult : -INFINITY;
+        me = 1.f;
+      }
+      // row max and sum over 8 independent chains (one row per thread: no shuffles)
+      float r8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) r8[k] = sv[k];
+#pragma unroll
+      for (int i = 8; i < 64; ++i) r8[i & 7] = fmaxf(r8[i & 7], sv[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(r8[0], r8[1]), fmaxf(r8[2], r8[3])),
+                             fmaxf(fmaxf(r8[4], r8[5]), fmaxf(r8[6], r8[7])));
+      const float mn = fmaxf(m, mx * me);  // scores scaled into the exp2 domain
+      const float mu = mn == -INFINITY ? 0.f : mn;
+      const float alpha = ex2_approx(m - mu);  // 0 while nothing was visible
+#pragma unroll
+      for (int k = 0; k < 8; ++k) r8[k] = 0.f;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        sv[i] = (t0 + i <= pos) ? sv[i] * mult : -INFINITY;  // causal, context and padding
-        mx = fmaxf(mx, sv[i]);
+        sv[i] = ex2_approx(fmaf(sv[i], me, -mu));
+        r8[i & 7] += sv[i];
       }
-      const float mn = fmaxf(m, mx);
-      const float alpha = mn == -INFINITY ? 1.f : exp2f(m - mn);
-      float sum = 0.f;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        sv[i] = mn == -INFINITY ? 0.f : exp2f(sv[i] - mn);
-        sum += sv[i];
-      }
+      const float sum = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       m = mn;
       l = l * alpha + sum;
       // P(jb) may overwrite the P operand once P.V(jb - 1) has completed
@@ -1965,7 +1989,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         const int vr = r >> 1, half = r & 1;
-        if (t0 + vr > pos_last) {
+        if (jb * kTcKv + vr > pos_last) {
           uint8_t* vrow = kvs + (jb % kTcStages) * 2 * kTcKvBytes + kTcKvBytes +
                           half * (kTcKvBytes / 2) + vr * 128;
 #pragma unroll

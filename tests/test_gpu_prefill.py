@@ -21,7 +21,7 @@ import flow
 pytestmark = pytest.mark.gpu
 
 
-def _run(wl, out_dtype):
+def _run(wl, out_dtype, scale=None):
     d = flow.to_device(wl)
     qs = wl.query_start.cuda()
     pa.pa_reshape_and_cache(d.new_key, d.new_value, d.key_cache, d.value_cache, d.slot_mapping)
@@ -29,19 +29,21 @@ def _run(wl, out_dtype):
     max_q = int((wl.query_start[1:] - wl.query_start[:-1]).max())
     pa.pa_paged_attention_prefill(out, d.query, d.key_cache, d.value_cache, d.block_tables,
                                   d.seq_lens, qs, max_query_len=max_q,
-                                  max_seq_len=flow.max_seq_len(wl), scale=wl.scale)
+                                  max_seq_len=flow.max_seq_len(wl),
+                                  scale=wl.scale if scale is None else scale)
     torch.cuda.synchronize()
     assert pa.pa_get_device_error() == 0
     return d, out
 
 
-def _check(wl, out_dtype):
-    d, out = _run(wl, out_dtype)
+def _check(wl, out_dtype, scale=None):
+    scale = wl.scale if scale is None else scale
+    d, out = _run(wl, out_dtype, scale)
     kc, vc = oracle.reshape_and_cache(wl.new_key, wl.new_value, wl.key_cache, wl.value_cache,
                                       wl.slot_mapping, src_dtype=wl.src_dtype,
                                       cache_dtype=wl.cfg.cache_dtype)
     ref = oracle.paged_attention_prefill(wl.query, kc, vc, wl.block_tables, wl.seq_lens,
-                                         wl.query_start, scale=wl.scale, q_dtype=wl.cfg.q_dtype,
+                                         wl.query_start, scale=scale, q_dtype=wl.cfg.q_dtype,
                                          cache_dtype=wl.cfg.cache_dtype)
     err = flow.max_abs_err(out, ref)
     assert err <= flow.TOL[out_dtype], f"max abs error {err:.3e}"
@@ -100,3 +102,12 @@ def test_prefill_ragged_chunks_both_kernels(dt):
     wl2 = W.make_prefill_workload(6, (700, 900), (1, 190), num_heads=32, num_kv_heads=8,
                                   dtype=dt, seed=12)
     _check(wl2, dt)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.06])
+@pytest.mark.parametrize("chunk", [(1, 12), (40, 90)])
+def test_prefill_zero_and_negative_scale(scale, chunk):
+    # a zero scale gives the mean of the visible V rows; a negative one reverses the order
+    wl = W.make_prefill_workload(3, (100, 400), chunk, num_heads=32, num_kv_heads=8,
+                                 dtype="bf16", seed=21)
+    _check(wl, "f32", scale=scale)
