@@ -1655,32 +1655,44 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
 // For chunks with at least 128 (query token, head) rows per kv head the
 // contraction is large enough for the CTA-wide MMA: one CTA holds 128 rows (one
 // TMEM lane each) and walks the sequence's KV in stages of 64 tokens (four
-// 16-token tiles placed by TMA as one 128-byte-swizzled K-major operand):
-//   S[128 x 64]  = Q[128 x 128] . K^T         (tcgen05.mma, fp32 in TMEM, two buffers)
-//   O_blk[128 x 128] = P[128 x 64] . V[64 x 128]   (V read as an MN-major operand)
-// Four softmax warps own 32 rows each (a row per thread, so row statistics need
-// no shuffles): they read S from TMEM, apply the causal and context masks and the
-// online softmax in fp32, write P (16-bit) into swizzled shared memory for the
-// second MMA, and fold each O_blk into a register accumulator with the running
-// rescale.  One warp feeds the TMA ring; one thread issues every MMA and tracks
-// completion with tcgen05.commit on mbarriers.  All waits are bounded.
+// 16-token tiles placed by TMA as one 128-byte-swizzled operand):
+//   S[128 x 64]   = Q[128 x 128] . K^T   A = Q, B = K from shared memory; fp32 S in
+//                                        TMEM, two buffers
+//   O[128 x 128] += P[128 x 64] . V      A = P from TMEM (written over its own S),
+//                                        B = V from shared memory (MN-major); O
+//                                        stays in TMEM for the whole pass
+// K and V have rings and producer warps of their own, so a K slot refills as
+// soon as its S is done and a V slot as soon as its P.V is done.  Eight softmax warps, two per TMEM lane quadrant,
+// each take 32 rows x 32 of the 64 columns (the row max of the two halves meets in
+// shared memory behind a 64-thread named barrier): masks, fp32 online softmax in
+// the exp2 domain, P as 16-bit pairs into TMEM.  P is taken relative to a per-row
+// reference max that moves only when a new score exceeds it by more than 2^8, so
+// O in TMEM is rescaled rarely.  One thread polls
+// the barriers and issues each S and P.V as soon as its inputs are ready
+// (tcgen05.commit reports completion).  All waits are bounded, and the named
+// barriers are reached the same number of times on every path.
 // kSplitP (bf16 operands with an fp32 output): P is held as two bf16 terms, hi
-// and lo = P - hi, and P.V takes both, so the 16-bit rounding of P (relative
-// 2^-9 in bf16) does not reach a full-precision output.
+// and lo = P - hi (stored over the second half of the same S buffer), and P.V
+// takes both, so the 16-bit rounding of P (relative 2^-9 in bf16) does not reach
+// a full-precision output.
 // ---------------------------------------------------------------------------
 constexpr int kTcRows = 128;                   // query rows per CTA = TMEM lanes
 constexpr int kTcKv = 64;                      // tokens per KV stage
 #ifndef PA_TC_STAGES
-#define PA_TC_STAGES 2
+#define PA_TC_STAGES 4
 #endif
-constexpr int kTcStages = PA_TC_STAGES;        // 32 KB of K+V per stage
-static_assert(kTcStages >= 2 && kTcStages <= 4, "Q, two P terms and the ring fit 227 KB");
-constexpr int kTcSoftmaxWarps = 4;
-constexpr int kTcThreads = (kTcSoftmaxWarps + 2) * 32;  // + TMA warp + MMA warp
-constexpr uint32_t kTcTmemCols = 256;          // S: 2 x 64 columns, O_blk: 128 columns
-constexpr int kTcQBytes = 2 * kTcRows * 128;   // [2 halves][128 rows][128 B]
-constexpr int kTcKvBytes = 2 * kTcKv * 128;    // K or V of one stage: [2][64][128 B]
-constexpr int kTcPBytes = kTcRows * 128;       // [128 rows][64 tokens x 2 B], per P term
+constexpr int kTcStages = PA_TC_STAGES;        // K and V rings, 16 KB per slot each
+static_assert(kTcStages >= 2 && kTcStages <= 5, "Q and both rings fit 227 KB");
+constexpr int kTcSoftmaxWarps = 8;             // two per TMEM lane quadrant
+constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;  // + K loads, MMA, V loads
+constexpr int kTcKWarp = kTcSoftmaxWarps;
+constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
+constexpr int kTcVWarp = kTcSoftmaxWarps + 2;
+constexpr uint32_t kTcTmemCols = 256;          // S (then P): 2 x 64 columns, O: 128 columns
+constexpr uint32_t kTcTmemO = 128;             // first column of O
+constexpr int kTcQBytes = 2 * kTcRows * 128;   // [2 halves of D][128 rows][128 B]
+constexpr int kTcTileBytes = 2 * kTcKv * 128;  // K or V of a stage: [2 halves][64 rows][128 B]
+constexpr float kTcRescaleLog2 = 8.f;          // reference max moves beyond 2^8
 
 struct TcPrefillParams {
   CUtensorMap tmk;
@@ -1691,8 +1703,8 @@ struct TcPrefillParams {
 };
 
 constexpr size_t tc_prefill_smem_bytes() {
-  return 1024 + size_t(kTcQBytes) + size_t(kTcStages) * 2 * kTcKvBytes + 2 * kTcPBytes +
-         (2 * kTcStages + 6) * sizeof(uint64_t) + 16;
+  return 1024 + size_t(kTcQBytes) + 2 * size_t(kTcStages) * kTcTileBytes +
+         6 * kTcRows * sizeof(float) + (4 * kTcStages + 7) * sizeof(uint64_t) + 16;
 }
 
 template <typename CT, bool kSplitP>
@@ -1707,17 +1719,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* qs = smem;                                    // Q operand
-  uint8_t* kvs = qs + kTcQBytes;                         // stage s: K at s*2*KV, V after it
-  uint8_t* ps = kvs + kTcStages * 2 * kTcKvBytes;        // P operand (hi term)
-  uint8_t* ps_lo = ps + kTcPBytes;                       // P - hi, with kSplitP
-  uint64_t* kv_full = reinterpret_cast<uint64_t*>(ps + 2 * kTcPBytes);
-  uint64_t* kv_empty = kv_full + kTcStages;
-  uint64_t* s_full = kv_empty + kTcStages;               // [2]
-  uint64_t* o_full = s_full + 2;
-  uint64_t* p_ready = o_full + 1;
-  uint64_t* done = p_ready + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
+  uint8_t* qs = smem;                                   // Q operand
+  uint8_t* ksm = qs + kTcQBytes;                        // K ring
+  uint8_t* vsm = ksm + kTcStages * kTcTileBytes;        // V ring
+  float* xmax = reinterpret_cast<float*>(vsm + kTcStages * kTcTileBytes);  // [2][2 halves][128]
+  float* lsum = xmax + 4 * kTcRows;                     // [2 halves][128]
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(lsum + 2 * kTcRows);
+  uint64_t* kempty = kfull + kTcStages;
+  uint64_t* vfull = kempty + kTcStages;
+  uint64_t* vempty = vfull + kTcStages;
+  uint64_t* s_full = vempty + kTcStages;  // [2]: S of stage jb (buffer jb & 1) written
+  uint64_t* o_full = s_full + 2;          // [2]: P.V of stage jb done
+  uint64_t* p_ready = o_full + 2;         // [2]: P of stage jb in TMEM, O rescaled
+  uint64_t* done = p_ready + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seq = blockIdx.x / pp.row_blocks;
@@ -1742,40 +1757,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (tid == 0) {
     for (int st = 0; st < kTcStages; ++st) {
-      mbar_init(&kv_full[st], 1);
-      mbar_init(&kv_empty[st], 1);
+      mbar_init(&kfull[st], 1);
+      mbar_init(&kempty[st], 1);
+      mbar_init(&vfull[st], 1);
+      mbar_init(&vempty[st], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(o_full, 1);
-    mbar_init(p_ready, kTcSoftmaxWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&p_ready[b], kTcSoftmaxWarps);
+    }
     mbar_init(done, 1);
     fence_barrier_init();
   }
-  if (warp == kTcSoftmaxWarps + 1) {  // the MMA warp owns the TMEM allocation
+  if (warp == kTcMmaWarp) {  // the MMA warp owns the TMEM allocation
     tmem_alloc(tmem_slot, kTcTmemCols);
     tmem_relinquish();
   }
-  // Q rows into the swizzled K-major operand: row r, 16-byte chunk c of 16.
+  // Q into the swizzled K-major operand: thread (half h, row r) moves 8 chunks.
   if (warp < kTcSoftmaxWarps) {
-    const int r = tid;
+    const int r = tid & (kTcRows - 1), h = tid >> 7;
     const int gr = row0 + r;
     const bool valid = gr < rows;
     const uint4* src = reinterpret_cast<const uint4*>(
         p.query + (int64_t(q0 + (valid ? gr / G : 0)) * p.num_heads + kvh * G +
-                   (valid ? gr % G : 0)) * D * 2);
+                   (valid ? gr % G : 0)) * D * 2) + 8 * h;
     // a negative scale is applied as |scale| to -Q (a sign flip is exact), so the
     // softmax may take the row max before scaling
     const uint32_t flip = p.q_mult < 0.f ? 0x80008000u : 0u;
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 0; c < 8; ++c) {
       uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
       v.x ^= flip;
       v.y ^= flip;
       v.z ^= flip;
       v.w ^= flip;
-      *reinterpret_cast<uint4*>(qs + (c >> 3) * (kTcRows * 128) + r * 128 +
-                                (((c & 7) ^ (r & 7)) << 4)) = v;
+      *reinterpret_cast<uint4*>(qs + h * (kTcRows * 128) + r * 128 + ((c ^ (r & 7)) << 4)) = v;
     }
     fence_proxy_async_smem();
   }
@@ -1784,8 +1801,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tcgen05_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kTcSoftmaxWarps) {
-    // ---------------- TMA producer: stage jb = sequence tiles 4jb .. 4jb+3 ----------------
+  if (warp == kTcKWarp || warp == kTcVWarp) {
+    // ---------------- TMA producers: stage jb = sequence tiles 4jb .. 4jb+3 ----------------
+    // one warp fills the K ring, the other the V ring, each at its own pace
+    const bool is_k = warp == kTcKWarp;
+    const CUtensorMap* map = is_k ? &pp.tmk : &pp.tmv;
+    uint8_t* ring = is_k ? ksm : vsm;
+    uint64_t* full = is_k ? kfull : vfull;
+    uint64_t* empty = is_k ? kempty : vempty;
     const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
     const uint64_t policy = l2_policy_evict_last();  // other row blocks read it again
     int issued = 0;
@@ -1798,7 +1821,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int t = 4 * jb + lane, e = t / p.tiles_per_block;
         int32_t phys = table_row[e];
         if (phys < 0 || phys >= p.num_blocks) {
-          atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
+          if (is_k) atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
           phys = 0;
         }
         tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
@@ -1807,259 +1830,241 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int t = 0; t < 4; ++t) tls[t] = __shfl_sync(kFullMask, tile, t);
       if (lane == 0) {
-        if (jb >= kTcStages && !mbar_wait_bounded(&kv_empty[stage], ((jb / kTcStages) - 1) & 1)) {
+        if (jb >= kTcStages && !mbar_wait_bounded(&empty[stage], ((jb / kTcStages) - 1) & 1)) {
           atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
           ok = false;
         }
         if (ok) {
-          uint8_t* kd = kvs + stage * 2 * kTcKvBytes;
-          uint8_t* vd = kd + kTcKvBytes;
-          mbar_arrive_expect_tx(&kv_full[stage], uint32_t(ntl) * 4 * 2048);
+          uint8_t* dst = ring + stage * kTcTileBytes;
+          mbar_arrive_expect_tx(&full[stage], uint32_t(ntl) * 2 * 2048);
           for (int t = 0; t < ntl; ++t) {
             const int row = tls[t] * kBlockSize;
-            tma_load_2d(kd + t * 2048, &pp.tmk, 0, row, &kv_full[stage], policy);
-            tma_load_2d(kd + kTcKvBytes / 2 + t * 2048, &pp.tmk, 64, row, &kv_full[stage], policy);
-            tma_load_2d(vd + t * 2048, &pp.tmv, 0, row, &kv_full[stage], policy);
-            tma_load_2d(vd + kTcKvBytes / 2 + t * 2048, &pp.tmv, 64, row, &kv_full[stage], policy);
+            tma_load_2d(dst + t * 2048, map, 0, row, &full[stage], policy);
+            tma_load_2d(dst + kTcTileBytes / 2 + t * 2048, map, 64, row, &full[stage], policy);
           }
           ++issued;
         }
       }
       ok = __shfl_sync(kFullMask, ok, 0);
     }
-    if (lane == 0) {
-      const int first = issued > kTcStages ? issued - kTcStages : 0;
-      for (int i = first; i < issued; ++i)
-        if (!mbar_wait_bounded(&kv_full[i % kTcStages], (i / kTcStages) & 1))
+    if (lane == 0) {  // no copy may still be landing when the CTA exits (one ring)
+      for (int i = max(0, issued - kTcStages); i < issued; ++i)
+        if (!mbar_wait_bounded(&full[i % kTcStages], (i / kTcStages) & 1))
           atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
     }
-  } else if (warp == kTcSoftmaxWarps + 1) {
-    // ---------------- MMA issuer (one thread) ----------------
+  } else if (warp == kTcMmaWarp) {
+    // ---------------- MMA issuer (one thread, polling) ----------------
     if (lane == 0) {
-      const uint32_t qaddr = smem_u32(qs);
-      const uint32_t paddr = smem_u32(ps);
-      auto issue_s = [&](int jb) {  // S[jb % 2] = Q . K(stage of jb)^T
-        const uint32_t kaddr = smem_u32(kvs + (jb % kTcStages) * 2 * kTcKvBytes);
-        const uint32_t d = tmem + uint32_t(jb & 1) * kTcKv;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t a = umma_smem_desc(qaddr + (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32,
-                                            16, 1024, kUmmaSwizzle128B);
-          const uint64_t b = umma_smem_desc(kaddr + (ks >> 2) * (kTcKvBytes / 2) + (ks & 3) * 32,
-                                            16, 1024, kUmmaSwizzle128B);
-          umma_f16_ss(d, a, b, kIdescS, ks > 0);
-        }
-        umma_commit(&s_full[jb & 1]);
-      };
-      auto issue_pv = [&](int jb) {  // O_blk = P . V(stage of jb)
-        const uint32_t vaddr = smem_u32(kvs + (jb % kTcStages) * 2 * kTcKvBytes + kTcKvBytes);
-#pragma unroll
-        for (int ks = 0; ks < kTcKv / 16; ++ks) {
-          const uint64_t a = umma_smem_desc(paddr + ks * 32, 16, 1024, kUmmaSwizzle128B);
-          const uint64_t b =
-              umma_smem_desc(vaddr + ks * 2048, kTcKvBytes / 2, 1024, kUmmaSwizzle128B);
-          umma_f16_ss(tmem + 128, a, b, kIdescPV, ks > 0);
-        }
-        if constexpr (kSplitP) {
-#pragma unroll
-          for (int ks = 0; ks < kTcKv / 16; ++ks) {
-            const uint64_t a =
-                umma_smem_desc(paddr + kTcPBytes + ks * 32, 16, 1024, kUmmaSwizzle128B);
-            const uint64_t b =
-                umma_smem_desc(vaddr + ks * 2048, kTcKvBytes / 2, 1024, kUmmaSwizzle128B);
-            umma_f16_ss(tmem + 128, a, b, kIdescPV, 1u);
-          }
-        }
-        umma_commit(o_full);
-        umma_commit(&kv_empty[jb % kTcStages]);
-      };
-      bool ok = mbar_wait_bounded(&kv_full[0], 0);
-      if (ok) {
-        tcgen05_fence_after();
-        issue_s(0);
-      }
-      for (int jb = 0; jb < nkb && ok; ++jb) {
-        if (jb + 1 < nkb) {
-          ok = mbar_wait_bounded(&kv_full[(jb + 1) % kTcStages], ((jb + 1) / kTcStages) & 1);
-          if (!ok) break;
+      const uint32_t qaddr = smem_u32(qs), kaddr0 = smem_u32(ksm), vaddr0 = smem_u32(vsm);
+      int ns = 0, npv = 0, idle = 0;
+      unsigned long long t_idle = 0;
+      bool ok = true;
+      while (npv < nkb) {
+        bool prog = false;
+        // S(ns) into buffer ns & 1, whose P(ns - 2) went to P.V(ns - 2) already
+        if (ns < nkb && ns <= npv + 1 && mbar_test(&kfull[ns % kTcStages], (ns / kTcStages) & 1)) {
           tcgen05_fence_after();
-          issue_s(jb + 1);
+          const uint32_t kaddr = kaddr0 + uint32_t((ns % kTcStages) * kTcTileBytes);
+          const uint32_t d = tmem + uint32_t(ns & 1) * kTcKv;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t a = umma_smem_desc(qaddr + (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32,
+                                              16, 1024, kUmmaSwizzle128B);
+            const uint64_t b = umma_smem_desc(kaddr + (ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32,
+                                              16, 1024, kUmmaSwizzle128B);
+            umma_f16_ss(d, a, b, kIdescS, ks > 0);
+          }
+          umma_commit(&s_full[ns & 1]);
+          umma_commit(&kempty[ns % kTcStages]);
+          ++ns;
+          prog = true;
         }
-        ok = mbar_wait_bounded(p_ready, jb & 1);
-        if (!ok) break;
-        tcgen05_fence_after();
-        issue_pv(jb);
+        // P.V(npv): P from TMEM over S buffer npv & 1, V from its ring slot
+        if (npv < ns && mbar_test(&p_ready[npv & 1], (npv >> 1) & 1) &&
+            mbar_test(&vfull[npv % kTcStages], (npv / kTcStages) & 1)) {
+          tcgen05_fence_after();
+          const uint32_t vaddr = vaddr0 + uint32_t((npv % kTcStages) * kTcTileBytes);
+          const uint32_t pt = tmem + uint32_t(npv & 1) * kTcKv;
+#pragma unroll
+          for (int t = 0; t < (kSplitP ? 2 : 1); ++t) {
+#pragma unroll
+            for (int ks = 0; ks < kTcKv / 16; ++ks) {
+              const uint64_t b =
+                  umma_smem_desc(vaddr + ks * 2048, kTcTileBytes / 2, 1024, kUmmaSwizzle128B);
+              umma_f16_ts(tmem + kTcTmemO, pt + uint32_t(t * 32 + ks * 8), b, kIdescPV,
+                          (npv > 0 || t > 0 || ks > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&o_full[npv & 1]);
+          umma_commit(&vempty[npv % kTcStages]);
+          ++npv;
+          prog = true;
+        }
+        if (prog) {
+          idle = 0;
+          continue;
+        }
+        if (idle == 0) t_idle = global_timer_ns();
+        if ((++idle & 63) == 0 && global_timer_ns() - t_idle > kWaitLimitNs) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
       umma_commit(done);  // fires once every MMA issued above has completed
     }
     __syncwarp();
   } else {
-    // ---------------- softmax warps: thread = row ----------------
-    const int r = tid;  // TMEM lane and Q row
+    // ---------------- softmax warps: thread = (row, column half) ----------------
+    const int h = warp >> 2, qd = warp & 3;
+    const int r = 32 * qd + lane;  // TMEM lane and Q row
     const int gr = row0 + r;
     const bool valid = gr < rows;
     const int pos = valid ? L - nq + gr / G : -1;
-    const uint32_t tl = tmem + (uint32_t(32 * warp) << 16);  // this warp's lane quadrant
+    const uint32_t tl = tmem + (uint32_t(32 * qd) << 16);  // this warp's lane quadrant
+    const uint32_t pair_bar = 1 + qd;                       // this warp and warp qd + 4*(1-h)
     const float mult = fabsf(p.q_mult);  // Q carries the sign
-    float o[128];
-#pragma unroll
-    for (int d = 0; d < 128; ++d) o[d] = 0.f;
-    float m = -INFINITY, l = 0.f, alpha_pend = 1.f;
-    bool ok = true;
+    float m = -INFINITY, l = 0.f;        // reference max (exp2 domain), sum of this half
+    bool ok = true;                      // warp-uniform; after a failure waits are skipped,
+                                         // but every named barrier is still reached
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
+    };
     for (int jb = 0; jb < nkb; ++jb) {
-      if (!__all_sync(kFullMask, mbar_wait_bounded(&s_full[jb & 1], (jb >> 1) & 1))) {
-        ok = false;
-        break;
-      }
+      const uint32_t sb = tl + uint32_t(jb & 1) * kTcKv;  // S, then P, of this stage
+      wait(&s_full[jb & 1], (jb >> 1) & 1);
       tcgen05_fence_after();
-      float sv[64];
-      {
-        float a[32], b[32];
-        tmem_ld32(tl + uint32_t(jb & 1) * kTcKv, a);
-        tmem_ld32(tl + uint32_t(jb & 1) * kTcKv + 32, b);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = a[i];
-          sv[32 + i] = b[i];
-        }
-      }
+      float sv[32];
+      tmem_ld32(sb + 32 * h, sv);
+      tmem_wait_ld();
       // causal, context and padding mask: only stages that cross this row's last
       // visible position pay for it
-      const int nvis = pos - jb * kTcKv + 1;
+      const int nvis = pos - jb * kTcKv - 32 * h + 1;
       float me = mult;  // multiplier still to apply to sv
-      if (nvis < kTcKv) {
+      if (nvis < 32) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) sv[i] = i < nvis ? sv[i] * mult : -INFINITY;
+        for (int i = 0; i < 32; ++i) sv[i] = i < nvis ? sv[i] * mult : -INFINITY;
         me = 1.f;
       }
-      // row max and sum over 8 independent chains (one row per thread: no shuffles)
-      float r8[8];
+      float r4[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) r8[k] = sv[k];
+      for (int k = 0; k < 4; ++k) r4[k] = sv[k];
 #pragma unroll
-      for (int i = 8; i < 64; ++i) r8[i & 7] = fmaxf(r8[i & 7], sv[i]);
-      const float mx = fmaxf(fmaxf(fmaxf(r8[0], r8[1]), fmaxf(r8[2], r8[3])),
-                             fmaxf(fmaxf(r8[4], r8[5]), fmaxf(r8[6], r8[7])));
-      const float mn = fmaxf(m, mx * me);  // scores scaled into the exp2 domain
-      const float mu = mn == -INFINITY ? 0.f : mn;
-      const float alpha = ex2_approx(m - mu);  // 0 while nothing was visible
+      for (int i = 4; i < 32; ++i) r4[i & 3] = fmaxf(r4[i & 3], sv[i]);
+      const float pmax = fmaxf(fmaxf(r4[0], r4[1]), fmaxf(r4[2], r4[3])) * me;
+      float* xm = xmax + (jb & 1) * 2 * kTcRows;
+      xm[h * kTcRows + r] = pmax;
+      named_bar_sync(pair_bar, 64);  // both halves have read S and posted their max
+      const float mx = fmaxf(pmax, xm[(1 - h) * kTcRows + r]);
+      if (jb == 0) {
+        m = mx;  // O is written, not accumulated, by the first P.V
+      } else {
+        const bool move = mx > m + kTcRescaleLog2;
+        if (__any_sync(kFullMask, move)) {
+          // rescale this warp's rows and columns of O once P.V(jb - 1) has landed
+          wait(&o_full[(jb - 1) & 1], ((jb - 1) >> 1) & 1);
+          tcgen05_fence_after();
+          const float f = move ? ex2_approx(m - mx) : 1.f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) r8[k] = 0.f;
+          for (int q = 0; q < 2; ++q) {
+            float v[32];
+            tmem_ld32(tl + kTcTmemO + 64 * h + 32 * q, v);
+            tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
+            for (int i = 0; i < 32; ++i) v[i] *= f;
+            tmem_st32(tl + kTcTmemO + 64 * h + 32 * q, v);
+          }
+          l *= f;
+          if (move) m = mx;
+        }
+      }
+      const float mu = m == -INFINITY ? 0.f : m;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) r4[k] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
         sv[i] = ex2_approx(fmaf(sv[i], me, -mu));
-        r8[i & 7] += sv[i];
+        r4[i & 3] += sv[i];
       }
-      const float sum = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-      m = mn;
-      l = l * alpha + sum;
-      // P(jb) may overwrite the P operand once P.V(jb - 1) has completed
-      if (jb > 0) {
-        if (!__all_sync(kFullMask, mbar_wait_bounded(o_full, (jb - 1) & 1))) {
-          ok = false;
-          break;
-        }
-        tcgen05_fence_after();
-      }
+      l += (r4[0] + r4[1]) + (r4[2] + r4[3]);
+      // P over the S columns both halves have read: this half's tokens 32h..32h+31
+      // as 16 columns of 16-bit pairs (the lo term 32 columns further on)
+      uint32_t pw[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 w;
-        w.x = pack2(sv[8 * c + 0], sv[8 * c + 1], CT{});
-        w.y = pack2(sv[8 * c + 2], sv[8 * c + 3], CT{});
-        w.z = pack2(sv[8 * c + 4], sv[8 * c + 5], CT{});
-        w.w = pack2(sv[8 * c + 6], sv[8 * c + 7], CT{});
-        *reinterpret_cast<uint4*>(ps + r * 128 + ((c ^ (r & 7)) << 4)) = w;
-        if constexpr (kSplitP) {
-          const float2 h0 = unpack2(w.x, CT{}), h1 = unpack2(w.y, CT{}), h2 = unpack2(w.z, CT{}),
-                       h3 = unpack2(w.w, CT{});
-          uint4 lo;
-          lo.x = pack2(sv[8 * c + 0] - h0.x, sv[8 * c + 1] - h0.y, CT{});
-          lo.y = pack2(sv[8 * c + 2] - h1.x, sv[8 * c + 3] - h1.y, CT{});
-          lo.z = pack2(sv[8 * c + 4] - h2.x, sv[8 * c + 5] - h2.y, CT{});
-          lo.w = pack2(sv[8 * c + 6] - h3.x, sv[8 * c + 7] - h3.y, CT{});
-          *reinterpret_cast<uint4*>(ps_lo + r * 128 + ((c ^ (r & 7)) << 4)) = lo;
+      for (int c = 0; c < 16; ++c) pw[c] = pack2(sv[2 * c], sv[2 * c + 1], CT{});
+      tmem_st16(sb + 16 * h, pw);
+      if constexpr (kSplitP) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float2 hi = unpack2(pw[c], CT{});
+          pw[c] = pack2(sv[2 * c] - hi.x, sv[2 * c + 1] - hi.y, CT{});
         }
+        tmem_st16(sb + 32 + 16 * h, pw);
       }
-      if (jb == nkb - 1) {
+      if (jb == nkb - 1 && h == 0) {
         // V rows past the last visible token may be stale or NaN: zero them
-        if (!__all_sync(kFullMask, mbar_wait_bounded(&kv_full[jb % kTcStages], (jb / kTcStages) & 1))) {
-          ok = false;
-          break;
-        }
+        wait(&vfull[jb % kTcStages], (jb / kTcStages) & 1);
         const int vr = r >> 1, half = r & 1;
-        if (jb * kTcKv + vr > pos_last) {
-          uint8_t* vrow = kvs + (jb % kTcStages) * 2 * kTcKvBytes + kTcKvBytes +
-                          half * (kTcKvBytes / 2) + vr * 128;
+        if (ok && jb * kTcKv + vr > pos_last) {
+          uint8_t* vrow = vsm + (jb % kTcStages) * kTcTileBytes + half * (kTcTileBytes / 2) +
+                          vr * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
-      // fold O_blk(jb - 1) in before P.V(jb) may overwrite it
-      if (jb > 0) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float v[32];
-          tmem_ld32(tl + 128 + 32 * q, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[32 * q + i] = fmaf(o[32 * q + i], alpha_pend, v[i]);
-        }
-      }
-      alpha_pend = alpha;
+      tmem_wait_st();
       tcgen05_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready);
+      if (lane == 0) mbar_arrive(&p_ready[jb & 1]);
     }
-    if (ok && __all_sync(kFullMask, mbar_wait_bounded(o_full, (nkb - 1) & 1))) {
-      tcgen05_fence_after();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float v[32];
-        tmem_ld32(tl + 128 + 32 * q, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[32 * q + i] = fmaf(o[32 * q + i], alpha_pend, v[i]);
-      }
-    } else {
-      ok = false;
-    }
+    wait(&o_full[(nkb - 1) & 1], ((nkb - 1) >> 1) & 1);
+    lsum[h * kTcRows + r] = l;
+    named_bar_sync(pair_bar, 64);
+    const float lt = l + lsum[(1 - h) * kTcRows + r];
     if (!ok && lane == 0) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
-    tcgen05_fence_before();
-    if (valid && ok) {
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+    if (ok) {
+      tcgen05_fence_after();
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
       uint8_t* dst = static_cast<uint8_t*>(p.out);
-      const int64_t orow = (int64_t(q0 + gr / G) * p.num_heads + kvh * G + gr % G) * D;
-      if (p.out_dtype == PA_F32) {
+      const int64_t orow = (int64_t(q0 + (valid ? gr / G : 0)) * p.num_heads + kvh * G +
+                            (valid ? gr % G : 0)) * D + 64 * h;
 #pragma unroll
-        for (int d = 0; d < 128; d += 4)
-          *reinterpret_cast<float4*>(dst + (orow + d) * 4) =
-              make_float4(o[d] * inv, o[d + 1] * inv, o[d + 2] * inv, o[d + 3] * inv);
-      } else {
+      for (int q = 0; q < 2; ++q) {
+        float v[32];
+        tmem_ld32(tl + kTcTmemO + 64 * h + 32 * q, v);
+        tmem_wait_ld();
+        if (!valid) continue;
+        if (p.out_dtype == PA_F32) {
 #pragma unroll
-        for (int d = 0; d < 128; d += 8) {
-          uint4 w;
-          if (p.out_dtype == PA_F16) {
-            w = make_uint4(pack2(o[d] * inv, o[d + 1] * inv, __half{}),
-                           pack2(o[d + 2] * inv, o[d + 3] * inv, __half{}),
-                           pack2(o[d + 4] * inv, o[d + 5] * inv, __half{}),
-                           pack2(o[d + 6] * inv, o[d + 7] * inv, __half{}));
-          } else {
-            w = make_uint4(pack2(o[d] * inv, o[d + 1] * inv, __nv_bfloat16{}),
-                           pack2(o[d + 2] * inv, o[d + 3] * inv, __nv_bfloat16{}),
-                           pack2(o[d + 4] * inv, o[d + 5] * inv, __nv_bfloat16{}),
-                           pack2(o[d + 6] * inv, o[d + 7] * inv, __nv_bfloat16{}));
-          }
-          *reinterpret_cast<uint4*>(dst + (orow + d) * 2) = w;
+          for (int d = 0; d < 32; d += 4)
+            *reinterpret_cast<float4*>(dst + (orow + 32 * q + d) * 4) =
+                make_float4(v[d] * inv, v[d + 1] * inv, v[d + 2] * inv, v[d + 3] * inv);
+        } else if (p.out_dtype == PA_F16) {
+#pragma unroll
+          for (int d = 0; d < 32; d += 8)
+            *reinterpret_cast<uint4*>(dst + (orow + 32 * q + d) * 2) =
+                make_uint4(pack2(v[d] * inv, v[d + 1] * inv, __half{}),
+                           pack2(v[d + 2] * inv, v[d + 3] * inv, __half{}),
+                           pack2(v[d + 4] * inv, v[d + 5] * inv, __half{}),
+                           pack2(v[d + 6] * inv, v[d + 7] * inv, __half{}));
+        } else {
+#pragma unroll
+          for (int d = 0; d < 32; d += 8)
+            *reinterpret_cast<uint4*>(dst + (orow + 32 * q + d) * 2) =
+                make_uint4(pack2(v[d] * inv, v[d + 1] * inv, __nv_bfloat16{}),
+                           pack2(v[d + 2] * inv, v[d + 3] * inv, __nv_bfloat16{}),
+                           pack2(v[d + 4] * inv, v[d + 5] * inv, __nv_bfloat16{}),
+                           pack2(v[d + 6] * inv, v[d + 7] * inv, __nv_bfloat16{}));
         }
       }
     }
+    tcgen05_fence_before();
   }
-  // Free TMEM only after every MMA has completed and every TMEM read is done.
+  // Free TMEM only after every MMA has completed and every TMEM access is done.
   __syncthreads();
-  if (warp == kTcSoftmaxWarps + 1) {
+  if (warp == kTcMmaWarp) {
     if (!__all_sync(kFullMask, mbar_wait_bounded(done, 0)) && lane == 0)
       atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
     tcgen05_fence_after();
