@@ -1656,11 +1656,12 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
 // contraction is large enough for the CTA-wide MMA: one CTA holds 128 rows (one
 // TMEM lane each) and walks the sequence's KV in stages of 64 tokens (four
 // 16-token tiles placed by TMA as one 128-byte-swizzled operand):
-//   S[128 x 64]   = Q[128 x 128] . K^T   A = Q, B = K from shared memory; fp32 S in
-//                                        TMEM, two buffers
+//   S[128 x 64]   = Q[128 x 128] . K^T   A = Q from TMEM (written once), B = K from
+//                                        shared memory; fp32 S in TMEM, two buffers
 //   O[128 x 128] += P[128 x 64] . V      A = P from TMEM (written over its own S),
 //                                        B = V from shared memory (MN-major); O
 //                                        stays in TMEM for the whole pass
+// Both MMAs take A from tensor memory, so shared memory feeds only K and V.
 // K and V have rings and producer warps of their own, so a K slot refills as
 // soon as its S is done and a V slot as soon as its P.V is done.  Eight softmax warps, two per TMEM lane quadrant,
 // each take 32 rows x 32 of the 64 columns (the row max of the two halves meets in
@@ -1682,17 +1683,18 @@ constexpr int kTcKv = 64;                      // tokens per KV stage
 #define PA_TC_STAGES 4
 #endif
 constexpr int kTcStages = PA_TC_STAGES;        // K and V rings, 16 KB per slot each
-static_assert(kTcStages >= 2 && kTcStages <= 5, "Q and both rings fit 227 KB");
+static_assert(kTcStages >= 2 && kTcStages <= 6, "both rings fit 227 KB");
 constexpr int kTcSoftmaxWarps = 8;             // two per TMEM lane quadrant
 constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;  // + K loads, MMA, V loads
 constexpr int kTcKWarp = kTcSoftmaxWarps;
 constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
 constexpr int kTcVWarp = kTcSoftmaxWarps + 2;
-constexpr uint32_t kTcTmemCols = 256;          // S (then P): 2 x 64 columns, O: 128 columns
+constexpr uint32_t kTcTmemCols = 512;          // S (then P): 2 x 64, O: 128, Q: 64 columns
 constexpr uint32_t kTcTmemO = 128;             // first column of O
-constexpr int kTcQBytes = 2 * kTcRows * 128;   // [2 halves of D][128 rows][128 B]
+constexpr uint32_t kTcTmemQ = 256;             // first column of Q (16-bit pairs)
 constexpr int kTcTileBytes = 2 * kTcKv * 128;  // K or V of a stage: [2 halves][64 rows][128 B]
 constexpr float kTcRescaleLog2 = 8.f;          // reference max moves beyond 2^8
+constexpr uint32_t kTcPollNs = 500;            // MMA issuer's longest sleep per poll
 
 struct TcPrefillParams {
   CUtensorMap tmk;
@@ -1703,7 +1705,7 @@ struct TcPrefillParams {
 };
 
 constexpr size_t tc_prefill_smem_bytes() {
-  return 1024 + size_t(kTcQBytes) + 2 * size_t(kTcStages) * kTcTileBytes +
+  return 1024 + 2 * size_t(kTcStages) * kTcTileBytes +
          6 * kTcRows * sizeof(float) + (4 * kTcStages + 7) * sizeof(uint64_t) + 16;
 }
 
@@ -1719,8 +1721,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* qs = smem;                                   // Q operand
-  uint8_t* ksm = qs + kTcQBytes;                        // K ring
+  uint8_t* ksm = smem;                                  // K ring
   uint8_t* vsm = ksm + kTcStages * kTcTileBytes;        // V ring
   float* xmax = reinterpret_cast<float*>(vsm + kTcStages * kTcTileBytes);  // [2][2 halves][128]
   float* lsum = xmax + 4 * kTcRows;                     // [2 halves][128]
@@ -1774,9 +1775,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(tmem_slot, kTcTmemCols);
     tmem_relinquish();
   }
-  // Q into the swizzled K-major operand: thread (half h, row r) moves 8 chunks.
+  tcgen05_fence_before();
+  __syncthreads();
+  tcgen05_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // Q rows into TMEM as the A operand of S: thread (half h, row r) stores d in
+  // [64h, 64h + 64) as 32 columns of 16-bit pairs.
   if (warp < kTcSoftmaxWarps) {
-    const int r = tid & (kTcRows - 1), h = tid >> 7;
+    const int r = 32 * (warp & 3) + lane, h = warp >> 2;
     const int gr = row0 + r;
     const bool valid = gr < rows;
     const uint4* src = reinterpret_cast<const uint4*>(
@@ -1785,21 +1791,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // a negative scale is applied as |scale| to -Q (a sign flip is exact), so the
     // softmax may take the row max before scaling
     const uint32_t flip = p.q_mult < 0.f ? 0x80008000u : 0u;
+    float qv[32];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-      v.x ^= flip;
-      v.y ^= flip;
-      v.z ^= flip;
-      v.w ^= flip;
-      *reinterpret_cast<uint4*>(qs + h * (kTcRows * 128) + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+      const uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      qv[4 * c + 0] = __uint_as_float(v.x ^ flip);
+      qv[4 * c + 1] = __uint_as_float(v.y ^ flip);
+      qv[4 * c + 2] = __uint_as_float(v.z ^ flip);
+      qv[4 * c + 3] = __uint_as_float(v.w ^ flip);
     }
-    fence_proxy_async_smem();
+    tmem_st32(tmem + (uint32_t(32 * (warp & 3)) << 16) + kTcTmemQ + 32 * h, qv);
+    tmem_wait_st();
   }
   tcgen05_fence_before();
   __syncthreads();
   tcgen05_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
   if (warp == kTcKWarp || warp == kTcVWarp) {
     // ---------------- TMA producers: stage jb = sequence tiles 4jb .. 4jb+3 ----------------
@@ -1812,23 +1818,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
     const uint64_t policy = l2_policy_evict_last();  // other row blocks read it again
     int issued = 0;
+    int ent = 0;  // this lane's pool tile of the current group of 8 stages (32 tiles)
     bool ok = true;
     for (int jb = 0; jb < nkb && ok; ++jb) {
       const int stage = jb % kTcStages;
       const int ntl = min(4, ntiles - 4 * jb);
-      int tile = 0;
-      if (lane < ntl) {
-        const int t = 4 * jb + lane, e = t / p.tiles_per_block;
-        int32_t phys = table_row[e];
-        if (phys < 0 || phys >= p.num_blocks) {
-          if (is_k) atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
-          phys = 0;
+      if ((jb & 7) == 0) {  // one table read per lane covers the next 8 stages
+        const int t = 4 * jb + lane;
+        ent = 0;
+        if (t < ntiles) {
+          const int e = t / p.tiles_per_block;
+          int32_t phys = table_row[e];
+          if (phys < 0 || phys >= p.num_blocks) {
+            if (is_k) atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
+            phys = 0;
+          }
+          ent = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
         }
-        tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
       }
       int tls[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) tls[t] = __shfl_sync(kFullMask, tile, t);
+      for (int t = 0; t < 4; ++t) tls[t] = __shfl_sync(kFullMask, ent, 4 * (jb & 7) + t);
       if (lane == 0) {
         if (jb >= kTcStages && !mbar_wait_bounded(&empty[stage], ((jb / kTcStages) - 1) & 1)) {
           atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
@@ -1855,7 +1865,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == kTcMmaWarp) {
     // ---------------- MMA issuer (one thread, polling) ----------------
     if (lane == 0) {
-      const uint32_t qaddr = smem_u32(qs), kaddr0 = smem_u32(ksm), vaddr0 = smem_u32(vsm);
+      // descriptors advance by a constant (byte offset >> 4) in the start-address field
+      const uint64_t kdesc0 = umma_smem_desc(smem_u32(ksm), 16, 1024, kUmmaSwizzle128B);
+      const uint64_t vdesc0 = umma_smem_desc(smem_u32(vsm), kTcTileBytes / 2, 1024,
+                                             kUmmaSwizzle128B);
       int ns = 0, npv = 0, idle = 0;
       unsigned long long t_idle = 0;
       bool ok = true;
@@ -1864,16 +1877,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // S(ns) into buffer ns & 1, whose P(ns - 2) went to P.V(ns - 2) already
         if (ns < nkb && ns <= npv + 1 && mbar_test(&kfull[ns % kTcStages], (ns / kTcStages) & 1)) {
           tcgen05_fence_after();
-          const uint32_t kaddr = kaddr0 + uint32_t((ns % kTcStages) * kTcTileBytes);
+          const uint64_t kd = kdesc0 + uint64_t(((ns % kTcStages) * kTcTileBytes) >> 4);
           const uint32_t d = tmem + uint32_t(ns & 1) * kTcKv;
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t a = umma_smem_desc(qaddr + (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32,
-                                              16, 1024, kUmmaSwizzle128B);
-            const uint64_t b = umma_smem_desc(kaddr + (ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32,
-                                              16, 1024, kUmmaSwizzle128B);
-            umma_f16_ss(d, a, b, kIdescS, ks > 0);
-          }
+          for (int ks = 0; ks < 8; ++ks)
+            umma_f16_ts(d, tmem + kTcTmemQ + uint32_t(8 * ks),
+                        kd + uint64_t(((ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32) >> 4),
+                        kIdescS, ks > 0 ? 1u : 0u);
           umma_commit(&s_full[ns & 1]);
           umma_commit(&kempty[ns % kTcStages]);
           ++ns;
@@ -1883,17 +1893,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (npv < ns && mbar_test(&p_ready[npv & 1], (npv >> 1) & 1) &&
             mbar_test(&vfull[npv % kTcStages], (npv / kTcStages) & 1)) {
           tcgen05_fence_after();
-          const uint32_t vaddr = vaddr0 + uint32_t((npv % kTcStages) * kTcTileBytes);
+          const uint64_t vd = vdesc0 + uint64_t(((npv % kTcStages) * kTcTileBytes) >> 4);
           const uint32_t pt = tmem + uint32_t(npv & 1) * kTcKv;
 #pragma unroll
           for (int t = 0; t < (kSplitP ? 2 : 1); ++t) {
 #pragma unroll
-            for (int ks = 0; ks < kTcKv / 16; ++ks) {
-              const uint64_t b =
-                  umma_smem_desc(vaddr + ks * 2048, kTcTileBytes / 2, 1024, kUmmaSwizzle128B);
-              umma_f16_ts(tmem + kTcTmemO, pt + uint32_t(t * 32 + ks * 8), b, kIdescPV,
+            for (int ks = 0; ks < kTcKv / 16; ++ks)
+              umma_f16_ts(tmem + kTcTmemO, pt + uint32_t(t * 32 + ks * 8),
+                          vd + uint64_t((ks * 2048) >> 4), kIdescPV,
                           (npv > 0 || t > 0 || ks > 0) ? 1u : 0u);
-            }
           }
           umma_commit(&o_full[npv & 1]);
           umma_commit(&vempty[npv % kTcStages]);
@@ -1904,6 +1912,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           idle = 0;
           continue;
         }
+        // sleep (no issue slots taken from the softmax warps) on the barrier the
+        // next step most likely waits for: P of the oldest stage once its S is out
+        if (npv < ns)
+          mbar_try_wait(&p_ready[npv & 1], (npv >> 1) & 1, kTcPollNs);
+        else
+          mbar_try_wait(&kfull[ns % kTcStages], (ns / kTcStages) & 1, kTcPollNs);
         if (idle == 0) t_idle = global_timer_ns();
         if ((++idle & 63) == 0 && global_timer_ns() - t_idle > kWaitLimitNs) {
           ok = false;
