@@ -1678,21 +1678,27 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
 // a full-precision output.
 // ---------------------------------------------------------------------------
 constexpr int kTcRows = 128;                   // query rows per CTA = TMEM lanes
-constexpr int kTcKv = 64;                      // tokens per KV stage
-#ifndef PA_TC_STAGES
-#define PA_TC_STAGES 4
+#ifndef PA_TC_KV
+#define PA_TC_KV 128
 #endif
-constexpr int kTcStages = PA_TC_STAGES;        // K and V rings, 16 KB per slot each
-static_assert(kTcStages >= 2 && kTcStages <= 6, "both rings fit 227 KB");
+constexpr int kTcKv = PA_TC_KV;                // tokens per KV stage (N of the S MMA)
+static_assert(kTcKv == 64 || kTcKv == 128, "stage of 64 or 128 tokens");
+constexpr int kTcTiles = kTcKv / kBlockSize;   // 16-token pool tiles per stage
+constexpr int kTcHalf = kTcKv / 2;             // S columns per softmax warp
+#ifndef PA_TC_STAGES
+#define PA_TC_STAGES (PA_TC_KV == 128 ? 2 : 4)
+#endif
+constexpr int kTcStages = PA_TC_STAGES;        // K and V rings
 constexpr int kTcSoftmaxWarps = 8;             // two per TMEM lane quadrant
 constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;  // + K loads, MMA, V loads
 constexpr int kTcKWarp = kTcSoftmaxWarps;
 constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
 constexpr int kTcVWarp = kTcSoftmaxWarps + 2;
-constexpr uint32_t kTcTmemCols = 512;          // S (then P): 2 x 64, O: 128, Q: 64 columns
-constexpr uint32_t kTcTmemO = 128;             // first column of O
-constexpr uint32_t kTcTmemQ = 256;             // first column of Q (16-bit pairs)
-constexpr int kTcTileBytes = 2 * kTcKv * 128;  // K or V of a stage: [2 halves][64 rows][128 B]
+constexpr uint32_t kTcTmemCols = 512;          // S (then P): 2 x kTcKv, O: 128, Q: 64 columns
+constexpr uint32_t kTcTmemO = 2 * kTcKv;       // first column of O
+constexpr uint32_t kTcTmemQ = 2 * kTcKv + 128; // first column of Q (16-bit pairs)
+static_assert(kTcTmemQ + 64 <= kTcTmemCols, "TMEM budget");
+constexpr int kTcTileBytes = 2 * kTcKv * 128;  // K or V of a stage: [2 halves][kTcKv rows][128 B]
 constexpr float kTcRescaleLog2 = 8.f;          // reference max moves beyond 2^8
 constexpr uint32_t kTcPollNs = 500;            // MMA issuer's longest sleep per poll
 
@@ -1708,6 +1714,8 @@ constexpr size_t tc_prefill_smem_bytes() {
   return 1024 + 2 * size_t(kTcStages) * kTcTileBytes +
          6 * kTcRows * sizeof(float) + (4 * kTcStages + 7) * sizeof(uint64_t) + 16;
 }
+
+static_assert(kTcStages >= 2 && tc_prefill_smem_bytes() <= 227 * 1024, "rings fit 227 KB");
 
 template <typename CT, bool kSplitP>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -1818,13 +1826,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
     const uint64_t policy = l2_policy_evict_last();  // other row blocks read it again
     int issued = 0;
-    int ent = 0;  // this lane's pool tile of the current group of 8 stages (32 tiles)
+    constexpr int kPre = 32 / kTcTiles;  // stages covered by one table read per lane
+    int ent = 0;  // this lane's pool tile of the current group of 32 tiles
     bool ok = true;
     for (int jb = 0; jb < nkb && ok; ++jb) {
       const int stage = jb % kTcStages;
-      const int ntl = min(4, ntiles - 4 * jb);
-      if ((jb & 7) == 0) {  // one table read per lane covers the next 8 stages
-        const int t = 4 * jb + lane;
+      const int ntl = min(kTcTiles, ntiles - kTcTiles * jb);
+      if (jb % kPre == 0) {
+        const int t = kTcTiles * jb + lane;
         ent = 0;
         if (t < ntiles) {
           const int e = t / p.tiles_per_block;
@@ -1836,9 +1845,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ent = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
         }
       }
-      int tls[4];
+      int tls[kTcTiles];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) tls[t] = __shfl_sync(kFullMask, ent, 4 * (jb & 7) + t);
+      for (int t = 0; t < kTcTiles; ++t)
+        tls[t] = __shfl_sync(kFullMask, ent, kTcTiles * (jb % kPre) + t);
       if (lane == 0) {
         if (jb >= kTcStages && !mbar_wait_bounded(&empty[stage], ((jb / kTcStages) - 1) & 1)) {
           atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
@@ -1899,7 +1909,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int t = 0; t < (kSplitP ? 2 : 1); ++t) {
 #pragma unroll
             for (int ks = 0; ks < kTcKv / 16; ++ks)
-              umma_f16_ts(tmem + kTcTmemO, pt + uint32_t(t * 32 + ks * 8),
+              umma_f16_ts(tmem + kTcTmemO, pt + uint32_t(t * (kTcKv / 2) + ks * 8),
                           vd + uint64_t((ks * 2048) >> 4), kIdescPV,
                           (npv > 0 || t > 0 || ks > 0) ? 1u : 0u);
           }
@@ -1948,24 +1958,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t sb = tl + uint32_t(jb & 1) * kTcKv;  // S, then P, of this stage
       wait(&s_full[jb & 1], (jb >> 1) & 1);
       tcgen05_fence_after();
-      float sv[32];
-      tmem_ld32(sb + 32 * h, sv);
+      float sv[kTcHalf];
+#pragma unroll
+      for (int q = 0; q < kTcHalf / 32; ++q) {
+        float v[32];
+        tmem_ld32(sb + kTcHalf * h + 32 * q, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sv[32 * q + i] = v[i];
+      }
       tmem_wait_ld();
       // causal, context and padding mask: only stages that cross this row's last
       // visible position pay for it
-      const int nvis = pos - jb * kTcKv - 32 * h + 1;
+      const int nvis = pos - jb * kTcKv - kTcHalf * h + 1;
       float me = mult;  // multiplier still to apply to sv
-      if (nvis < 32) {
+      if (nvis < kTcHalf) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sv[i] = i < nvis ? sv[i] * mult : -INFINITY;
+        for (int i = 0; i < kTcHalf; ++i) sv[i] = i < nvis ? sv[i] * mult : -INFINITY;
         me = 1.f;
       }
-      float r4[4];
+      float r8[8];  // 8 independent chains
 #pragma unroll
-      for (int k = 0; k < 4; ++k) r4[k] = sv[k];
+      for (int k = 0; k < 8; ++k) r8[k] = sv[k];
 #pragma unroll
-      for (int i = 4; i < 32; ++i) r4[i & 3] = fmaxf(r4[i & 3], sv[i]);
-      const float pmax = fmaxf(fmaxf(r4[0], r4[1]), fmaxf(r4[2], r4[3])) * me;
+      for (int i = 8; i < kTcHalf; ++i) r8[i & 7] = fmaxf(r8[i & 7], sv[i]);
+      const float pmax = fmaxf(fmaxf(fmaxf(r8[0], r8[1]), fmaxf(r8[2], r8[3])),
+                               fmaxf(fmaxf(r8[4], r8[5]), fmaxf(r8[6], r8[7]))) * me;
       float* xm = xmax + (jb & 1) * 2 * kTcRows;
       xm[h * kTcRows + r] = pmax;
       named_bar_sync(pair_bar, 64);  // both halves have read S and posted their max
@@ -1994,31 +2011,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const float mu = m == -INFINITY ? 0.f : m;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) r4[k] = 0.f;
+      for (int k = 0; k < 8; ++k) r8[k] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < kTcHalf; ++i) {
         sv[i] = ex2_approx(fmaf(sv[i], me, -mu));
-        r4[i & 3] += sv[i];
+        r8[i & 7] += sv[i];
       }
-      l += (r4[0] + r4[1]) + (r4[2] + r4[3]);
-      // P over the S columns both halves have read: this half's tokens 32h..32h+31
-      // as 16 columns of 16-bit pairs (the lo term 32 columns further on)
-      uint32_t pw[16];
+      l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+      // P over the S columns both halves have read: this half's tokens as 16-bit
+      // pairs in columns [h * kTcHalf / 2, (h + 1) * kTcHalf / 2), the lo term
+      // kTcKv / 2 columns further on
 #pragma unroll
-      for (int c = 0; c < 16; ++c) pw[c] = pack2(sv[2 * c], sv[2 * c + 1], CT{});
-      tmem_st16(sb + 16 * h, pw);
-      if constexpr (kSplitP) {
+      for (int q = 0; q < kTcHalf / 32; ++q) {
+        uint32_t pw[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float2 hi = unpack2(pw[c], CT{});
-          pw[c] = pack2(sv[2 * c] - hi.x, sv[2 * c + 1] - hi.y, CT{});
+        for (int c = 0; c < 16; ++c)
+          pw[c] = pack2(sv[32 * q + 2 * c], sv[32 * q + 2 * c + 1], CT{});
+        tmem_st16(sb + (kTcHalf / 2) * h + 16 * q, pw);
+        if constexpr (kSplitP) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float2 hi = unpack2(pw[c], CT{});
+            pw[c] = pack2(sv[32 * q + 2 * c] - hi.x, sv[32 * q + 2 * c + 1] - hi.y, CT{});
+          }
+          tmem_st16(sb + kTcKv / 2 + (kTcHalf / 2) * h + 16 * q, pw);
         }
-        tmem_st16(sb + 32 + 16 * h, pw);
       }
-      if (jb == nkb - 1 && h == 0) {
+      if (jb == nkb - 1 && tid < 2 * kTcKv) {
         // V rows past the last visible token may be stale or NaN: zero them
         wait(&vfull[jb % kTcStages], (jb / kTcStages) & 1);
-        const int vr = r >> 1, half = r & 1;
+        const int vr = tid >> 1, half = tid & 1;
         if (ok && jb * kTcKv + vr > pos_last) {
           uint8_t* vrow = vsm + (jb % kTcStages) * kTcTileBytes + half * (kTcTileBytes / 2) +
                           vr * 128;
