@@ -1694,10 +1694,10 @@ constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;  // + K loads, MMA, V loa
 constexpr int kTcKWarp = kTcSoftmaxWarps;
 constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
 constexpr int kTcVWarp = kTcSoftmaxWarps + 2;
-constexpr uint32_t kTcTmemCols = 512;          // S (then P): 2 x kTcKv, O: 128, Q: 64 columns
+constexpr uint32_t kTcTmemCols = 512;          // S (then P): 2 x kTcKv, O: 128, Q: 2 x 64
 constexpr uint32_t kTcTmemO = 2 * kTcKv;       // first column of O
-constexpr uint32_t kTcTmemQ = 2 * kTcKv + 128; // first column of Q (16-bit pairs)
-static_assert(kTcTmemQ + 64 <= kTcTmemCols, "TMEM budget");
+constexpr uint32_t kTcTmemQ = 2 * kTcKv + 128; // Q slot b at kTcTmemQ + 64 b (16-bit pairs)
+static_assert(kTcTmemQ + 128 <= kTcTmemCols, "TMEM budget");
 constexpr int kTcTileBytes = 2 * kTcKv * 128;  // K or V of a stage: [2 halves][kTcKv rows][128 B]
 constexpr float kTcRescaleLog2 = 8.f;          // reference max moves beyond 2^8
 constexpr uint32_t kTcPollNs = 500;            // MMA issuer's longest sleep per poll
@@ -1707,15 +1707,102 @@ struct TcPrefillParams {
   CUtensorMap tmv;
   Params p;
   const int32_t* query_start;
-  int row_blocks;
+  int row_blocks;  // 128-row tiles per (sequence, kv head)
+  int num_tiles;   // num_seqs * num_kv_heads * row_blocks
 };
 
 constexpr size_t tc_prefill_smem_bytes() {
-  return 1024 + 2 * size_t(kTcStages) * kTcTileBytes +
-         6 * kTcRows * sizeof(float) + (4 * kTcStages + 7) * sizeof(uint64_t) + 16;
+  return 1024 + 2 * size_t(kTcStages) * kTcTileBytes + 6 * kTcRows * sizeof(float) +
+         (4 * kTcStages + 9) * sizeof(uint64_t) + 16;
 }
 
+// One 128-row tile: tile = (seq * num_kv_heads + kvh) * row_blocks + row block, so
+// consecutive tiles share a sequence's KV (read through L2).
+struct TcTile {
+  int seq, kvh, q0, nq, L, rows, row0, pos_last, ntiles, nkb;
+};
+
+__device__ __forceinline__ bool tc_tile(const TcPrefillParams& pp, int tile, TcTile& t,
+                                        bool report) {
+  const Params& p = pp.p;
+  const int per_seq = p.num_kv_heads * pp.row_blocks;
+  t.seq = tile / per_seq;
+  const int rem = tile - t.seq * per_seq;
+  t.kvh = rem / pp.row_blocks;
+  const int rblk = rem - t.kvh * pp.row_blocks;
+  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+  int L = p.seq_lens[t.seq];
+  t.q0 = pp.query_start[t.seq];
+  int nq = pp.query_start[t.seq + 1] - t.q0;
+  if (L < 0 || L > cap || nq < 0 || nq > L) {
+    if (report && rblk == 0 && t.kvh == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
+    L = L < 0 ? 0 : (L > cap ? cap : L);
+    nq = nq < 0 ? 0 : (nq > L ? L : nq);
+  }
+  t.L = L;
+  t.nq = nq;
+  t.rows = nq * p.group;
+  t.row0 = rblk * kTcRows;
+  if (t.row0 >= t.rows) return false;  // a short sequence's unused row block
+  t.pos_last = L - nq + (min(t.rows, t.row0 + kTcRows) - 1) / p.group;
+  t.ntiles = t.pos_last / kBlockSize + 1;
+  t.nkb = (t.pos_last + kTcKv) / kTcKv;
+  return true;
+}
+
+// The next non-empty tile of this CTA's round-robin share after `tile` (or the
+// first one when tile < 0); false when none is left.
+__device__ __forceinline__ bool tc_next_tile(const TcPrefillParams& pp, int& tile, TcTile& t,
+                                             bool report) {
+  for (tile = tile < 0 ? int(blockIdx.x) : tile + int(gridDim.x); tile < pp.num_tiles;
+       tile += gridDim.x)
+    if (tc_tile(pp, tile, t, report)) return true;
+  return false;
+}
+
+// A walk over this CTA's stages in order: (tile, stage within the tile), plus the
+// count of tiles begun (which selects the Q slot).
+struct TcCursor {
+  int tile = -1, jb = 0, nkb = 0, tcount = -1;
+  bool valid = false;
+  __device__ __forceinline__ void advance(const TcPrefillParams& pp) {
+    if (valid && ++jb < nkb) return;
+    TcTile t;
+    valid = tc_next_tile(pp, tile, t, false);
+    jb = 0;
+    nkb = valid ? t.nkb : 0;
+    ++tcount;
+  }
+};
+
 static_assert(kTcStages >= 2 && tc_prefill_smem_bytes() <= 227 * 1024, "rings fit 227 KB");
+
+// Q rows of a tile into TMEM slot `slot` as the A operand of S: thread (half h,
+// row r) stores d in [64h, 64h + 64) as 32 columns of 16-bit pairs.  A negative
+// scale is applied as |scale| to -Q (a sign flip is exact), so the softmax may
+// take the row max before scaling.
+__device__ __forceinline__ void tc_store_q(const Params& p, const TcTile& t, uint32_t tl,
+                                           uint32_t slot, int r, int h) {
+  constexpr int D = 128;
+  const int gr = t.row0 + r;
+  const bool valid = gr < t.rows;
+  const int G = p.group;
+  const uint4* src = reinterpret_cast<const uint4*>(
+      p.query + (int64_t(t.q0 + (valid ? gr / G : 0)) * p.num_heads + t.kvh * G +
+                 (valid ? gr % G : 0)) * D * 2) + 8 * h;
+  const uint32_t flip = p.q_mult < 0.f ? 0x80008000u : 0u;
+  float qv[32];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+    qv[4 * c + 0] = __uint_as_float(v.x ^ flip);
+    qv[4 * c + 1] = __uint_as_float(v.y ^ flip);
+    qv[4 * c + 2] = __uint_as_float(v.z ^ flip);
+    qv[4 * c + 3] = __uint_as_float(v.w ^ flip);
+  }
+  tmem_st32(tl + kTcTmemQ + 64 * slot + 32 * h, qv);
+  tmem_wait_st();
+}
 
 template <typename CT, bool kSplitP>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -1737,33 +1824,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* kempty = kfull + kTcStages;
   uint64_t* vfull = kempty + kTcStages;
   uint64_t* vempty = vfull + kTcStages;
-  uint64_t* s_full = vempty + kTcStages;  // [2]: S of stage jb (buffer jb & 1) written
-  uint64_t* o_full = s_full + 2;          // [2]: P.V of stage jb done
-  uint64_t* p_ready = o_full + 2;         // [2]: P of stage jb in TMEM, O rescaled
-  uint64_t* done = p_ready + 2;
+  uint64_t* s_full = vempty + kTcStages;  // [2]: S of stage g (buffer g & 1) written
+  uint64_t* o_full = s_full + 2;          // [2]: P.V of stage g done
+  uint64_t* p_ready = o_full + 2;         // [2]: P of stage g in TMEM, O rescaled
+  uint64_t* q_ready = p_ready + 2;        // [2]: Q of this CTA's tile number c in slot c & 1
+  uint64_t* done = q_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int seq = blockIdx.x / pp.row_blocks;
-  const int rblk = blockIdx.x - seq * pp.row_blocks;
-  const int kvh = blockIdx.y;
-  const int G = p.group;
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
-  int L = p.seq_lens[seq];
-  const int q0 = pp.query_start[seq];
-  int nq = pp.query_start[seq + 1] - q0;
-  if (L < 0 || L > cap || nq < 0 || nq > L) {
-    if (tid == 0 && rblk == 0 && kvh == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
-    L = L < 0 ? 0 : (L > cap ? cap : L);
-    nq = nq < 0 ? 0 : (nq > L ? L : nq);
-  }
-  const int rows = nq * G;
-  const int row0 = rblk * kTcRows;
-  if (row0 >= rows) return;  // uniform: before any barrier or TMEM allocation
-  const int pos_last = L - nq + (min(rows, row0 + kTcRows) - 1) / G;
-  const int ntiles = pos_last / kBlockSize + 1;
-  const int nkb = (pos_last + kTcKv) / kTcKv;  // KV stages to process
-
   if (tid == 0) {
     for (int st = 0; st < kTcStages; ++st) {
       mbar_init(&kfull[st], 1);
@@ -1775,6 +1843,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&s_full[b], 1);
       mbar_init(&o_full[b], 1);
       mbar_init(&p_ready[b], kTcSoftmaxWarps);
+      mbar_init(&q_ready[b], kTcSoftmaxWarps);
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -1787,88 +1856,67 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tcgen05_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Q rows into TMEM as the A operand of S: thread (half h, row r) stores d in
-  // [64h, 64h + 64) as 32 columns of 16-bit pairs.
-  if (warp < kTcSoftmaxWarps) {
-    const int r = 32 * (warp & 3) + lane, h = warp >> 2;
-    const int gr = row0 + r;
-    const bool valid = gr < rows;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        p.query + (int64_t(q0 + (valid ? gr / G : 0)) * p.num_heads + kvh * G +
-                   (valid ? gr % G : 0)) * D * 2) + 8 * h;
-    // a negative scale is applied as |scale| to -Q (a sign flip is exact), so the
-    // softmax may take the row max before scaling
-    const uint32_t flip = p.q_mult < 0.f ? 0x80008000u : 0u;
-    float qv[32];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-      qv[4 * c + 0] = __uint_as_float(v.x ^ flip);
-      qv[4 * c + 1] = __uint_as_float(v.y ^ flip);
-      qv[4 * c + 2] = __uint_as_float(v.z ^ flip);
-      qv[4 * c + 3] = __uint_as_float(v.w ^ flip);
-    }
-    tmem_st32(tmem + (uint32_t(32 * (warp & 3)) << 16) + kTcTmemQ + 32 * h, qv);
-    tmem_wait_st();
-  }
-  tcgen05_fence_before();
-  __syncthreads();
-  tcgen05_fence_after();
 
   if (warp == kTcKWarp || warp == kTcVWarp) {
-    // ---------------- TMA producers: stage jb = sequence tiles 4jb .. 4jb+3 ----------------
-    // one warp fills the K ring, the other the V ring, each at its own pace
+    // ---------------- TMA producers: stage = sequence tiles 16 j .. 16 j + 15 ----------------
+    // one warp fills the K ring, the other the V ring, each at its own pace and
+    // straight on into the next tile
     const bool is_k = warp == kTcKWarp;
     const CUtensorMap* map = is_k ? &pp.tmk : &pp.tmv;
     uint8_t* ring = is_k ? ksm : vsm;
     uint64_t* full = is_k ? kfull : vfull;
     uint64_t* empty = is_k ? kempty : vempty;
-    const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
     const uint64_t policy = l2_policy_evict_last();  // other row blocks read it again
-    int issued = 0;
     constexpr int kPre = 32 / kTcTiles;  // stages covered by one table read per lane
-    int ent = 0;  // this lane's pool tile of the current group of 32 tiles
+    int g = 0;                           // stages issued by this CTA
     bool ok = true;
-    for (int jb = 0; jb < nkb && ok; ++jb) {
-      const int stage = jb % kTcStages;
-      const int ntl = min(kTcTiles, ntiles - kTcTiles * jb);
-      if (jb % kPre == 0) {
-        const int t = kTcTiles * jb + lane;
-        ent = 0;
-        if (t < ntiles) {
-          const int e = t / p.tiles_per_block;
-          int32_t phys = table_row[e];
-          if (phys < 0 || phys >= p.num_blocks) {
-            if (is_k) atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
-            phys = 0;
+    int tile = -1;
+    TcTile t;
+    while (ok && tc_next_tile(pp, tile, t, is_k && lane == 0)) {
+      const int32_t* table_row = p.block_tables + int64_t(t.seq) * p.max_blocks_per_seq;
+      int ent = 0;  // this lane's pool tile of the current group of 32 tiles
+      for (int jb = 0; jb < t.nkb && ok; ++jb, ++g) {
+        const int stage = g % kTcStages;
+        const int ntl = min(kTcTiles, t.ntiles - kTcTiles * jb);
+        if (jb % kPre == 0) {
+          const int tt = kTcTiles * jb + lane;
+          ent = 0;
+          if (tt < t.ntiles) {
+            const int e = tt / p.tiles_per_block;
+            int32_t phys = table_row[e];
+            if (phys < 0 || phys >= p.num_blocks) {
+              if (is_k) atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
+              phys = 0;
+            }
+            ent = (phys * p.num_kv_heads + t.kvh) * p.tiles_per_block +
+                  (tt - e * p.tiles_per_block);
           }
-          ent = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
         }
-      }
-      int tls[kTcTiles];
+        int tls[kTcTiles];
 #pragma unroll
-      for (int t = 0; t < kTcTiles; ++t)
-        tls[t] = __shfl_sync(kFullMask, ent, kTcTiles * (jb % kPre) + t);
-      if (lane == 0) {
-        if (jb >= kTcStages && !mbar_wait_bounded(&empty[stage], ((jb / kTcStages) - 1) & 1)) {
-          atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
-          ok = false;
-        }
-        if (ok) {
-          uint8_t* dst = ring + stage * kTcTileBytes;
-          mbar_arrive_expect_tx(&full[stage], uint32_t(ntl) * 2 * 2048);
-          for (int t = 0; t < ntl; ++t) {
-            const int row = tls[t] * kBlockSize;
-            tma_load_2d(dst + t * 2048, map, 0, row, &full[stage], policy);
-            tma_load_2d(dst + kTcTileBytes / 2 + t * 2048, map, 64, row, &full[stage], policy);
+        for (int i = 0; i < kTcTiles; ++i)
+          tls[i] = __shfl_sync(kFullMask, ent, kTcTiles * (jb % kPre) + i);
+        if (lane == 0) {
+          if (g >= kTcStages && !mbar_wait_bounded(&empty[stage], ((g / kTcStages) - 1) & 1)) {
+            atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
+            ok = false;
           }
-          ++issued;
+          if (ok) {
+            uint8_t* dst = ring + stage * kTcTileBytes;
+            mbar_arrive_expect_tx(&full[stage], uint32_t(ntl) * 2 * 2048);
+            for (int i = 0; i < ntl; ++i) {
+              const int row = tls[i] * kBlockSize;
+              tma_load_2d(dst + i * 2048, map, 0, row, &full[stage], policy);
+              tma_load_2d(dst + kTcTileBytes / 2 + i * 2048, map, 64, row, &full[stage], policy);
+            }
+          }
         }
+        ok = __shfl_sync(kFullMask, ok, 0);
+        if (!ok) break;
       }
-      ok = __shfl_sync(kFullMask, ok, 0);
     }
     if (lane == 0) {  // no copy may still be landing when the CTA exits (one ring)
-      for (int i = max(0, issued - kTcStages); i < issued; ++i)
+      for (int i = max(0, g - kTcStages); i < g; ++i)
         if (!mbar_wait_bounded(&full[i % kTcStages], (i / kTcStages) & 1))
           atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
     }
@@ -1879,27 +1927,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint64_t kdesc0 = umma_smem_desc(smem_u32(ksm), 16, 1024, kUmmaSwizzle128B);
       const uint64_t vdesc0 = umma_smem_desc(smem_u32(vsm), kTcTileBytes / 2, 1024,
                                              kUmmaSwizzle128B);
-      int ns = 0, npv = 0, idle = 0;
+      TcCursor cs, cp;  // next S and next P.V
+      cs.advance(pp);
+      cp.advance(pp);
+      int ns = 0, npv = 0, idle = 0;  // stages issued (global over this CTA's tiles)
       unsigned long long t_idle = 0;
       bool ok = true;
-      while (npv < nkb) {
+      while (cp.valid) {
         bool prog = false;
-        // S(ns) into buffer ns & 1, whose P(ns - 2) went to P.V(ns - 2) already
-        if (ns < nkb && ns <= npv + 1 && mbar_test(&kfull[ns % kTcStages], (ns / kTcStages) & 1)) {
+        // S(ns) into buffer ns & 1, whose P(ns - 2) went to P.V(ns - 2) already; the
+        // first stage of a tile also needs that tile's Q
+        if (cs.valid && ns <= npv + 1 &&
+            (cs.jb > 0 || mbar_test(&q_ready[cs.tcount & 1], (cs.tcount >> 1) & 1)) &&
+            mbar_test(&kfull[ns % kTcStages], (ns / kTcStages) & 1)) {
           tcgen05_fence_after();
           const uint64_t kd = kdesc0 + uint64_t(((ns % kTcStages) * kTcTileBytes) >> 4);
           const uint32_t d = tmem + uint32_t(ns & 1) * kTcKv;
+          const uint32_t qa = tmem + kTcTmemQ + 64 * uint32_t(cs.tcount & 1);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            umma_f16_ts(d, tmem + kTcTmemQ + uint32_t(8 * ks),
+            umma_f16_ts(d, qa + uint32_t(8 * ks),
                         kd + uint64_t(((ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32) >> 4),
                         kIdescS, ks > 0 ? 1u : 0u);
           umma_commit(&s_full[ns & 1]);
           umma_commit(&kempty[ns % kTcStages]);
           ++ns;
+          cs.advance(pp);
           prog = true;
         }
-        // P.V(npv): P from TMEM over S buffer npv & 1, V from its ring slot
+        // P.V(npv): P from TMEM over S buffer npv & 1, V from its ring slot; the
+        // first stage of a tile writes O, the others accumulate
         if (npv < ns && mbar_test(&p_ready[npv & 1], (npv >> 1) & 1) &&
             mbar_test(&vfull[npv % kTcStages], (npv / kTcStages) & 1)) {
           tcgen05_fence_after();
@@ -1911,11 +1968,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int ks = 0; ks < kTcKv / 16; ++ks)
               umma_f16_ts(tmem + kTcTmemO, pt + uint32_t(t * (kTcKv / 2) + ks * 8),
                           vd + uint64_t((ks * 2048) >> 4), kIdescPV,
-                          (npv > 0 || t > 0 || ks > 0) ? 1u : 0u);
+                          (cp.jb > 0 || t > 0 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&o_full[npv & 1]);
           umma_commit(&vempty[npv % kTcStages]);
           ++npv;
+          cp.advance(pp);
           prog = true;
         }
         if (prog) {
@@ -1941,162 +1999,186 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     // ---------------- softmax warps: thread = (row, column half) ----------------
     const int h = warp >> 2, qd = warp & 3;
-    const int r = 32 * qd + lane;  // TMEM lane and Q row
-    const int gr = row0 + r;
-    const bool valid = gr < rows;
-    const int pos = valid ? L - nq + gr / G : -1;
+    const int r = 32 * qd + lane;  // TMEM lane and row within a tile
     const uint32_t tl = tmem + (uint32_t(32 * qd) << 16);  // this warp's lane quadrant
     const uint32_t pair_bar = 1 + qd;                       // this warp and warp qd + 4*(1-h)
     const float mult = fabsf(p.q_mult);  // Q carries the sign
-    float m = -INFINITY, l = 0.f;        // reference max (exp2 domain), sum of this half
     bool ok = true;                      // warp-uniform; after a failure waits are skipped,
                                          // but every named barrier is still reached
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
     };
-    for (int jb = 0; jb < nkb; ++jb) {
-      const uint32_t sb = tl + uint32_t(jb & 1) * kTcKv;  // S, then P, of this stage
-      wait(&s_full[jb & 1], (jb >> 1) & 1);
-      tcgen05_fence_after();
-      float sv[kTcHalf];
-#pragma unroll
-      for (int q = 0; q < kTcHalf / 32; ++q) {
-        float v[32];
-        tmem_ld32(sb + kTcHalf * h + 32 * q, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[32 * q + i] = v[i];
-      }
-      tmem_wait_ld();
-      // causal, context and padding mask: only stages that cross this row's last
-      // visible position pay for it
-      const int nvis = pos - jb * kTcKv - kTcHalf * h + 1;
-      float me = mult;  // multiplier still to apply to sv
-      if (nvis < kTcHalf) {
-#pragma unroll
-        for (int i = 0; i < kTcHalf; ++i) sv[i] = i < nvis ? sv[i] * mult : -INFINITY;
-        me = 1.f;
-      }
-      float r8[8];  // 8 independent chains
-#pragma unroll
-      for (int k = 0; k < 8; ++k) r8[k] = sv[k];
-#pragma unroll
-      for (int i = 8; i < kTcHalf; ++i) r8[i & 7] = fmaxf(r8[i & 7], sv[i]);
-      const float pmax = fmaxf(fmaxf(fmaxf(r8[0], r8[1]), fmaxf(r8[2], r8[3])),
-                               fmaxf(fmaxf(r8[4], r8[5]), fmaxf(r8[6], r8[7]))) * me;
-      float* xm = xmax + (jb & 1) * 2 * kTcRows;
-      xm[h * kTcRows + r] = pmax;
-      named_bar_sync(pair_bar, 64);  // both halves have read S and posted their max
-      const float mx = fmaxf(pmax, xm[(1 - h) * kTcRows + r]);
-      if (jb == 0) {
-        m = mx;  // O is written, not accumulated, by the first P.V
-      } else {
-        const bool move = mx > m + kTcRescaleLog2;
-        if (__any_sync(kFullMask, move)) {
-          // rescale this warp's rows and columns of O once P.V(jb - 1) has landed
-          wait(&o_full[(jb - 1) & 1], ((jb - 1) >> 1) & 1);
-          tcgen05_fence_after();
-          const float f = move ? ex2_approx(m - mx) : 1.f;
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            float v[32];
-            tmem_ld32(tl + kTcTmemO + 64 * h + 32 * q, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= f;
-            tmem_st32(tl + kTcTmemO + 64 * h + 32 * q, v);
-          }
-          l *= f;
-          if (move) m = mx;
-        }
-      }
-      const float mu = m == -INFINITY ? 0.f : m;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) r8[k] = 0.f;
-#pragma unroll
-      for (int i = 0; i < kTcHalf; ++i) {
-        sv[i] = ex2_approx(fmaf(sv[i], me, -mu));
-        r8[i & 7] += sv[i];
-      }
-      l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-      // P over the S columns both halves have read: this half's tokens as 16-bit
-      // pairs in columns [h * kTcHalf / 2, (h + 1) * kTcHalf / 2), the lo term
-      // kTcKv / 2 columns further on
-#pragma unroll
-      for (int q = 0; q < kTcHalf / 32; ++q) {
-        uint32_t pw[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pw[c] = pack2(sv[32 * q + 2 * c], sv[32 * q + 2 * c + 1], CT{});
-        tmem_st16(sb + (kTcHalf / 2) * h + 16 * q, pw);
-        if constexpr (kSplitP) {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float2 hi = unpack2(pw[c], CT{});
-            pw[c] = pack2(sv[32 * q + 2 * c] - hi.x, sv[32 * q + 2 * c + 1] - hi.y, CT{});
-          }
-          tmem_st16(sb + kTcKv / 2 + (kTcHalf / 2) * h + 16 * q, pw);
-        }
-      }
-      if (jb == nkb - 1 && tid < 2 * kTcKv) {
-        // V rows past the last visible token may be stale or NaN: zero them
-        wait(&vfull[jb % kTcStages], (jb / kTcStages) & 1);
-        const int vr = tid >> 1, half = tid & 1;
-        if (ok && jb * kTcKv + vr > pos_last) {
-          uint8_t* vrow = vsm + (jb % kTcStages) * kTcTileBytes + half * (kTcTileBytes / 2) +
-                          vr * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-      }
-      tmem_wait_st();
+    auto arrive = [&](uint64_t* bar) {
       tcgen05_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[jb & 1]);
+      if (lane == 0) mbar_arrive(bar);
+    };
+    int tile = -1, g = 0, tc = 0;
+    TcTile t;
+    bool have = tc_next_tile(pp, tile, t, false);
+    if (have) {
+      tc_store_q(p, t, tl, 0, r, h);
+      arrive(&q_ready[0]);
     }
-    wait(&o_full[(nkb - 1) & 1], ((nkb - 1) >> 1) & 1);
-    lsum[h * kTcRows + r] = l;
-    named_bar_sync(pair_bar, 64);
-    const float lt = l + lsum[(1 - h) * kTcRows + r];
-    if (!ok && lane == 0) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
-    if (ok) {
-      tcgen05_fence_after();
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      uint8_t* dst = static_cast<uint8_t*>(p.out);
-      const int64_t orow = (int64_t(q0 + (valid ? gr / G : 0)) * p.num_heads + kvh * G +
-                            (valid ? gr % G : 0)) * D + 64 * h;
+    while (have) {
+      const int gr = t.row0 + r;
+      const bool valid = gr < t.rows;
+      const int pos = valid ? t.L - t.nq + gr / p.group : -1;
+      float m = -INFINITY, l = 0.f;  // reference max (exp2 domain), sum of this half
+      for (int jb = 0; jb < t.nkb; ++jb, ++g) {
+        const uint32_t sb = tl + uint32_t(g & 1) * kTcKv;  // S, then P, of this stage
+        wait(&s_full[g & 1], (g >> 1) & 1);
+        tcgen05_fence_after();
+        float sv[kTcHalf];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        float v[32];
-        tmem_ld32(tl + kTcTmemO + 64 * h + 32 * q, v);
+        for (int q = 0; q < kTcHalf / 32; ++q) {
+          float v[32];
+          tmem_ld32(sb + kTcHalf * h + 32 * q, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sv[32 * q + i] = v[i];
+        }
         tmem_wait_ld();
-        if (!valid) continue;
-        if (p.out_dtype == PA_F32) {
+        // causal, context and padding mask: only stages that cross this row's last
+        // visible position pay for it
+        const int nvis = pos - jb * kTcKv - kTcHalf * h + 1;
+        float me = mult;  // multiplier still to apply to sv
+        if (nvis < kTcHalf) {
 #pragma unroll
-          for (int d = 0; d < 32; d += 4)
-            *reinterpret_cast<float4*>(dst + (orow + 32 * q + d) * 4) =
-                make_float4(v[d] * inv, v[d + 1] * inv, v[d + 2] * inv, v[d + 3] * inv);
-        } else if (p.out_dtype == PA_F16) {
+          for (int i = 0; i < kTcHalf; ++i) sv[i] = i < nvis ? sv[i] * mult : -INFINITY;
+          me = 1.f;
+        }
+        float r8[8];  // 8 independent chains
 #pragma unroll
-          for (int d = 0; d < 32; d += 8)
-            *reinterpret_cast<uint4*>(dst + (orow + 32 * q + d) * 2) =
-                make_uint4(pack2(v[d] * inv, v[d + 1] * inv, __half{}),
-                           pack2(v[d + 2] * inv, v[d + 3] * inv, __half{}),
-                           pack2(v[d + 4] * inv, v[d + 5] * inv, __half{}),
-                           pack2(v[d + 6] * inv, v[d + 7] * inv, __half{}));
+        for (int k = 0; k < 8; ++k) r8[k] = sv[k];
+#pragma unroll
+        for (int i = 8; i < kTcHalf; ++i) r8[i & 7] = fmaxf(r8[i & 7], sv[i]);
+        const float pmax = fmaxf(fmaxf(fmaxf(r8[0], r8[1]), fmaxf(r8[2], r8[3])),
+                                 fmaxf(fmaxf(r8[4], r8[5]), fmaxf(r8[6], r8[7]))) * me;
+        float* xm = xmax + (g & 1) * 2 * kTcRows;
+        xm[h * kTcRows + r] = pmax;
+        named_bar_sync(pair_bar, 64);  // both halves have read S and posted their max
+        const float mx = fmaxf(pmax, xm[(1 - h) * kTcRows + r]);
+        if (jb == 0) {
+          m = mx;  // O is written, not accumulated, by the tile's first P.V
         } else {
+          const bool move = mx > m + kTcRescaleLog2;
+          if (__any_sync(kFullMask, move)) {
+            // rescale this warp's rows and columns of O once P.V(g - 1) has landed
+            wait(&o_full[(g - 1) & 1], ((g - 1) >> 1) & 1);
+            tcgen05_fence_after();
+            const float f = move ? ex2_approx(m - mx) : 1.f;
 #pragma unroll
-          for (int d = 0; d < 32; d += 8)
-            *reinterpret_cast<uint4*>(dst + (orow + 32 * q + d) * 2) =
-                make_uint4(pack2(v[d] * inv, v[d + 1] * inv, __nv_bfloat16{}),
-                           pack2(v[d + 2] * inv, v[d + 3] * inv, __nv_bfloat16{}),
-                           pack2(v[d + 4] * inv, v[d + 5] * inv, __nv_bfloat16{}),
-                           pack2(v[d + 6] * inv, v[d + 7] * inv, __nv_bfloat16{}));
+            for (int q = 0; q < 2; ++q) {
+              float v[32];
+              tmem_ld32(tl + kTcTmemO + 64 * h + 32 * q, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] *= f;
+              tmem_st32(tl + kTcTmemO + 64 * h + 32 * q, v);
+            }
+            l *= f;
+            if (move) m = mx;
+          }
+        }
+        const float mu = m == -INFINITY ? 0.f : m;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) r8[k] = 0.f;
+#pragma unroll
+        for (int i = 0; i < kTcHalf; ++i) {
+          sv[i] = ex2_approx(fmaf(sv[i], me, -mu));
+          r8[i & 7] += sv[i];
+        }
+        l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+        // P over the S columns both halves have read: this half's tokens as 16-bit
+        // pairs in columns [h * kTcHalf / 2, (h + 1) * kTcHalf / 2), the lo term
+        // kTcKv / 2 columns further on
+#pragma unroll
+        for (int q = 0; q < kTcHalf / 32; ++q) {
+          uint32_t pw[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pw[c] = pack2(sv[32 * q + 2 * c], sv[32 * q + 2 * c + 1], CT{});
+          tmem_st16(sb + (kTcHalf / 2) * h + 16 * q, pw);
+          if constexpr (kSplitP) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float2 hi = unpack2(pw[c], CT{});
+              pw[c] = pack2(sv[32 * q + 2 * c] - hi.x, sv[32 * q + 2 * c + 1] - hi.y, CT{});
+            }
+            tmem_st16(sb + kTcKv / 2 + (kTcHalf / 2) * h + 16 * q, pw);
+          }
+        }
+        if (jb == t.nkb - 1 && tid < 2 * kTcKv) {
+          // V rows past the tile's last visible token may be stale or NaN: zero them
+          wait(&vfull[g % kTcStages], (g / kTcStages) & 1);
+          const int vr = tid >> 1, half = tid & 1;
+          if (ok && jb * kTcKv + vr > t.pos_last) {
+            uint8_t* vrow = vsm + (g % kTcStages) * kTcTileBytes + half * (kTcTileBytes / 2) +
+                            vr * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+        tmem_wait_st();
+        arrive(&p_ready[g & 1]);
+      }
+      // the next tile's Q goes in before this tile's epilogue, so its first S can
+      // run on the tensor core meanwhile (its slot's last reader, the S MMAs of the
+      // tile before this one, finished before this tile's last S)
+      const bool v_out = valid;
+      const int64_t orow = (int64_t(t.q0 + (valid ? gr / p.group : 0)) * p.num_heads +
+                            t.kvh * p.group + (valid ? gr % p.group : 0)) * D + 64 * h;
+      have = tc_next_tile(pp, tile, t, false);
+      if (have) {
+        tc_store_q(p, t, tl, uint32_t((tc + 1) & 1), r, h);
+        arrive(&q_ready[(tc + 1) & 1]);
+      }
+      // epilogue: O / l of this tile's rows, this warp's 64 columns
+      wait(&o_full[(g - 1) & 1], ((g - 1) >> 1) & 1);
+      lsum[h * kTcRows + r] = l;
+      named_bar_sync(pair_bar, 64);
+      const float lt = l + lsum[(1 - h) * kTcRows + r];
+      named_bar_sync(pair_bar, 64);  // both read lsum before the next tile writes it
+      if (ok) {
+        tcgen05_fence_after();
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        uint8_t* dst = static_cast<uint8_t*>(p.out);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          float v[32];
+          tmem_ld32(tl + kTcTmemO + 64 * h + 32 * q, v);
+          tmem_wait_ld();
+          if (!v_out) continue;
+          if (p.out_dtype == PA_F32) {
+#pragma unroll
+            for (int d = 0; d < 32; d += 4)
+              *reinterpret_cast<float4*>(dst + (orow + 32 * q + d) * 4) =
+                  make_float4(v[d] * inv, v[d + 1] * inv, v[d + 2] * inv, v[d + 3] * inv);
+          } else if (p.out_dtype == PA_F16) {
+#pragma unroll
+            for (int d = 0; d < 32; d += 8)
+              *reinterpret_cast<uint4*>(dst + (orow + 32 * q + d) * 2) =
+                  make_uint4(pack2(v[d] * inv, v[d + 1] * inv, __half{}),
+                             pack2(v[d + 2] * inv, v[d + 3] * inv, __half{}),
+                             pack2(v[d + 4] * inv, v[d + 5] * inv, __half{}),
+                             pack2(v[d + 6] * inv, v[d + 7] * inv, __half{}));
+          } else {
+#pragma unroll
+            for (int d = 0; d < 32; d += 8)
+              *reinterpret_cast<uint4*>(dst + (orow + 32 * q + d) * 2) =
+                  make_uint4(pack2(v[d] * inv, v[d + 1] * inv, __nv_bfloat16{}),
+                             pack2(v[d + 2] * inv, v[d + 3] * inv, __nv_bfloat16{}),
+                             pack2(v[d + 4] * inv, v[d + 5] * inv, __nv_bfloat16{}),
+                             pack2(v[d + 6] * inv, v[d + 7] * inv, __nv_bfloat16{}));
+          }
         }
       }
+      tcgen05_fence_before();  // O is read before the next tile's first P.V overwrites it
+      ++tc;
     }
-    tcgen05_fence_before();
+    if (!ok && lane == 0) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
   }
   // Free TMEM only after every MMA has completed and every TMEM access is done.
   __syncthreads();
@@ -2417,8 +2499,15 @@ int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_quer
     tp.p = pp.p;
     tp.query_start = pp.query_start;
     tp.row_blocks = int((int64_t(max_query_len) * group + kTcRows - 1) / kTcRows);
-    const int64_t gx = int64_t(a.num_seqs) * tp.row_blocks;
-    if (gx > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    const int64_t tiles = int64_t(a.num_seqs) * a.num_kv_heads * tp.row_blocks;
+    if (tiles > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    tp.num_tiles = int(tiles);
+    // persistent: one CTA per SM walks its round-robin share of the tiles
+    int dev_sm = 0, sms = 0;
+    if (cudaGetDevice(&dev_sm) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_sm) != cudaSuccess)
+      return PA_ERR_CUDA;
+    const unsigned grid_tc = unsigned(tiles < sms ? tiles : sms);
     constexpr size_t smem = tc_prefill_smem_bytes();
     auto launch = [&](auto kern, unsigned long long& mask) -> int {
       int dev = 0;
@@ -2430,7 +2519,7 @@ int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_quer
           return PA_ERR_CUDA;
         mask |= bit;
       }
-      kern<<<dim3(unsigned(gx), unsigned(a.num_kv_heads)), kTcThreads, smem, stream>>>(tp);
+      kern<<<grid_tc, kTcThreads, smem, stream>>>(tp);
       return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
     };
     static unsigned long long tmask_h = 0, tmask_b = 0, tmask_bs = 0;
