@@ -143,14 +143,25 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+DECODE_SOURCES = ("pa_decode.cu", "pa_kernels.cuh", "pa_common.cuh", "pa_internal.h")
+
+
+def decode_source_sha() -> str:
+    """sha256 prefix over the decode kernels' sources, in a fixed order."""
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_413_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(config: str):
     """DRAM bytes per decode launch from the committed ncu summary of this workload,
     valid only while the decode source is the one that was profiled."""
     path = os.path.join(ROOT, "profiles", f"paged_attention_decode_{config}.md")
-    src = os.path.join(ROOT, "paged_kv_cache_413_b200", "csrc", "pa_decode.cu")
     try:
         text = open(path).read()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        sha = decode_source_sha()
         m = re.search(r"decode_source_sha256_16:\s*([0-9a-f]{16})", text)
         t = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
         if m and t and m.group(1) == sha:
