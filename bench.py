@@ -144,15 +144,36 @@ def measured_peak():
 
 
 DECODE_SOURCES = ("pa_decode.cu", "pa_kernels.cuh", "pa_common.cuh", "pa_internal.h")
+PREFILL_SOURCES = ("pa_prefill.cu", "pa_tcgen05.cuh", "pa_kernels.cuh", "pa_common.cuh",
+                   "pa_internal.h")
 
 
-def decode_source_sha() -> str:
-    """sha256 prefix over the decode kernels' sources, in a fixed order."""
+def source_sha(names=DECODE_SOURCES) -> str:
+    """sha256 prefix over a kernel's sources, in a fixed order."""
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
+    for name in names:
         with open(os.path.join(ROOT, "paged_kv_cache_413_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def decode_source_sha() -> str:
+    return source_sha(DECODE_SOURCES)
+
+
+def recorded_prefill_traffic(config: str):
+    """DRAM bytes per prefill launch from the committed ncu summary of this workload,
+    valid only while the prefill sources are the ones that were profiled."""
+    path = os.path.join(ROOT, "profiles", f"prefill_tc_{config}.md")
+    try:
+        text = open(path).read()
+        m = re.search(r"prefill_source_sha256_16:\s*([0-9a-f]{16})", text)
+        t = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+        if m and t and m.group(1) == source_sha(PREFILL_SOURCES):
+            return int(t.group(1))
+    except OSError:
+        pass
+    return None
 
 
 def recorded_traffic(config: str):
@@ -537,7 +558,8 @@ def run_prefill(args, rank, world, local_rank):
                        "l2": f"KV read {kv_bytes / 1e6:.0f} MB per step, above the 126 MB L2"},
             "roofline": {"bound": "tensor", "kernel": kernel,
                          "achieved": round(achieved, 2), "peak": peak, "peak_kind": kind,
-                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "traffic": recorded_prefill_traffic(args.config),
                          "launch_ms": round(kern_ms, 5),
                          "hbm_gbs": round((kv_bytes + qo_bytes) / (kern_ms * 1e-3) / 1e9, 1)},
             "gpu_launches": 2 * args.steps,
