@@ -48,6 +48,105 @@ static_assert(kStagesSimt % kConsumerWarps == 0 && kStagesMma16 % kConsumerWarps
                   kStagesMmaFp8 % kConsumerWarps == 0,
               "each ring stage must belong to one consumer warp");
 
+// ---------------------------------------------------------------------------
+// Work order.  CTAs start roughly in linear block order, so handing out the
+// longest sequences first (list scheduling, longest first) leaves the shortest
+// units for the tail of the launch instead of whichever sequence came last.  The
+// linear block index b is split into a rank (b / units per sequence), a partition
+// and a (kv head, head group).  With p.lpt the sequence of a rank comes from a
+// ranking of seq_lens by length in kLptBuckets buckets of 16-token tiles (longest
+// first, ties by index), computed by one warp from one read of seq_lens; the
+// launcher sets p.lpt only where that costs less than the tail it removes (long
+// units, at most kLptMaxSeqs sequences).  Otherwise rank = sequence.
+// ---------------------------------------------------------------------------
+#ifndef PA_DECODE_LPT
+#define PA_DECODE_LPT 1
+#endif
+constexpr int kLptBuckets = 256;
+constexpr int kLptMaxSeqs = 256;      // lengths held in registers: 8 per lane
+constexpr int kLptMinTokens = 1024;   // shortest unit (tokens) worth the ranking
+
+struct LptScratch {
+  int start[kLptBuckets];  // counts, then exclusive start offsets, per bucket
+  int seq;
+};
+
+// Every thread of the CTA calls this once, before any role split.
+__device__ __forceinline__ void decode_unit(const Params& p, LptScratch& sc, int& seq, int& part,
+                                            int& hg) {
+  const int HG = p.num_kv_heads * p.head_groups;
+  const int64_t b = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
+  const int per_seq = p.max_parts * HG;
+  const int rank = int(b / per_seq);
+  const int rem = int(b - int64_t(rank) * per_seq);
+  part = rem / HG;
+  hg = rem - part * HG;
+  seq = rank;
+#if PA_DECODE_LPT
+  if (!p.lpt) return;  // uniform over the grid
+  constexpr int kPer = kLptMaxSeqs / 32;
+  static_assert(kLptBuckets == 32 * kPer, "one scan slice of buckets per lane");
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x, n = p.num_seqs;
+    const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+    const int max_tiles = max(1, (cap + kBlockSize - 1) / kBlockSize);
+    int bk[kPer];  // bucket of sequence lane + 32 k (0 = longest), -1 past the batch
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int i = lane + 32 * k;
+      int L = i < n ? p.seq_lens[i] : 0;
+      L = L < 0 ? 0 : (L > cap ? cap : L);
+      const int tiles = (L + kBlockSize - 1) / kBlockSize;
+      bk[k] = i < n ? (kLptBuckets - 1) - int(int64_t(tiles) * (kLptBuckets - 1) / max_tiles)
+                    : -1;
+      sc.start[lane * kPer + k] = 0;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+      if (bk[k] >= 0) atomicAdd(&sc.start[bk[k]], 1);
+    __syncwarp();
+    // exclusive scan of the counts; this lane's buckets [kPer lane, kPer lane + kPer)
+    int v[kPer], sum = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) sum += (v[k] = sc.start[lane * kPer + k]);
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(kFullMask, incl, o);
+      if (lane >= o) incl += t;
+    }
+    // the bucket holding `rank`, and rank's place inside it
+    int run = incl - sum, kk = -1, j = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      if (run <= rank && rank < run + v[k]) {
+        kk = lane * kPer + k;
+        j = rank - run;
+      }
+      run += v[k];
+    }
+    const unsigned own = __ballot_sync(kFullMask, kk >= 0);
+    const int src = __ffs(own) - 1;  // exactly one lane holds it
+    kk = __shfl_sync(kFullMask, kk, src);
+    j = __shfl_sync(kFullMask, j, src);
+    // the j-th sequence, by index, in bucket kk
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const unsigned bal = __ballot_sync(kFullMask, bk[k] == kk);
+      const int c = __popc(bal);
+      if (j < c) {
+        if (bk[k] == kk && __popc(bal & ((1u << lane) - 1u)) == j) sc.seq = lane + 32 * k;
+        break;
+      }
+      j -= c;
+    }
+  }
+  __syncthreads();
+  seq = sc.seq;
+#endif
+}
+
 // This lane's DPL = D/32 consecutive elements of row `row` of a [16][D] tile.
 template <typename CT, int D>
 __device__ __forceinline__ void load_lane_row(const uint8_t* tile, int row, int lane,
@@ -212,10 +311,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   float* sp = reinterpret_cast<float*>(empty + kStages);  // [warps][GT][16] probabilities
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int seq = blockIdx.x / p.max_parts;
-  const int part = blockIdx.x - seq * p.max_parts;
-  const int kvh = blockIdx.y / p.head_groups;
-  const int hsub = blockIdx.y - kvh * p.head_groups;
+  __shared__ LptScratch lpt;
+  int seq, part, hg;
+  decode_unit(p, lpt, seq, part, hg);
+  const int kvh = hg / p.head_groups;
+  const int hsub = hg - kvh * p.head_groups;
   const int head0 = kvh * p.group + hsub * GT;  // first query head of this CTA
 
   // The producer starts the first block-table read before anything else; the row
@@ -229,7 +329,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   int L = p.seq_lens[seq];
   const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
   if (L < 0 || L > cap) {
-    if (tid == 0 && part == 0 && blockIdx.y == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
+    if (tid == 0 && part == 0 && hg == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
     L = L < 0 ? 0 : cap;
   }
   const int nparts = (L + p.partition - 1) / p.partition;
@@ -467,10 +567,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
   uint64_t* empty = full + kStages;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int seq = blockIdx.x / p.max_parts;
-  const int part = blockIdx.x - seq * p.max_parts;
-  const int kvh = blockIdx.y / p.head_groups;
-  const int hsub = blockIdx.y - kvh * p.head_groups;
+  __shared__ LptScratch lpt;
+  int seq, part, hg;
+  decode_unit(p, lpt, seq, part, hg);
+  const int kvh = hg / p.head_groups;
+  const int hsub = hg - kvh * p.head_groups;
   const int head0 = kvh * p.group + hsub * GT;
 
   const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
@@ -481,7 +582,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
   int L = p.seq_lens[seq];
   const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
   if (L < 0 || L > cap) {
-    if (tid == 0 && part == 0 && blockIdx.y == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
+    if (tid == 0 && part == 0 && hg == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
     L = L < 0 ? 0 : cap;
   }
   const int nparts = (L + p.partition - 1) / p.partition;
@@ -1499,6 +1600,7 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
   p.max_parts = 1;
   p.out_dtype = a.out_dtype;
   p.num_blocks = a.num_blocks;
+  p.num_seqs = a.num_seqs;
   const bool fp8 = a.cache_dtype == PA_FP8_E4M3;
   p.q_mult = a.scale * kLog2e * (fp8 ? a.k_scale : 1.f);
   p.v_mult = fp8 ? a.v_scale : 1.f;
@@ -1552,6 +1654,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.max_parts = a.ws.max_parts > 0 ? a.ws.max_parts : 1;
   p.out_dtype = a.out_dtype;
   p.num_blocks = a.num_blocks;
+  p.num_seqs = a.num_seqs;
+  p.lpt = a.num_seqs <= kLptMaxSeqs && min(a.partition, a.max_seq_len) >= kLptMinTokens;
   const bool fp8 = a.cache_dtype == PA_FP8_E4M3;
   p.q_mult = a.scale * kLog2e * (fp8 ? a.k_scale : 1.f);
   p.v_mult = fp8 ? a.v_scale : 1.f;

@@ -42,6 +42,8 @@ struct Params {
   int max_parts;
   int out_dtype;
   int64_t num_blocks;
+  int num_seqs;     // sequences of the launch
+  int lpt;          // decode: dispatch the longest sequences first (see decode_unit)
   float q_mult;     // scale * log2(e) [* k_scale]
   float v_mult;     // 1 or v_scale
 };
