@@ -915,8 +915,11 @@ constexpr size_t shared_smem_bytes() {
          size_t(kSharedCols) * (2 + combine_row<128>()) * sizeof(float);
 }
 
+#ifndef PA_SHARED_MIN_CTAS
+#define PA_SHARED_MIN_CTAS 4  // resident CTAs per SM the register budget must allow
+#endif
 template <typename CT, typename QT, int kStages>
-__global__ void __launch_bounds__(kThreads) decode_shared_prefix_kernel(
+__global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_prefix_kernel(
     const __grid_constant__ SharedParams sp) {
   constexpr int D = 128;
   constexpr int NT = 2;
