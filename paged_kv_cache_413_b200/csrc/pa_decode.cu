@@ -1613,7 +1613,8 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
   sp.ctas_per_group = (max_group_size + sp.seqs_per_cta - 1) / sp.seqs_per_cta;
   const int64_t grid_x = int64_t(num_groups) * sp.ctas_per_group;
   // Split each unit's block stream over a cluster of up to 8 CTAs when there are
-  // too few units to keep the GPU streaming, keeping chunks of >= 8 blocks.
+  // too few units to keep the GPU streaming, keeping chunks of at least
+  // PA_SHARED_MIN_CHUNK blocks.
   {
     const int64_t units = grid_x * a.num_kv_heads;
     int c = int((kAutoTargetCtas + units - 1) / (units > 0 ? units : 1));

@@ -344,6 +344,35 @@ constexpr int kTcTileBytes = 2 * kTcKv * 128;  // K or V of a stage: [2 halves][
 constexpr float kTcRescaleLog2 = 8.f;          // reference max moves beyond 2^8
 constexpr uint32_t kTcPollNs = 500;            // MMA issuer's longest sleep per poll
 
+// Packed fp32 pairs (sm_100): one instruction does the work of two, each lane
+// IEEE round-to-nearest like fmaf / fadd; and the three-input maximum.
+__device__ __forceinline__ unsigned long long f2_bits(float2 a) {
+  unsigned long long u;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(u) : "f"(a.x), "f"(a.y));
+  return u;
+}
+__device__ __forceinline__ float2 bits_f2(unsigned long long u) {
+  float2 a;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(u));
+  return a;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)),
+      "l"(f2_bits(c)));
+  return bits_f2(r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(r);
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 struct TcPrefillParams {
   CUtensorMap tmk;
   CUtensorMap tmv;
@@ -689,11 +718,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < kTcHalf; ++i) sv[i] = i < nvis ? sv[i] * mult : -INFINITY;
           me = 1.f;
         }
-        float r8[8];  // 8 independent chains
+        float r8[8];  // 8 independent chains, two new columns per step
 #pragma unroll
         for (int k = 0; k < 8; ++k) r8[k] = sv[k];
 #pragma unroll
-        for (int i = 8; i < kTcHalf; ++i) r8[i & 7] = fmaxf(r8[i & 7], sv[i]);
+        for (int i = 8; i < kTcHalf; i += 2) r8[(i >> 1) & 7] = max3(r8[(i >> 1) & 7], sv[i], sv[i + 1]);
         const float pmax = fmaxf(fmaxf(fmaxf(r8[0], r8[1]), fmaxf(r8[2], r8[3])),
                                  fmaxf(fmaxf(r8[4], r8[5]), fmaxf(r8[6], r8[7]))) * me;
         float* xm = xmax + (g & 1) * 2 * kTcRows;
@@ -723,14 +752,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         const float mu = m == -INFINITY ? 0.f : m;
+        const float2 me2 = make_float2(me, me), nmu2 = make_float2(-mu, -mu);
+        float2 a4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};  // 4 chains of column pairs
 #pragma unroll
-        for (int k = 0; k < 8; ++k) r8[k] = 0.f;
-#pragma unroll
-        for (int i = 0; i < kTcHalf; ++i) {
-          sv[i] = ex2_approx(fmaf(sv[i], me, -mu));
-          r8[i & 7] += sv[i];
+        for (int c = 0; c < kTcHalf / 2; ++c) {
+          const float2 x = fma2(make_float2(sv[2 * c], sv[2 * c + 1]), me2, nmu2);
+          sv[2 * c] = ex2_approx(x.x);
+          sv[2 * c + 1] = ex2_approx(x.y);
+          a4[c & 3] = add2(a4[c & 3], make_float2(sv[2 * c], sv[2 * c + 1]));
         }
-        l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+        const float2 a2 = add2(add2(a4[0], a4[1]), add2(a4[2], a4[3]));
+        l += a2.x + a2.y;
         // P over the S columns both halves have read: this half's tokens as 16-bit
         // pairs in columns [h * kTcHalf / 2, (h + 1) * kTcHalf / 2), the lo term
         // kTcKv / 2 columns further on
