@@ -321,34 +321,44 @@ def run_ours(args, rank, world, local_rank):
     launches = 1 + 1 + (1 if reduce_runs else 0) + (1 if bm is not None else 0)
 
     shared = wl.group_starts is not None and args.decode in ("auto", "shared")
+    gs = pl = None
     if shared:
         gs, pl = f(wl.group_starts), f(wl.prefix_lens)
         max_group = int((wl.group_starts[1:] - wl.group_starts[:-1]).max())
         launches -= 1 if reduce_runs else 0  # the shared-prefix decode needs no merge
     ev = []
+    # the step's inputs: what a serving loop hands over every step
+    inputs = {"q": q, "nk": nk, "nv": nv, "sm": sm, "bt": bt, "sl": sl}
+    if bm is not None:
+        inputs["bm"] = bm
+    if shared:
+        inputs.update(gs=gs, pl=pl)
 
-    def decode():
-        if shared:
-            pa.pa_paged_attention_decode_shared_prefix(
-                out, q, kc, vc, bt, sl, gs, pl, max_seq_len=max_len, max_group_size=max_group,
-                scale=wl.scale, k_scale=wl.k_scale, v_scale=wl.v_scale)
-        else:
-            pa.pa_paged_attention_decode(out, q, kc, vc, bt, sl, max_seq_len=max_len,
-                                         scale=wl.scale, k_scale=wl.k_scale, v_scale=wl.v_scale,
-                                         partition_size=part, workspace=ws)
-
-    def step(timed: bool):
-        if bm is not None:
-            pa.pa_copy_blocks([kc], [vc], bm)
-        pa.pa_reshape_and_cache(nk, nv, kc, vc, sm, k_scale=wl.k_scale, v_scale=wl.v_scale)
+    def run_step(t, out_t, timed: bool = False):
+        if "bm" in t:
+            pa.pa_copy_blocks([kc], [vc], t["bm"])
+        pa.pa_reshape_and_cache(t["nk"], t["nv"], kc, vc, t["sm"], k_scale=wl.k_scale,
+                                v_scale=wl.v_scale)
         if timed:
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        decode()
+        if shared:
+            pa.pa_paged_attention_decode_shared_prefix(
+                out_t, t["q"], kc, vc, t["bt"], t["sl"], t["gs"], t["pl"], max_seq_len=max_len,
+                max_group_size=max_group, scale=wl.scale, k_scale=wl.k_scale,
+                v_scale=wl.v_scale)
+        else:
+            pa.pa_paged_attention_decode(out_t, t["q"], kc, vc, t["bt"], t["sl"],
+                                         max_seq_len=max_len, scale=wl.scale,
+                                         k_scale=wl.k_scale, v_scale=wl.v_scale,
+                                         partition_size=part, workspace=ws)
         if timed:
             e1.record(stream)
             ev.append((e0, e1))
+
+    def step(timed: bool):
+        run_step(inputs, out, timed)
 
     for _ in range(args.warmup):
         step(False)
@@ -384,36 +394,66 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = elapsed_ms / args.steps
     value = whole_job_gbs(step_bytes, world, args.steps, elapsed_ms)
 
-    # ---- end to end through the public API with host buffers
-    pin = lambda t: None if t is None else t.pin_memory()
-    h_q, h_nk, h_nv, h_sm = pin(wl.query), pin(wl.new_key), pin(wl.new_value), pin(wl.slot_mapping)
-    h_bt, h_sl = pin(wl.block_tables), pin(wl.seq_lens)
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_nk, h_nv, h_sm, h_bt, h_sl))
-    d2h = h_out.numel() * h_out.element_size()
+    # ---- end to end through the public API with host buffers ----
+    # Every step uploads its inputs from page-locked host memory (packed in one
+    # buffer, one copy) and downloads its output.  Uploads run on one copy stream
+    # and downloads on another, with two device buffers of each, so step k+1's
+    # upload and step k-1's download overlap step k's compute, as a serving loop
+    # would run them.  The timed region runs from the first upload to the last
+    # download.
+    host_src = {"q": wl.query, "nk": wl.new_key, "nv": wl.new_value, "sm": wl.slot_mapping,
+                "bt": wl.block_tables, "sl": wl.seq_lens, "bm": wl.block_mapping,
+                "gs": wl.group_starts, "pl": wl.prefix_lens}
+    layout, off = {}, 0
+    for name, t in inputs.items():
+        layout[name] = (off, t.numel() * t.element_size(), t.dtype, tuple(t.shape))
+        off += (layout[name][1] + 255) // 256 * 256
+    h_in = torch.zeros(off, dtype=torch.uint8).pin_memory()
+    for name, (o, n, dt, shape) in layout.items():
+        h_in[o:o + n].copy_(host_src[name].contiguous().view(torch.uint8).reshape(-1))
+    d_in = [torch.empty(off, dtype=torch.uint8, device=dev) for _ in range(2)]
+    d_views = [{name: buf[o:o + n].view(dt).view(shape)
+                for name, (o, n, dt, shape) in layout.items()} for buf in d_in]
+    d_out = [torch.empty_like(out) for _ in range(2)]
+    h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    h2d = off
+    d2h = h_out[0].numel() * h_out[0].element_size()
     e2e_steps = max(10, args.steps // 4)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]  # also: d_in[b] free again
+    downloaded = [torch.cuda.Event() for _ in range(2)]  # d_out[b] free again
 
-    def e2e_step():
-        q.copy_(h_q, non_blocking=True)
-        nk.copy_(h_nk, non_blocking=True)
-        nv.copy_(h_nv, non_blocking=True)
-        sm.copy_(h_sm, non_blocking=True)
-        bt.copy_(h_bt, non_blocking=True)
-        sl.copy_(h_sl, non_blocking=True)
-        step(False)
-        h_out.copy_(out, non_blocking=True)
+    def e2e_step(k):
+        b = k & 1
+        if k >= 2:
+            up.wait_event(computed[b])
+        with torch.cuda.stream(up):
+            d_in[b].copy_(h_in, non_blocking=True)
+        uploaded[b].record(up)
+        stream.wait_event(uploaded[b])
+        if k >= 2:
+            stream.wait_event(downloaded[b])
+        run_step(d_views[b], d_out[b])
+        computed[b].record(stream)
+        down.wait_event(computed[b])
+        with torch.cuda.stream(down):
+            h_out[b].copy_(d_out[b], non_blocking=True)
+        downloaded[b].record(down)
 
-    for _ in range(3):
-        e2e_step()
+    for k in range(3):
+        e2e_step(k)
     torch.cuda.synchronize(dev)
+    if not torch.equal(h_out[0].to(dev), out):  # same inputs, deterministic kernels
+        raise RuntimeError("the end-to-end output differs from the device-timed output")
     if world > 1:
         torch.distributed.barrier()
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    a1.record(stream)
+    a0.record(up)  # every timed operation follows it: uploads on `up`, the rest waits on them
+    for k in range(e2e_steps):
+        e2e_step(k)
+    a1.record(down)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks([a0.elapsed_time(a1)], world, dev)[0]
     e2e_value = whole_job_gbs(step_bytes, world, e2e_steps, e2e_ms)
