@@ -206,6 +206,12 @@ int pa_paged_attention_decode_shared_prefix(
  *   other arguments as for pa_paged_attention_decode
  * Supported: head_dim 128; (q_dtype, cache_dtype) (F16, F16) or (BF16, BF16); out
  * F16, BF16 or F32; block_size 16, 32, 64 or 128.
+ * Numerics: scores, softmax and accumulation in fp32; P enters the P.V product in
+ * 16 bits (as two bf16 terms, hi and P - hi, when the cache is BF16 and out is F32).
+ * Device data errors set bits in the device error word (pa_get_device_error):
+ * PA_DEVERR_SEQ_LEN (length or chunk out of range; clamped), PA_DEVERR_BLOCK_RANGE
+ * (block id outside the pool; block 0 read instead), PA_DEVERR_PIPE_TIMEOUT (an
+ * internal wait gave up; the output is undefined).  Never a fault.
  */
 int pa_paged_attention_prefill(void* out, const void* query, const void* key_cache,
                                const void* value_cache, const int32_t* block_tables,
