@@ -288,6 +288,109 @@ def cpu_baseline(wl: W.Workload, out_dtype: str, budget_s: float = 12.0):
                       f"tokens + fp64 decode), {dt:.1f} s"}
 
 
+def prefill_oracle_sample(wl: W.Workload, seqs):
+    """Run the oracle (cache write of the sampled sequences' chunks + their causal
+    multi-query attention).  Returns (seconds, useful FLOPs of the sample)."""
+    import oracle
+
+    cfg = wl.cfg
+    seqs = np.asarray(seqs)
+    qs = wl.query_start.numpy().astype(np.int64)
+    rows = np.concatenate([np.arange(qs[s], qs[s + 1]) for s in seqs])
+    nt = torch.as_tensor(rows)
+    sub_qs = np.concatenate([[0], np.cumsum([qs[s + 1] - qs[s] for s in seqs])]).astype(np.int32)
+    t0 = time.perf_counter()
+    kc, vc = oracle.reshape_and_cache(wl.new_key[nt], wl.new_value[nt], wl.key_cache,
+                                      wl.value_cache, wl.slot_mapping.numpy()[rows],
+                                      src_dtype=wl.src_dtype, cache_dtype=cfg.cache_dtype,
+                                      inplace=True)
+    oracle.paged_attention_prefill(wl.query[nt], kc, vc, wl.block_tables.numpy()[seqs],
+                                   wl.seq_lens.numpy()[seqs], sub_qs, scale=wl.scale,
+                                   q_dtype=cfg.q_dtype, cache_dtype=cfg.cache_dtype)
+    dt = time.perf_counter() - t0
+    L = wl.seq_lens.numpy().astype(np.int64)
+    pairs = sum(int((L[s] - (qs[s + 1] - qs[s]) + np.arange(qs[s + 1] - qs[s]) + 1).sum())
+                for s in seqs)
+    return dt, pairs * cfg.num_heads * cfg.head_dim * 4
+
+
+def prefill_cpu_baseline(wl: W.Workload, budget_s: float = 15.0):
+    """The oracle timed on a bounded sample of the workload's sequences."""
+    import oracle
+
+    n = wl.seq_lens.numel()
+    order = np.random.default_rng(0).permutation(n)
+    dt1, _ = prefill_oracle_sample(wl, order[:1])              # calibration
+    k = int(max(1, min(n, budget_s / max(dt1, 1e-4))))
+    dt, fl = prefill_oracle_sample(wl, order[:k])
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{k} of {n} sequences of the workload (cache write of their chunks + "
+                      f"fp64 causal attention), {dt:.1f} s"}
+
+
+def pipelined_e2e(dev, stream, inputs, host_src, out, run_step, steps, world):
+    """End to end through the public API with host buffers.
+
+    Every step uploads its inputs from page-locked host memory (packed in one
+    buffer, one copy) and downloads its output.  Uploads run on one copy stream
+    and downloads on another, with two device buffers of each, so step k+1's
+    upload and step k-1's download overlap step k's compute, as a serving loop
+    would run them.  Timed from the first upload to the last download, on the
+    device.  Before timing, the output must equal `out` (the device-timed
+    result of the same inputs) bit for bit.  Returns (ms, h2d bytes, d2h bytes)
+    per step."""
+    layout, off = {}, 0
+    for name, t in inputs.items():
+        layout[name] = (off, t.numel() * t.element_size(), t.dtype, tuple(t.shape))
+        off += (layout[name][1] + 255) // 256 * 256
+    h_in = torch.zeros(off, dtype=torch.uint8).pin_memory()
+    for name, (o, n, dt, shape) in layout.items():
+        h_in[o:o + n].copy_(host_src[name].contiguous().view(torch.uint8).reshape(-1))
+    d_in = [torch.empty(off, dtype=torch.uint8, device=dev) for _ in range(2)]
+    d_views = [{name: buf[o:o + n].view(dt).view(shape)
+                for name, (o, n, dt, shape) in layout.items()} for buf in d_in]
+    d_out = [torch.empty_like(out) for _ in range(2)]
+    h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]  # also: d_in[b] free again
+    downloaded = [torch.cuda.Event() for _ in range(2)]  # d_out[b] free again
+
+    def e2e_step(k):
+        b = k & 1
+        if k >= 2:
+            up.wait_event(computed[b])
+        with torch.cuda.stream(up):
+            d_in[b].copy_(h_in, non_blocking=True)
+        uploaded[b].record(up)
+        stream.wait_event(uploaded[b])
+        if k >= 2:
+            stream.wait_event(downloaded[b])
+        run_step(d_views[b], d_out[b])
+        computed[b].record(stream)
+        down.wait_event(computed[b])
+        with torch.cuda.stream(down):
+            h_out[b].copy_(d_out[b], non_blocking=True)
+        downloaded[b].record(down)
+
+    for k in range(3):
+        e2e_step(k)
+    torch.cuda.synchronize(dev)
+    if not torch.equal(h_out[0].to(dev), out):  # same inputs, deterministic kernels
+        raise RuntimeError("the end-to-end output differs from the device-timed output")
+    if world > 1:
+        torch.distributed.barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(up)  # every timed operation follows it: uploads on `up`, the rest waits on them
+    for k in range(steps):
+        e2e_step(k)
+    a1.record(down)
+    torch.cuda.synchronize(dev)
+    return a0.elapsed_time(a1), off, h_out[0].numel() * h_out[0].element_size()
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_ours(args, rank, world, local_rank):
     import paged_kv_cache_413_b200 as pa
@@ -394,68 +497,14 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = elapsed_ms / args.steps
     value = whole_job_gbs(step_bytes, world, args.steps, elapsed_ms)
 
-    # ---- end to end through the public API with host buffers ----
-    # Every step uploads its inputs from page-locked host memory (packed in one
-    # buffer, one copy) and downloads its output.  Uploads run on one copy stream
-    # and downloads on another, with two device buffers of each, so step k+1's
-    # upload and step k-1's download overlap step k's compute, as a serving loop
-    # would run them.  The timed region runs from the first upload to the last
-    # download.
+    # ---- end to end through the public API with host buffers
     host_src = {"q": wl.query, "nk": wl.new_key, "nv": wl.new_value, "sm": wl.slot_mapping,
                 "bt": wl.block_tables, "sl": wl.seq_lens, "bm": wl.block_mapping,
                 "gs": wl.group_starts, "pl": wl.prefix_lens}
-    layout, off = {}, 0
-    for name, t in inputs.items():
-        layout[name] = (off, t.numel() * t.element_size(), t.dtype, tuple(t.shape))
-        off += (layout[name][1] + 255) // 256 * 256
-    h_in = torch.zeros(off, dtype=torch.uint8).pin_memory()
-    for name, (o, n, dt, shape) in layout.items():
-        h_in[o:o + n].copy_(host_src[name].contiguous().view(torch.uint8).reshape(-1))
-    d_in = [torch.empty(off, dtype=torch.uint8, device=dev) for _ in range(2)]
-    d_views = [{name: buf[o:o + n].view(dt).view(shape)
-                for name, (o, n, dt, shape) in layout.items()} for buf in d_in]
-    d_out = [torch.empty_like(out) for _ in range(2)]
-    h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    h2d = off
-    d2h = h_out[0].numel() * h_out[0].element_size()
     e2e_steps = max(10, args.steps // 4)
-    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    uploaded = [torch.cuda.Event() for _ in range(2)]
-    computed = [torch.cuda.Event() for _ in range(2)]  # also: d_in[b] free again
-    downloaded = [torch.cuda.Event() for _ in range(2)]  # d_out[b] free again
-
-    def e2e_step(k):
-        b = k & 1
-        if k >= 2:
-            up.wait_event(computed[b])
-        with torch.cuda.stream(up):
-            d_in[b].copy_(h_in, non_blocking=True)
-        uploaded[b].record(up)
-        stream.wait_event(uploaded[b])
-        if k >= 2:
-            stream.wait_event(downloaded[b])
-        run_step(d_views[b], d_out[b])
-        computed[b].record(stream)
-        down.wait_event(computed[b])
-        with torch.cuda.stream(down):
-            h_out[b].copy_(d_out[b], non_blocking=True)
-        downloaded[b].record(down)
-
-    for k in range(3):
-        e2e_step(k)
-    torch.cuda.synchronize(dev)
-    if not torch.equal(h_out[0].to(dev), out):  # same inputs, deterministic kernels
-        raise RuntimeError("the end-to-end output differs from the device-timed output")
-    if world > 1:
-        torch.distributed.barrier()
-    a0 = torch.cuda.Event(enable_timing=True)
-    a1 = torch.cuda.Event(enable_timing=True)
-    a0.record(up)  # every timed operation follows it: uploads on `up`, the rest waits on them
-    for k in range(e2e_steps):
-        e2e_step(k)
-    a1.record(down)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks([a0.elapsed_time(a1)], world, dev)[0]
+    e2e_ms, h2d, d2h = pipelined_e2e(dev, stream, inputs, host_src, out, run_step, e2e_steps,
+                                     world)
+    e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
     e2e_value = whole_job_gbs(step_bytes, world, e2e_steps, e2e_ms)
 
     if rank != 0:
@@ -536,17 +585,21 @@ def run_prefill(args, rank, world, local_rank):
     max_len = int(wl.seq_lens.max())
     stream = torch.cuda.current_stream(dev)
     ev = []
+    inputs = {"q": q, "nk": nk, "nv": nv, "sm": sm, "bt": bt, "sl": sl, "qs": qs}
 
-    def step(timed):
-        pa.pa_reshape_and_cache(nk, nv, kc, vc, sm)
+    def run_step(t, out_t, timed=False):
+        pa.pa_reshape_and_cache(t["nk"], t["nv"], kc, vc, t["sm"])
         if timed:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        pa.pa_paged_attention_prefill(out, q, kc, vc, bt, sl, qs, max_query_len=max_q,
-                                      max_seq_len=max_len, scale=wl.scale)
+        pa.pa_paged_attention_prefill(out_t, t["q"], kc, vc, t["bt"], t["sl"], t["qs"],
+                                      max_query_len=max_q, max_seq_len=max_len, scale=wl.scale)
         if timed:
             e1.record(stream)
             ev.append((e0, e1))
+
+    def step(timed):
+        run_step(inputs, out, timed)
 
     for _ in range(args.warmup):
         step(False)
@@ -568,6 +621,12 @@ def run_prefill(args, rank, world, local_rank):
         [t0.elapsed_time(t1), statistics.mean(a.elapsed_time(b) for a, b in ev)], world, dev)
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error bits set")
+    host_src = {"q": wl.query, "nk": wl.new_key, "nv": wl.new_value, "sm": wl.slot_mapping,
+                "bt": wl.block_tables, "sl": wl.seq_lens, "qs": wl.query_start}
+    e2e_steps = max(10, args.steps // 4)
+    e2e_ms, h2d, d2h = pipelined_e2e(dev, stream, inputs, host_src, out, run_step, e2e_steps,
+                                     world)
+    e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
     if rank != 0:
         return None
     flops = prefill_flops(wl)
@@ -602,6 +661,11 @@ def run_prefill(args, rank, world, local_rank):
                          "traffic": recorded_prefill_traffic(args.config),
                          "launch_ms": round(kern_ms, 5),
                          "hbm_gbs": round((kv_bytes + qo_bytes) / (kern_ms * 1e-3) / 1e9, 1)},
+            "e2e": {"value": round(flops * world * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2),
+                    "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 5)},
+            "cpu_baseline": (None if args.no_cpu_baseline or world > 1
+                             else prefill_cpu_baseline(wl)),
             "gpu_launches": 2 * args.steps,
             "clocks": sampler.summary() if sampler else None}
 
