@@ -546,7 +546,11 @@ constexpr size_t mma_smem_bytes() {
 }
 
 template <int GT, typename CT, typename QT, int kStages>
-__global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_constant__ TmaParams tp) {
+// Resident CTAs per SM the register budget must allow: 5 for groups of 8 (a few
+// L1-cached spills; 0.903-0.910 -> 0.920 on the 70B-GQA workload), 4 for groups of
+// 4, where 5 measured slightly slower.
+__global__ void __launch_bounds__(kThreads, GT == 8 ? 5 : 4) decode_mma_kernel(
+    const __grid_constant__ TmaParams tp) {
   constexpr int D = 128;
   constexpr bool kFp8 = CacheTraits<CT>::bytes == 1;
   constexpr int TILE = kBlockSize * D * CacheTraits<CT>::bytes;

@@ -111,3 +111,30 @@ def test_prefill_zero_and_negative_scale(scale, chunk):
     wl = W.make_prefill_workload(3, (100, 400), chunk, num_heads=32, num_kv_heads=8,
                                  dtype="bf16", seed=21)
     _check(wl, "f32", scale=scale)
+
+
+def test_full_chunked_prefill_70b():
+    # the workload and launch the benchmark times (16 sequences, 512-token chunks over
+    # 2048..4096-token contexts, GQA-8, bf16 out: the persistent tcgen05 kernel),
+    # checked on the shortest and the longest sequence and one in between
+    import bench
+
+    spec = dict(bench.PREFILL["chunked_prefill_70b"])
+    wl = W.make_prefill_workload(spec.pop("num_seqs"), spec.pop("context"), spec.pop("chunk"),
+                                 **spec)
+    d, out = _run(wl, "bf16")
+    L = wl.seq_lens.numpy()
+    seqs = sorted({int(L.argmin()), int(L.argmax()), 7})
+    qs = wl.query_start.numpy().astype(np.int64)
+    rows = np.concatenate([np.arange(qs[s], qs[s + 1]) for s in seqs])
+    nt = torch.as_tensor(rows)
+    kc, vc = oracle.reshape_and_cache(wl.new_key[nt], wl.new_value[nt], wl.key_cache,
+                                      wl.value_cache, wl.slot_mapping.numpy()[rows],
+                                      src_dtype=wl.src_dtype, cache_dtype=wl.cfg.cache_dtype)
+    sub_qs = np.concatenate([[0], np.cumsum([qs[s + 1] - qs[s] for s in seqs])])
+    ref = oracle.paged_attention_prefill(wl.query[nt], kc, vc, wl.block_tables.numpy()[seqs],
+                                         L[seqs], sub_qs, scale=wl.scale, q_dtype="bf16",
+                                         cache_dtype="bf16")
+    err = flow.max_abs_err(out[torch.as_tensor(rows, device=out.device)], ref)
+    assert err <= flow.TOL["bf16"], f"max abs error {err:.3e}"
+    assert torch.isfinite(out.float()).all()
