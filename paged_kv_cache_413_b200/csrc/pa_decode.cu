@@ -39,9 +39,10 @@ __device__ unsigned int g_decode_err;
 #define PA_MMA16_STAGES 4
 #endif
 #ifndef PA_SIMT_STAGES
-#define PA_SIMT_STAGES 8
+#define PA_SIMT_STAGES 4
 #endif
-constexpr int kStagesSimt = PA_SIMT_STAGES;     // 8 KB K+V per stage at D = 128, 16-bit
+constexpr int kStagesSimt = PA_SIMT_STAGES;     // 8 KB K+V per stage at D = 128, 16-bit;
+                                                // 4 stages: 6 CTAs per SM
 constexpr int kStagesMma16 = PA_MMA16_STAGES;   // 8 KB per stage; 4 CTAs per SM
 constexpr int kStagesMmaFp8 = 8;                // 4 KB per stage
 static_assert(kStagesSimt % kConsumerWarps == 0 && kStagesMma16 % kConsumerWarps == 0 &&
@@ -549,7 +550,10 @@ template <int GT, typename CT, typename QT, int kStages>
 // Resident CTAs per SM the register budget must allow: 5 for groups of 8 (a few
 // L1-cached spills; 0.903-0.910 -> 0.920 on the 70B-GQA workload), 4 for groups of
 // 4, where 5 measured slightly slower.
-__global__ void __launch_bounds__(kThreads, GT == 8 ? 5 : 4) decode_mma_kernel(
+#ifndef PA_MMA8_MIN_CTAS
+#define PA_MMA8_MIN_CTAS 5  // 6 (64 registers, more spills) measured 0.82
+#endif
+__global__ void __launch_bounds__(kThreads, GT == 8 ? PA_MMA8_MIN_CTAS : 4) decode_mma_kernel(
     const __grid_constant__ TmaParams tp) {
   constexpr int D = 128;
   constexpr bool kFp8 = CacheTraits<CT>::bytes == 1;
