@@ -39,7 +39,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_and_replica_seeds():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a threaded process
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     assert out[0][0] == [11.0, 2.0] and out[1][0] == [11.0, 2.0]
