@@ -21,12 +21,13 @@ import flow
 pytestmark = pytest.mark.gpu
 
 
-def _run(wl, out_dtype, scale=None):
+def _run(wl, out_dtype, scale=None, max_q=None):
     d = flow.to_device(wl)
     qs = wl.query_start.cuda()
     pa.pa_reshape_and_cache(d.new_key, d.new_value, d.key_cache, d.value_cache, d.slot_mapping)
     out = torch.full(d.query.shape, float("nan"), dtype=flow.TORCH_DT[out_dtype], device="cuda")
-    max_q = int((wl.query_start[1:] - wl.query_start[:-1]).max())
+    if max_q is None:
+        max_q = int((wl.query_start[1:] - wl.query_start[:-1]).max())
     pa.pa_paged_attention_prefill(out, d.query, d.key_cache, d.value_cache, d.block_tables,
                                   d.seq_lens, qs, max_query_len=max_q,
                                   max_seq_len=flow.max_seq_len(wl),
@@ -36,9 +37,9 @@ def _run(wl, out_dtype, scale=None):
     return d, out
 
 
-def _check(wl, out_dtype, scale=None):
+def _check(wl, out_dtype, scale=None, max_q=None):
     scale = wl.scale if scale is None else scale
-    d, out = _run(wl, out_dtype, scale)
+    d, out = _run(wl, out_dtype, scale, max_q)
     kc, vc = oracle.reshape_and_cache(wl.new_key, wl.new_value, wl.key_cache, wl.value_cache,
                                       wl.slot_mapping, src_dtype=wl.src_dtype,
                                       cache_dtype=wl.cfg.cache_dtype)
@@ -138,3 +139,16 @@ def test_full_chunked_prefill_70b():
     err = flow.max_abs_err(out[torch.as_tensor(rows, device=out.device)], ref)
     assert err <= flow.TOL["bf16"], f"max abs error {err:.3e}"
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("seed,chunk,dt", [(16, (0, 60), "bf16"), (0, (0, 8), "f16")])
+def test_prefill_empty_chunks_and_loose_bound(seed, chunk, dt):
+    # some sequences have no query rows this step (q_i = 0); the first case runs the
+    # tcgen05 kernel (up to 60 x 4 rows), the second the mma.sync one
+    wl = W.make_prefill_workload(6, (60, 400), chunk, num_heads=32, num_kv_heads=8, dtype=dt,
+                                 seed=seed)
+    q = (wl.query_start[1:] - wl.query_start[:-1]).numpy()
+    assert (q == 0).any()
+    _check(wl, dt)
+    # a host bound above the real longest chunk only adds tiles with no rows
+    _check(wl, dt, max_q=int(q.max()) * 3 + 5)
