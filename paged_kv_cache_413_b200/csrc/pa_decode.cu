@@ -1426,53 +1426,83 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
 
 // Log-sum-exp merge of the partitions of sequences with more than one:
 // M = max m_p, w_p = l_p exp(m_p - M), out = sum w_p o_p / sum w_p.
-// One warp per (sequence, head) row, 8 rows per CTA; lanes own D/32 dims.
+// One CTA of kReduceWarps warps per (sequence, head) row.  Warp w takes the
+// partitions p = w, w + kReduceWarps, ..., four at a time with their loads in
+// flight together; lanes own D/32 dims; the warps' sums meet in shared memory.
 // Launched as a programmatic dependent of the decode kernel: it waits for that
 // grid's results before reading the workspace.
+constexpr int kReduceWarps = 4;
+
 template <int D>
-__global__ void __launch_bounds__(256) lse_reduce_kernel(void* out, const float* __restrict__ ws_m,
-                                                         const float* __restrict__ ws_l,
-                                                         const float* __restrict__ ws_o,
-                                                         const int32_t* __restrict__ seq_lens,
-                                                         int num_rows, int num_heads,
-                                                         int max_parts, int partition, int cap,
-                                                         int out_dtype) {
+__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(
+    void* out, const float* __restrict__ ws_m, const float* __restrict__ ws_l,
+    const float* __restrict__ ws_o, const int32_t* __restrict__ seq_lens, int num_rows,
+    int num_heads, int max_parts, int partition, int cap, int out_dtype) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int DPL = D / 32;
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  __shared__ float s_max[kReduceWarps];
+  __shared__ float s_acc[kReduceWarps][D];
+  __shared__ float s_w[kReduceWarps];
+  const int row = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (row >= num_rows) return;
   int L = seq_lens[row / num_heads];
   L = L < 0 ? 0 : (L > cap ? cap : L);
   const int nparts = (L + partition - 1) / partition;
-  if (nparts <= 1) return;  // written by the decode kernel
+  if (nparts <= 1) return;  // written by the decode kernel (uniform over the CTA)
   const float* m = ws_m + int64_t(row) * max_parts;
   const float* l = ws_l + int64_t(row) * max_parts;
   const float* o = ws_o + int64_t(row) * max_parts * D + lane * DPL;
   float M = -INFINITY;
-  for (int q = lane; q < nparts; q += 32) M = fmaxf(M, m[q]);
+  for (int q = threadIdx.x; q < nparts; q += kReduceWarps * 32) M = fmaxf(M, m[q]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
+  if (lane == 0) s_max[warp] = M;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kReduceWarps; ++w) M = fmaxf(M, s_max[w]);
   float acc[DPL] = {};
   float W = 0.f;
-  for (int q = 0; q < nparts; ++q) {
-    const float w = l[q] * exp2f((m[q] - M) * kLog2e);
-    W += w;
-    if constexpr (DPL == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(o + int64_t(q) * D);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
-      acc[2] = fmaf(w, v.z, acc[2]);
-      acc[3] = fmaf(w, v.w, acc[3]);
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(o + int64_t(q) * D);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
+  int q = warp;
+  for (; q + 3 * kReduceWarps < nparts; q += 4 * kReduceWarps) {
+    float w4[4];
+    float v4[4][DPL];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int qq = q + u * kReduceWarps;
+      w4[u] = l[qq] * exp2f((m[qq] - M) * kLog2e);
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) v4[u][e] = o[int64_t(qq) * D + e];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      W += w4[u];
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w4[u], v4[u][e], acc[e]);
     }
   }
-  const float inv = 1.f / W;
+  for (; q < nparts; q += kReduceWarps) {
+    const float w = l[q] * exp2f((m[q] - M) * kLog2e);
+    W += w;
 #pragma unroll
-  for (int e = 0; e < DPL; ++e)
-    store_out(out, int64_t(row) * D + lane * DPL + e, acc[e] * inv, out_dtype);
+    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, o[int64_t(q) * D + e], acc[e]);
+  }
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) s_acc[warp][lane * DPL + e] = acc[e];
+  if (lane == 0) s_w[warp] = W;
+  __syncthreads();
+  if (warp == 0) {
+    float Wt = 0.f;
+#pragma unroll
+    for (int w = 0; w < kReduceWarps; ++w) Wt += s_w[w];
+    const float inv = 1.f / Wt;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kReduceWarps; ++w) t += s_acc[w][lane * DPL + e];
+      store_out(out, int64_t(row) * D + lane * DPL + e, t * inv, out_dtype);
+    }
+  }
 }
 
 template <int D, int GT, typename CT, typename QT>
@@ -1710,8 +1740,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
                       : a.max_blocks_per_seq * a.block_size;
   const int out_rows = a.num_seqs * a.num_heads;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned((out_rows + 7) / 8));
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3(unsigned(out_rows));
+  cfg.blockDim = dim3(kReduceWarps * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
