@@ -285,3 +285,52 @@ def test_prefill_first_query_of_a_full_prompt_sees_one_token():
     # query 1 (position 1): scores 0 and 2 over tokens 0, 1
     w = np.exp([0.0, 2.0]) / np.exp([0.0, 2.0]).sum()
     np.testing.assert_allclose(out[1, 0], w[0] * vc[0, 0, 0] + w[1] * vc[0, 0, 1], atol=1e-15)
+
+
+def _layout(rng, seqs_kv, bs, hkv, d):
+    """Scatter each sequence's logical [Hkv, L, D] K/V into bs-token blocks of a
+    shuffled pool; unused rows hold NaN.  Returns (kc, vc, tables)."""
+    nblk = [-(-kv[0].shape[1] // bs) for kv in seqs_kv]
+    nb = sum(nblk) + 3
+    phys = rng.permutation(nb)
+    kc = np.full((nb, hkv, bs, d), np.nan, dtype=np.float32)
+    vc = np.full((nb, hkv, bs, d), np.nan, dtype=np.float32)
+    bt = np.full((len(seqs_kv), max(nblk)), -1, dtype=np.int32)
+    nxt = 0
+    for i, (k, v) in enumerate(seqs_kv):
+        L = k.shape[1]
+        for j in range(nblk[i]):
+            b = phys[nxt]
+            nxt += 1
+            bt[i, j] = b
+            n = min(bs, L - j * bs)
+            kc[b, :, :n] = k[:, j * bs:j * bs + n]
+            vc[b, :, :n] = v[:, j * bs:j * bs + n]
+    return kc, vc, bt
+
+
+def test_block_size_relayout_is_bitwise_invariant():
+    # the same logical K/V, stored in 16-, 32-, 64- or 128-token blocks of a shuffled
+    # pool, gives bit-identical decode and chunked-prefill outputs
+    rng = np.random.default_rng(12)
+    hkv, d, h = 2, 16, 8
+    lens = [1, 15, 16, 17, 63, 64, 65, 130]
+    f32 = lambda *shape: rng.standard_normal(shape).astype(np.float32)
+    seqs = [(f32(hkv, L, d), f32(hkv, L, d)) for L in lens]
+    q = f32(len(lens), h, d)
+    nq = [min(L, 3) for L in lens]
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    qp = f32(int(qs[-1]), h, d)
+    sl = np.array(lens, np.int32)
+    dec, pre = [], []
+    for bs in (16, 32, 64, 128):
+        kc, vc, bt = _layout(np.random.default_rng(bs), seqs, bs, hkv, d)
+        dec.append(oracle.paged_attention_decode(q, kc, vc, bt, sl, scale=0.4, q_dtype="f32",
+                                                 cache_dtype="f32"))
+        pre.append(oracle.paged_attention_prefill(qp, kc, vc, bt, sl, qs, scale=0.4,
+                                                  q_dtype="f32", cache_dtype="f32"))
+    for a in dec[1:]:
+        assert np.array_equal(a, dec[0])
+    for a in pre[1:]:
+        assert np.array_equal(a, pre[0])
+    assert np.isfinite(dec[0]).all() and np.isfinite(pre[0]).all()

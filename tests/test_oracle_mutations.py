@@ -31,6 +31,8 @@ MUTANTS = {
     "f16_subnormal": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
     "dequant_scale_dropped": ("        k *= k_scale;\n", "\n"),
     "swap_wrong_pool": ("(const char*)src_key_caches[l] + src * block_bytes", "(const char*)dst_key_caches[l] + src * block_bytes"),
+    "blocks_of_16": ("int64_t phys = table[l / block_size];\n    int64_t off = l % block_size;",
+                     "int64_t phys = table[l / 16];\n    int64_t off = l % 16;"),
     "prefill_not_causal": ("attend_rows(out + row, NULL, NULL, q, K, V, 0, pos + 1, head_dim, scale, sc);", "attend_rows(out + row, NULL, NULL, q, K, V, 0, L, head_dim, scale, sc);"),
     "copy_wrong_direction": ("memcpy((char*)key_caches[l] + dst * block_bytes, (char*)key_caches[l] + src * block_bytes,",
                              "memcpy((char*)key_caches[l] + src * block_bytes, (char*)key_caches[l] + dst * block_bytes,"),
