@@ -33,6 +33,10 @@ MUTANTS = {
     "swap_wrong_pool": ("(const char*)src_key_caches[l] + src * block_bytes", "(const char*)dst_key_caches[l] + src * block_bytes"),
     "blocks_of_16": ("int64_t phys = table[l / block_size];\n    int64_t off = l % block_size;",
                      "int64_t phys = table[l / 16];\n    int64_t off = l % 16;"),
+    "prefill_position_off_by_one": ("int pos = L - nq + j; /* this query token's position */",
+                                    "int pos = L - nq + j - 1; /* this query token's position */"),
+    "prefill_gqa_interleaved": ("int h = kvh * group + g;\n          int64_t row = ((int64_t)(q0 + j)",
+                                "int h = g * num_kv_heads + kvh;\n          int64_t row = ((int64_t)(q0 + j)"),
     "prefill_not_causal": ("attend_rows(out + row, NULL, NULL, q, K, V, 0, pos + 1, head_dim, scale, sc);", "attend_rows(out + row, NULL, NULL, q, K, V, 0, L, head_dim, scale, sc);"),
     "copy_wrong_direction": ("memcpy((char*)key_caches[l] + dst * block_bytes, (char*)key_caches[l] + src * block_bytes,",
                              "memcpy((char*)key_caches[l] + src * block_bytes, (char*)key_caches[l] + dst * block_bytes,"),
