@@ -906,6 +906,14 @@ struct SharedParams {
 };
 
 constexpr int kSharedCols = 16;  // query heads per CTA (two n8 tiles)
+constexpr float kSharedRescaleLog2 = 8.f;  // lazy running max: largest weight 2^8
+
+// 2^x by the MUFU approximation (inputs here are <= 8 or -inf; -inf gives 0)
+__device__ __forceinline__ float ex2_approx_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 #ifndef PA_SHARED_MIN_CHUNK
 #define PA_SHARED_MIN_CHUNK 128      // fewest blocks per CTA when a unit is split
 #endif
@@ -1214,16 +1222,20 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
           mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
           mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
         }
-        const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+        // lazy running max: it moves only when a tile's max passes it by more than
+        // 2^8, so weights stay <= 256 and most tiles skip the accumulator rescale;
+        // O and l are always relative to the same max, so the result is unchanged
+        const float mn0 = mx0 > m[nt][0] + kSharedRescaleLog2 ? mx0 : m[nt][0];
+        const float mn1 = mx1 > m[nt][1] + kSharedRescaleLog2 ? mx1 : m[nt][1];
         // a column that has seen no token yet keeps m = -inf: scale 1, weights 0
-        al[nt][0] = mn0 == -INFINITY ? 1.f : exp2f(m[nt][0] - mn0);
-        al[nt][1] = mn1 == -INFINITY ? 1.f : exp2f(m[nt][1] - mn1);
+        al[nt][0] = mn0 == -INFINITY ? 1.f : ex2_approx_ftz(m[nt][0] - mn0);
+        al[nt][1] = mn1 == -INFINITY ? 1.f : ex2_approx_ftz(m[nt][1] - mn1);
         m[nt][0] = mn0;
         m[nt][1] = mn1;
-        const float p0 = mn0 == -INFINITY ? 0.f : exp2f(sc[nt][0] - mn0);
-        const float p1 = mn1 == -INFINITY ? 0.f : exp2f(sc[nt][1] - mn1);
-        const float p2 = mn0 == -INFINITY ? 0.f : exp2f(sc[nt][2] - mn0);
-        const float p3 = mn1 == -INFINITY ? 0.f : exp2f(sc[nt][3] - mn1);
+        const float p0 = mn0 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][0] - mn0);
+        const float p1 = mn1 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][1] - mn1);
+        const float p2 = mn0 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][2] - mn0);
+        const float p3 = mn1 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][3] - mn1);
         l[nt][0] = l[nt][0] * al[nt][0] + (p0 + p2);
         l[nt][1] = l[nt][1] * al[nt][1] + (p1 + p3);
         const uint32_t x0 = pack2(p0, p1, MT{}), x1 = pack2(p2, p3, MT{});
@@ -1236,15 +1248,17 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
           bl1[nt] = movmatrix_trans(pack2(p2 - h1.x, p3 - h1.y, MT{}));
         }
       }
+      if (__any_sync(kFullMask, al[0][0] != 1.f || al[0][1] != 1.f || al[1][0] != 1.f ||
+                                    al[1][1] != 1.f))
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
+        for (int t = 0; t < 8; ++t)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          acc[t][nt][0] *= al[nt][0];
-          acc[t][nt][1] *= al[nt][1];
-          acc[t][nt][2] *= al[nt][0];
-          acc[t][nt][3] *= al[nt][1];
-        }
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[t][nt][0] *= al[nt][0];
+            acc[t][nt][1] *= al[nt][1];
+            acc[t][nt][2] *= al[nt][0];
+            acc[t][nt][3] *= al[nt][1];
+          }
       uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
       if (nvalid < kBlockSize) {
         mlo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
