@@ -55,3 +55,50 @@ def test_prefill_flops_enumerated():
             for _key in range(pos + 1):
                 pairs += 1
     assert bench.prefill_flops(wl) == pairs * cfg.num_heads * cfg.head_dim * 4
+
+
+def _profile_record(path, key):
+    import re
+    text = open(path).read()
+    sha = re.search(key + r":\s*([0-9a-f]{16})", text)
+    dram = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    return sha.group(1), int(dram.group(1))
+
+
+def test_recorded_traffic_only_while_the_profiled_sources_hash_the_same(monkeypatch):
+    """A committed ncu figure is reported only for the sources it was taken on."""
+    import glob
+    import os
+    decode = sorted(glob.glob(os.path.join(bench.ROOT, "profiles",
+                                           "paged_attention_decode_*.md")))
+    prefill = sorted(glob.glob(os.path.join(bench.ROOT, "profiles", "prefill_tc_*.md")))
+    assert decode and prefill
+    now_d = bench.source_sha(bench.DECODE_SOURCES)
+    now_p = bench.source_sha(bench.PREFILL_SOURCES)
+    for path in decode:
+        cfg = os.path.basename(path)[len("paged_attention_decode_"):-3]
+        sha, dram = _profile_record(path, "decode_source_sha256_16")
+        assert bench.recorded_traffic(cfg) == (dram if sha == now_d else None)
+    for path in prefill:
+        cfg = os.path.basename(path)[len("prefill_tc_"):-3]
+        sha, dram = _profile_record(path, "prefill_source_sha256_16")
+        assert bench.recorded_prefill_traffic(cfg) == (dram if sha == now_p else None)
+    # both branches, whatever the committed sources hash to: the figure while the
+    # hash matches, none after any change
+    for path in decode:
+        cfg = os.path.basename(path)[len("paged_attention_decode_"):-3]
+        sha, dram = _profile_record(path, "decode_source_sha256_16")
+        monkeypatch.setattr(bench, "source_sha", lambda names=None, s=sha: s)
+        assert bench.recorded_traffic(cfg) == dram
+        monkeypatch.setattr(bench, "source_sha", lambda names=None: "0" * 16)
+        assert bench.recorded_traffic(cfg) is None
+    for path in prefill:
+        cfg = os.path.basename(path)[len("prefill_tc_"):-3]
+        sha, dram = _profile_record(path, "prefill_source_sha256_16")
+        monkeypatch.setattr(bench, "source_sha", lambda names=None, s=sha: s)
+        assert bench.recorded_prefill_traffic(cfg) == dram
+        monkeypatch.setattr(bench, "source_sha", lambda names=None: "0" * 16)
+        assert bench.recorded_prefill_traffic(cfg) is None
+    # and a workload without a profile has none
+    monkeypatch.undo()
+    assert bench.recorded_traffic("no_such_workload") is None
