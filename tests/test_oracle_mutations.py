@@ -40,6 +40,12 @@ MUTANTS = {
     "prefill_not_causal": ("attend_rows(out + row, NULL, NULL, q, K, V, 0, pos + 1, head_dim, scale, sc);", "attend_rows(out + row, NULL, NULL, q, K, V, 0, L, head_dim, scale, sc);"),
     "copy_wrong_direction": ("memcpy((char*)key_caches[l] + dst * block_bytes, (char*)key_caches[l] + src * block_bytes,",
                              "memcpy((char*)key_caches[l] + src * block_bytes, (char*)key_caches[l] + dst * block_bytes,"),
+    "partition_overlap": ("int lo = p * partition_size, hi = lo + partition_size;",
+                          "int lo = p * partition_size, hi = lo + partition_size + 1;"),
+    "reshape_value_from_key": ("memcpy((char*)value_cache + dst_row * ec, (const char*)value + src_row * es,",
+                               "memcpy((char*)value_cache + dst_row * ec, (const char*)key + src_row * es,"),
+    "bf16_shift": ("uint32_t u = (uint32_t)b << 16;", "uint32_t u = (uint32_t)b << 15;"),
+    "merge_not_normalised": ("    for (int d = 0; d < head_dim; ++d) out[r * head_dim + d] /= W;\n", "\n"),
 }
 
 
