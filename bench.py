@@ -146,6 +146,7 @@ def measured_peak():
 DECODE_SOURCES = ("pa_decode.cu", "pa_kernels.cuh", "pa_common.cuh", "pa_internal.h")
 PREFILL_SOURCES = ("pa_prefill.cu", "pa_tcgen05.cuh", "pa_kernels.cuh", "pa_common.cuh",
                    "pa_internal.h")
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def source_sha(names=DECODE_SOURCES) -> str:
@@ -157,39 +158,29 @@ def source_sha(names=DECODE_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def decode_source_sha() -> str:
-    return source_sha(DECODE_SOURCES)
-
-
-def recorded_prefill_traffic(config: str):
-    """DRAM bytes per prefill launch from the committed ncu summary of this workload,
-    valid only while the prefill sources are the ones that were profiled."""
-    path = os.path.join(ROOT, "profiles", f"prefill_tc_{config}.md")
+def recorded_traffic(workload: str):
+    """DRAM bytes (read + written) per launch of the workload's hot kernel, from the
+    ncu capture recorded in profiles/traffic.json; None unless the sources it
+    lists still hash to the value recorded with the capture."""
     try:
-        text = open(path).read()
-        m = re.search(r"prefill_source_sha256_16:\s*([0-9a-f]{16})", text)
-        t = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-        if m and t and m.group(1) == source_sha(PREFILL_SOURCES):
-            return int(t.group(1))
-    except OSError:
+        with open(TRAFFIC_JSON) as f:
+            rec = json.load(f)["workloads"][workload]
+        if source_sha(tuple(rec["sources"])) == rec["sources_sha256_16"]:
+            return int(rec["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError, TypeError):
         pass
     return None
 
 
-def recorded_traffic(config: str):
-    """DRAM bytes per decode launch from the committed ncu summary of this workload,
-    valid only while the decode source is the one that was profiled."""
-    path = os.path.join(ROOT, "profiles", f"paged_attention_decode_{config}.md")
+def cpu_model() -> str:
     try:
-        text = open(path).read()
-        sha = decode_source_sha()
-        m = re.search(r"decode_source_sha256_16:\s*([0-9a-f]{16})", text)
-        t = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-        if m and t and m.group(1) == sha:
-            return int(t.group(1))
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
     except OSError:
         pass
-    return None
+    return "unknown"
 
 
 class ClockSampler:
@@ -274,7 +265,9 @@ def oracle_sample(wl: W.Workload, seqs, out_dtype: str):
 
 
 def cpu_baseline(wl: W.Workload, out_dtype: str, budget_s: float = 12.0):
-    """The oracle timed on a bounded sample of the workload's sequences."""
+    """The oracle timed on a bounded sample of the workload's sequences, with all the
+    host's OpenMP threads and then with one thread on the same sample (or on a
+    prefix of it when one thread would exceed the budget)."""
     import oracle
 
     n = wl.seq_lens.numel()
@@ -282,10 +275,19 @@ def cpu_baseline(wl: W.Workload, out_dtype: str, budget_s: float = 12.0):
     dt1, _ = oracle_sample(wl, order[:1], out_dtype)              # calibration
     k = int(max(1, min(n, budget_s / max(dt1, 1e-4))))
     dt, b = oracle_sample(wl, order[:k], out_dtype)
-    return {"value": b / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+    cores = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        k1 = int(max(1, min(k, k * budget_s / max(dt * cores, 1e-4))))
+        dt_1, b_1 = oracle_sample(wl, order[:k1], out_dtype)
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": b / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"{k} of {n} sequences of the workload (cache write of their new "
-                      f"tokens + fp64 decode), {dt:.1f} s"}
+                      f"tokens + fp64 decode), {dt:.1f} s",
+            "single_thread": {"value": b_1 / dt_1 / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": f"{k1} of the same sequences, {dt_1:.1f} s"}}
 
 
 def prefill_oracle_sample(wl: W.Workload, seqs):
@@ -315,7 +317,8 @@ def prefill_oracle_sample(wl: W.Workload, seqs):
 
 
 def prefill_cpu_baseline(wl: W.Workload, budget_s: float = 15.0):
-    """The oracle timed on a bounded sample of the workload's sequences."""
+    """The oracle timed on a bounded sample of the workload's sequences (all threads,
+    then one thread on the same sample or a prefix of it)."""
     import oracle
 
     n = wl.seq_lens.numel()
@@ -323,10 +326,19 @@ def prefill_cpu_baseline(wl: W.Workload, budget_s: float = 15.0):
     dt1, _ = prefill_oracle_sample(wl, order[:1])              # calibration
     k = int(max(1, min(n, budget_s / max(dt1, 1e-4))))
     dt, fl = prefill_oracle_sample(wl, order[:k])
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+    cores = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        k1 = int(max(1, min(k, k * budget_s / max(dt * cores, 1e-4))))
+        dt_1, fl_1 = prefill_oracle_sample(wl, order[:k1])
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"{k} of {n} sequences of the workload (cache write of their chunks + "
-                      f"fp64 causal attention), {dt:.1f} s"}
+                      f"fp64 causal attention), {dt:.1f} s",
+            "single_thread": {"value": fl_1 / dt_1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                              "sample": f"{k1} of the same sequences, {dt_1:.1f} s"}}
 
 
 def pipelined_e2e(dev, stream, inputs, host_src, out, run_step, steps, world):
@@ -392,14 +404,51 @@ def pipelined_e2e(dev, stream, inputs, host_src, out, run_step, steps, world):
 
 
 # ---------------------------------------------------------------- GPU arm
-def run_ours(args, rank, world, local_rank):
+def timed_loop(step, launches, steps, warmup, dev, stream, world, rank):
+    """`warmup` untimed steps, then exactly `steps` timed ones bracketed by a
+    barrier and a device synchronize on both sides, with clocks sampled meanwhile
+    on rank 0.  step(timed) appends its hot launch's (start, end) events to
+    `launches` when timed.  Returns (max-over-ranks elapsed ms, mean launch ms,
+    clock summary or None)."""
+    for _ in range(warmup):
+        step(False)
+    torch.cuda.synchronize(dev)
     import paged_kv_cache_413_b200 as pa
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    cfg = W.CONFIGS[args.config]
-    if args.block_size:
-        cfg = cfg.scaled(block_size=args.block_size)
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error bits set during warm-up")
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.__enter__()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches.clear()
+    t0.record(stream)
+    for _ in range(steps):
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    if sampler:
+        sampler.__exit__(None, None, None)
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error bits set during the timed steps")
+    elapsed_ms = t0.elapsed_time(t1)
+    launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in launches)
+    elapsed_ms, launch_ms = max_over_ranks([elapsed_ms, launch_ms], world, dev)
+    return elapsed_ms, launch_ms, (sampler.summary() if sampler else None)
+
+
+def decode_case(cfg, dev, args, world, rank, decode_mode="auto", partition=None,
+                with_e2e=True, with_cpu=False):
+    """One decode workload, resident in HBM: W + K steps of (copy-on-write copies,
+    cache write, decode), timed as a whole and per decode launch; optionally end to
+    end through the public API with host buffers, and the CPU oracle baseline."""
+    import paged_kv_cache_413_b200 as pa
+
     wl = W.make_workload(cfg, seed=cfg.seed + 1000 * rank) if rank else W.make_workload(cfg)
     out_dtype = cfg.out_dtype
     f = lambda t: None if t is None else t.to(dev)
@@ -408,7 +457,7 @@ def run_ours(args, rank, world, local_rank):
     nk, nv, sm = f(wl.new_key), f(wl.new_value), f(wl.slot_mapping)
     bm = f(wl.block_mapping) if wl.block_mapping is not None and wl.block_mapping.numel() else None
     max_len = int(wl.seq_lens.max())
-    part = args.partition if args.partition is not None else cfg.partition_size
+    part = partition if partition is not None else cfg.partition_size
     ws_n = pa.pa_paged_attention_workspace_size(q.shape[0], cfg.num_heads, cfg.num_kv_heads,
                                                 cfg.head_dim, max_len, part)
     ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
@@ -421,14 +470,12 @@ def run_ours(args, rank, world, local_rank):
     part_eff = pa.pa_paged_attention_partition_size(q.shape[0], cfg.num_heads, cfg.num_kv_heads,
                                                     max_len, part)
     reduce_runs = max_len > part_eff
-    launches = 1 + 1 + (1 if reduce_runs else 0) + (1 if bm is not None else 0)
-
-    shared = wl.group_starts is not None and args.decode in ("auto", "shared")
+    shared = wl.group_starts is not None and decode_mode in ("auto", "shared")
+    launches = 1 + 1 + (1 if bm is not None else 0) + (1 if reduce_runs and not shared else 0)
     gs = pl = None
     if shared:
         gs, pl = f(wl.group_starts), f(wl.prefix_lens)
         max_group = int((wl.group_starts[1:] - wl.group_starts[:-1]).max())
-        launches -= 1 if reduce_runs else 0  # the shared-prefix decode needs no merge
     ev = []
     # the step's inputs: what a serving loop hands over every step
     inputs = {"q": q, "nk": nk, "nv": nv, "sm": sm, "bt": bt, "sl": sl}
@@ -443,8 +490,7 @@ def run_ours(args, rank, world, local_rank):
         pa.pa_reshape_and_cache(t["nk"], t["nv"], kc, vc, t["sm"], k_scale=wl.k_scale,
                                 v_scale=wl.v_scale)
         if timed:
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
         if shared:
             pa.pa_paged_attention_decode_shared_prefix(
@@ -460,60 +506,62 @@ def run_ours(args, rank, world, local_rank):
             e1.record(stream)
             ev.append((e0, e1))
 
-    def step(timed: bool):
-        run_step(inputs, out, timed)
-
-    for _ in range(args.warmup):
-        step(False)
-    torch.cuda.synchronize(dev)
-    if pa.pa_get_device_error() != 0:
-        raise RuntimeError("device error bits set during warm-up")
-
-    sampler = ClockSampler(local_rank) if rank == 0 else None
-    if sampler:
-        sampler.__enter__()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step(True)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    if sampler:
-        sampler.__exit__(None, None, None)
-    elapsed_ms = t0.elapsed_time(t1)
-    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    elapsed_ms, decode_ms = max_over_ranks([elapsed_ms, decode_ms], world, dev)
-    if pa.pa_get_device_error() != 0:
-        raise RuntimeError("device error bits set during the timed steps")
-
+    elapsed_ms, decode_ms, clocks = timed_loop(lambda timed: run_step(inputs, out, timed), ev,
+                                               args.steps, args.warmup, dev, stream, world, rank)
     dec_b = shared_decode_bytes(wl, out_dtype) if shared else decode_bytes(wl, out_dtype)
     step_bytes = dec_b + cache_write_bytes(wl) + copy_bytes(wl)
-    ms_per_step = elapsed_ms / args.steps
-    value = whole_job_gbs(step_bytes, world, args.steps, elapsed_ms)
+    res = {"wl": wl, "shared": shared, "part_eff": part_eff, "dec_b": dec_b,
+           "step_bytes": step_bytes, "elapsed_ms": elapsed_ms, "decode_ms": decode_ms,
+           "clocks": clocks, "launches": launches, "out_dtype": out_dtype}
+    if with_e2e:
+        host_src = {"q": wl.query, "nk": wl.new_key, "nv": wl.new_value, "sm": wl.slot_mapping,
+                    "bt": wl.block_tables, "sl": wl.seq_lens, "bm": wl.block_mapping,
+                    "gs": wl.group_starts, "pl": wl.prefix_lens}
+        e2e_steps = max(10, args.steps // 4)
+        e2e_ms, h2d, d2h = pipelined_e2e(dev, stream, inputs, host_src, out, run_step,
+                                         e2e_steps, world)
+        res["e2e"] = (max_over_ranks([e2e_ms], world, dev)[0], e2e_steps, h2d, d2h)
+    if with_cpu and not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline(wl, out_dtype)
+    return res
 
-    # ---- end to end through the public API with host buffers
-    host_src = {"q": wl.query, "nk": wl.new_key, "nv": wl.new_value, "sm": wl.slot_mapping,
-                "bt": wl.block_tables, "sl": wl.seq_lens, "bm": wl.block_mapping,
-                "gs": wl.group_starts, "pl": wl.prefix_lens}
-    e2e_steps = max(10, args.steps // 4)
-    e2e_ms, h2d, d2h = pipelined_e2e(dev, stream, inputs, host_src, out, run_step, e2e_steps,
-                                     world)
-    e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
-    e2e_value = whole_job_gbs(step_bytes, world, e2e_steps, e2e_ms)
 
+def decode_roofline(r, peak, peak_kind, traffic):
+    achieved = r["dec_b"] / (r["decode_ms"] * 1e-3) / 1e9
+    return {"bound": "hbm",
+            "kernel": ("paged_attention_decode_shared_prefix" if r["shared"] else
+                       "paged_attention_decode (+ LSE reduce)"),
+            "achieved": round(achieved, 2), "peak": peak,
+            "peak_kind": f"{peak_kind} (hbm_gbs, copy burst)", "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "algorithmic_bytes_per_launch": r["dec_b"],
+            "launch_ms": round(r["decode_ms"], 5)}
+
+
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = W.CONFIGS[args.config]
+    if args.block_size:
+        cfg = cfg.scaled(block_size=args.block_size)
+    part = args.partition if args.partition is not None else cfg.partition_size
+    r = decode_case(cfg, dev, args, world, rank, args.decode, part, with_e2e=True,
+                    with_cpu=(rank == 0))
+    extra = {}
+    if args.config == DEFAULT_CONFIG and not args.no_configs and not args.block_size and \
+            args.partition is None:
+        extra = other_configs(dev, args, world, rank)
     if rank != 0:
         return None
+    wl, out_dtype = r["wl"], r["out_dtype"]
     peak, peak_kind = measured_peak()
-    achieved = dec_b / (decode_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(args.config)
+    ms_per_step = r["elapsed_ms"] / args.steps
+    value = whole_job_gbs(r["step_bytes"], world, args.steps, r["elapsed_ms"])
+    e2e_ms, e2e_steps, h2d, d2h = r["e2e"]
     L = wl.seq_lens.numpy().astype(np.int64)
     n_seqs = len(L)
+    traffic_key = args.config if args.decode != "standard" or wl.group_starts is None \
+        else args.config + "_per_sequence"
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
@@ -521,36 +569,227 @@ def run_ours(args, rank, world, local_rank):
         "kv_dtype": cfg.cache_dtype, "data": "synthetic",
         "config": {"workload": f"{args.config}: {DESCR[args.config]}",
                    "block_size": cfg.block_size,
-                   "partition_tokens": part_eff, "out_dtype": out_dtype,
+                   "partition_tokens": r["part_eff"], "out_dtype": out_dtype,
                    "l2": "no flush: inputs larger than L2 (%.2f GB read per step vs 126 MB L2)"
-                         % (dec_b / 1e9),
+                         % (r["dec_b"] / 1e9),
                    "parallelism": f"replicas x{world}"},
         "pct_of_peak": round(100.0 * value / peak, 2),
         "decode_tokens_per_s_per_layer": round(n_seqs * world / (ms_per_step * 1e-3), 1),
         "context_tokens_per_s_per_layer": round(int(L.sum()) * world / (ms_per_step * 1e-3), 1),
-        "roofline": {"bound": "hbm",
-                     "kernel": ("paged_attention_decode_shared_prefix" if shared else
-                                "paged_attention_decode (+ LSE reduce)"),
-                     "achieved": round(achieved, 2), "peak": peak,
-                     "peak_kind": f"{peak_kind} (hbm_gbs, copy burst)", "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes_per_launch": dec_b,
-                     "launch_ms": round(decode_ms, 5)},
-        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "ms_per_step": round(e2e_ms / e2e_steps, 5)},
-        "gpu_launches": launches * args.steps,
-        "clocks": sampler.summary() if sampler else None,
+        "roofline": decode_roofline(r, peak, peak_kind,
+                                    None if args.block_size or args.partition is not None
+                                    else recorded_traffic(traffic_key)),
+        "e2e": {"value": round(whole_job_gbs(r["step_bytes"], world, e2e_steps, e2e_ms), 2),
+                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 5)},
+        "gpu_launches": r["launches"] * args.steps,
+        "clocks": r["clocks"],
     }
     if wl.prefix_key is not None:
         logical = decode_bytes(wl, out_dtype)
-        line["decode_bytes"] = {"distinct": dec_b if shared else shared_decode_bytes(wl, out_dtype),
+        line["decode_bytes"] = {"distinct": r["dec_b"] if r["shared"] else
+                                shared_decode_bytes(wl, out_dtype),
                                 "per_sequence": logical,
-                                "per_sequence_gbs": round(logical / (decode_ms * 1e-3) / 1e9, 2)}
-        line["config"]["decode"] = "shared-prefix" if shared else "per-sequence"
-    if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(wl, out_dtype)
+                                "per_sequence_gbs": round(logical / (r["decode_ms"] * 1e-3) / 1e9,
+                                                          2)}
+        line["config"]["decode"] = "shared-prefix" if r["shared"] else "per-sequence"
+    if "cpu_baseline" in r:
+        line["cpu_baseline"] = r["cpu_baseline"]
+    if extra:
+        line["configs"] = extra
     return line
+
+
+def decode_entry(name, r, steps, world, peak, peak_kind, traffic_key):
+    """The `configs` map entry of one decode workload (rank 0)."""
+    wl = r["wl"]
+    ms_per_step = r["elapsed_ms"] / steps
+    L = wl.seq_lens.numpy().astype(np.int64)
+    roof = decode_roofline(r, peak, peak_kind, recorded_traffic(traffic_key))
+    e = {"workload": f"{name}: {DESCR[name]}",
+         "decode": ("shared-prefix" if r["shared"] else "per-sequence"),
+         "launch_ms": roof["launch_ms"], "algorithmic_bytes_per_launch": r["dec_b"],
+         "achieved_gbs": roof["achieved"], "frac": roof["frac"], "peak": peak,
+         "peak_kind": roof["peak_kind"], "traffic": roof["traffic"],
+         "step_value": round(whole_job_gbs(r["step_bytes"], world, steps, r["elapsed_ms"]), 2),
+         "unit": "GB/s", "ms_per_step": round(ms_per_step, 5), "steps": steps,
+         "partition_tokens": r["part_eff"],
+         "decode_tokens_per_s_per_layer": round(len(L) * world / (ms_per_step * 1e-3), 1),
+         "context_tokens_per_s_per_layer": round(int(L.sum()) * world / (ms_per_step * 1e-3), 1),
+         "gpu_launches": r["launches"] * steps, "clocks": r["clocks"]}
+    if wl.prefix_key is not None:
+        logical = decode_bytes(wl, r["out_dtype"])
+        e["per_sequence_bytes"] = logical
+        e["per_sequence_gbs"] = round(logical / (r["decode_ms"] * 1e-3) / 1e9, 2)
+        e["distinct_bytes"] = r["dec_b"] if r["shared"] else shared_decode_bytes(wl, r["out_dtype"])
+    return e
+
+
+def other_configs(dev, args, world, rank):
+    """Every other workload of the benchmark set, each resident in HBM and timed the
+    same way (W warm-up + K timed steps, per-launch CUDA events, clocks): the
+    70B-shaped GQA decode, the long-context split-K decode, the beam-search
+    copy-on-write FP8 step (shared-prefix decode, and the per-sequence decode of
+    the same step), the chunked prefill, and the beam pool's block swaps."""
+    peak, peak_kind = measured_peak()
+    out = {}
+    for name, mode, key in (("llama2_70b_gqa", "auto", "llama2_70b_gqa"),
+                            ("long_splitk", "auto", "long_splitk"),
+                            ("beam_cow_fp8", "shared", "beam_cow_fp8"),
+                            ("beam_cow_fp8", "standard", "beam_cow_fp8_per_sequence")):
+        r = decode_case(W.CONFIGS[name], dev, args, world, rank, mode, None, with_e2e=False)
+        if rank == 0:
+            out[key] = decode_entry(name, r, args.steps, world, peak, peak_kind, key)
+        del r
+        torch.cuda.empty_cache()
+    p = prefill_case("chunked_prefill_70b", dev, args, world, rank, with_e2e=False)
+    if rank == 0:
+        out["chunked_prefill_70b"] = prefill_entry("chunked_prefill_70b", p, args.steps, world)
+    del p
+    torch.cuda.empty_cache()
+    sw = swap_case(dev, args, world, rank)
+    if rank == 0:
+        out["swap_blocks_beam"] = sw
+    torch.cuda.empty_cache()
+    return out
+
+
+def swap_case(dev, args, world, rank):
+    """swap_blocks on the beam workload's pool: the 192 copy-on-write blocks of one
+    layer (K and V) out to page-locked host memory and back, one launch each way
+    (the kernel reads and writes host memory through its mapping), against one
+    cudaMemcpyAsync per block and pool; then the swaps on a second stream while the
+    shared-prefix decode runs, and the decode's slowdown."""
+    import paged_kv_cache_413_b200 as pa
+
+    cfg = W.CONFIGS["beam_cow_fp8"]
+    wl = W.make_workload(cfg, seed=cfg.seed + 1000 * rank) if rank else W.make_workload(cfg)
+    f = lambda t: t.to(dev)
+    kc, vc = f(wl.key_cache), f(wl.value_cache)
+    pa.pa_reshape_and_cache(f(wl.prefix_key), f(wl.prefix_value), kc, vc,
+                            f(wl.prefix_slot_mapping), k_scale=wl.k_scale, v_scale=wl.v_scale)
+    pa.pa_copy_blocks([kc], [vc], f(wl.block_mapping))
+    pa.pa_reshape_and_cache(f(wl.new_key), f(wl.new_value), kc, vc, f(wl.slot_mapping),
+                            k_scale=wl.k_scale, v_scale=wl.v_scale)
+    # out: the beams' own blocks (the decode reads them too); in: as many blocks that
+    # no sequence owns, so that the swaps never write what the decode reads
+    blocks = wl.block_mapping[:, 1].clone()
+    n = blocks.numel()
+    owned = set(int(b) for b in wl.block_tables.flatten().tolist() if b >= 0)
+    free = torch.tensor([b for b in range(wl.num_blocks) if b not in owned][:n])
+    if free.numel() < n:
+        raise RuntimeError("the beam pool has too few free blocks for the swap measurement")
+    host_k = torch.empty((n,) + tuple(kc.shape[1:]), dtype=kc.dtype).pin_memory()
+    host_v = torch.empty_like(host_k).pin_memory()
+    out_map = torch.stack([blocks, torch.arange(n)], 1).contiguous().to(dev)   # dev -> host
+    in_map = torch.stack([torch.arange(n), free], 1).contiguous().to(dev)      # host -> dev
+    blocks_d, free_d = blocks.to(dev), free.to(dev)
+    block_bytes = kc[0].numel() * kc.element_size()
+    moved = 2 * n * block_bytes                                  # K + V, one direction
+    side = torch.cuda.Stream(dev)
+    main = torch.cuda.current_stream(dev)
+    reps = max(5, min(args.steps, 200))
+
+    def swap_pair():
+        pa.pa_swap_blocks([host_k], [host_v], [kc], [vc], out_map, stream=side)
+        pa.pa_swap_blocks([kc], [vc], [host_k], [host_v], in_map, stream=side)
+
+    src_ids, dst_ids = blocks.tolist(), free.tolist()
+
+    def memcpy_pair():
+        with torch.cuda.stream(side):
+            for i, b in enumerate(src_ids):
+                host_k[i].copy_(kc[b], non_blocking=True)
+                host_v[i].copy_(vc[b], non_blocking=True)
+            for i, b in enumerate(dst_ids):
+                kc[b].copy_(host_k[i], non_blocking=True)
+                vc[b].copy_(host_v[i], non_blocking=True)
+
+    def time_on_side(fn, k):
+        for _ in range(3):
+            fn()
+        side.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(side)
+        for _ in range(k):
+            fn()
+        e1.record(side)
+        side.synchronize()
+        return e0.elapsed_time(e1) / k
+
+    swap_ms = time_on_side(swap_pair, reps)
+    kb, vb = kc.view(torch.uint8), vc.view(torch.uint8)
+    kb[free_d] = 0x7F                                           # E4M3 NaN: the swap-in must
+    vb[free_d] = 0x7F                                           # rewrite every byte
+    torch.cuda.synchronize(dev)
+    swap_pair()
+    side.synchronize()
+    if not (torch.equal(kb[free_d], kb[blocks_d]) and torch.equal(vb[free_d], vb[blocks_d])):
+        raise RuntimeError("the blocks swapped out and back in differ from the originals")
+    memcpy_reps = max(3, min(reps, 20))
+    memcpy_ms = time_on_side(memcpy_pair, memcpy_reps)
+    torch.cuda.synchronize(dev)
+
+    # overlap: the shared-prefix decode on the main stream, alone and with swaps
+    gs, pl = f(wl.group_starts), f(wl.prefix_lens)
+    q, bt, sl = f(wl.query), f(wl.block_tables), f(wl.seq_lens)
+    outd = torch.empty(q.shape, dtype=TORCH_DT[cfg.out_dtype], device=dev)
+    max_len = int(wl.seq_lens.max())
+    max_group = int((wl.group_starts[1:] - wl.group_starts[:-1]).max())
+
+    def decode():
+        pa.pa_paged_attention_decode_shared_prefix(
+            outd, q, kc, vc, bt, sl, gs, pl, max_seq_len=max_len, max_group_size=max_group,
+            scale=wl.scale, k_scale=wl.k_scale, v_scale=wl.v_scale)
+
+    def decode_ms(k):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(main)
+        for _ in range(k):
+            decode()
+        e1.record(main)
+        return e0, e1
+
+    for _ in range(3):
+        decode()
+    torch.cuda.synchronize(dev)
+    k_dec = 4 * reps
+    a0, a1 = decode_ms(k_dec)
+    torch.cuda.synchronize(dev)
+    alone = a0.elapsed_time(a1) / k_dec
+    # swaps for as long as the decodes run: start them together
+    start = torch.cuda.Event()
+    start.record(main)
+    side.wait_event(start)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(side)
+    n_swaps = max(1, int(k_dec * alone / max(swap_ms, 1e-3)))
+    for _ in range(n_swaps):
+        swap_pair()
+    s1.record(side)
+    b0, b1 = decode_ms(k_dec)
+    torch.cuda.synchronize(dev)
+    with_swaps = b0.elapsed_time(b1) / k_dec
+    swap_overlap_ms = s0.elapsed_time(s1) / n_swaps
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error bits set by the swap measurement")
+    vals = max_over_ranks([swap_ms, memcpy_ms, alone, with_swaps, swap_overlap_ms], world, dev)
+    swap_ms, memcpy_ms, alone, with_swaps, swap_overlap_ms = vals
+    if rank != 0:
+        return None
+    gbs = lambda ms: round(2 * moved / (ms * 1e-3) / 1e9, 2)
+    return {"workload": f"beam_cow_fp8 pool: {n} blocks x (K + V) of {block_bytes} B, out to "
+                        "page-locked host memory and back",
+            "bytes_per_direction": moved, "unit": "GB/s (host link, both directions)",
+            "swap_blocks_ms": round(swap_ms, 5), "swap_blocks_gbs": gbs(swap_ms),
+            "per_block_memcpy_ms": round(memcpy_ms, 5), "per_block_memcpy_gbs": gbs(memcpy_ms),
+            "per_block_memcpy_calls": 4 * n,
+            "overlap": {"decode_ms_alone": round(alone, 5),
+                        "decode_ms_with_swaps": round(with_swaps, 5),
+                        "decode_slowdown": round(with_swaps / alone, 4),
+                        "swap_blocks_gbs_during_decode": gbs(swap_overlap_ms),
+                        "swaps_on": "a second stream, launched together with the decodes"},
+            "gpu_launches": 2 * (reps + 4) + 2 * n_swaps + 2 * k_dec + 6}
 
 
 def prefill_flops(wl: W.Workload) -> int:
@@ -566,13 +805,19 @@ def prefill_flops(wl: W.Workload) -> int:
     return pairs * cfg.num_heads * cfg.head_dim * 4
 
 
-def run_prefill(args, rank, world, local_rank):
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return float(json.load(fh)["bf16_tflops"]), "measured (bf16_tflops, cuBLAS burst)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def prefill_case(name, dev, args, world, rank, with_e2e=True, with_cpu=False):
     """The multi-query (chunked prefill) step: cache write of the chunks + attention."""
     import paged_kv_cache_413_b200 as pa
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    spec = dict(PREFILL[args.config])
+    spec = dict(PREFILL[name])
     spec["seed"] += 1000 * rank
     wl = W.make_prefill_workload(spec.pop("num_seqs"), spec.pop("context"), spec.pop("chunk"),
                                  **spec)
@@ -598,76 +843,76 @@ def run_prefill(args, rank, world, local_rank):
             e1.record(stream)
             ev.append((e0, e1))
 
-    def step(timed):
-        run_step(inputs, out, timed)
-
-    for _ in range(args.warmup):
-        step(False)
-    torch.cuda.synchronize(dev)
-    sampler = ClockSampler(local_rank) if rank == 0 else None
-    if sampler:
-        sampler.__enter__()
-    if world > 1:
-        torch.distributed.barrier()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step(True)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    if sampler:
-        sampler.__exit__(None, None, None)
-    elapsed_ms, kern_ms = max_over_ranks(
-        [t0.elapsed_time(t1), statistics.mean(a.elapsed_time(b) for a, b in ev)], world, dev)
-    if pa.pa_get_device_error() != 0:
-        raise RuntimeError("device error bits set")
-    host_src = {"q": wl.query, "nk": wl.new_key, "nv": wl.new_value, "sm": wl.slot_mapping,
-                "bt": wl.block_tables, "sl": wl.seq_lens, "qs": wl.query_start}
-    e2e_steps = max(10, args.steps // 4)
-    e2e_ms, h2d, d2h = pipelined_e2e(dev, stream, inputs, host_src, out, run_step, e2e_steps,
-                                     world)
-    e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
-    if rank != 0:
-        return None
-    flops = prefill_flops(wl)
+    elapsed_ms, kern_ms, clocks = timed_loop(lambda timed: run_step(inputs, out, timed), ev,
+                                             args.steps, args.warmup, dev, stream, world, rank)
     cfg = wl.cfg
+    L = wl.seq_lens.numpy().astype(np.int64)
+    res = {"wl": wl, "elapsed_ms": elapsed_ms, "kern_ms": kern_ms, "clocks": clocks,
+           "flops": prefill_flops(wl), "max_q": max_q,
+           "kv_bytes": int(L.sum()) * cfg.num_kv_heads * cfg.head_dim * 2 * 2,
+           "qo_bytes": 2 * q.numel() * 2, "query_tokens": int(wl.query_start[-1])}
+    if with_e2e:
+        host_src = {"q": wl.query, "nk": wl.new_key, "nv": wl.new_value, "sm": wl.slot_mapping,
+                    "bt": wl.block_tables, "sl": wl.seq_lens, "qs": wl.query_start}
+        e2e_steps = max(10, args.steps // 4)
+        e2e_ms, h2d, d2h = pipelined_e2e(dev, stream, inputs, host_src, out, run_step,
+                                         e2e_steps, world)
+        res["e2e"] = (max_over_ranks([e2e_ms], world, dev)[0], e2e_steps, h2d, d2h)
+    if with_cpu and not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = prefill_cpu_baseline(wl)
+    return res
+
+
+def prefill_roofline(name, p):
+    cfg = p["wl"].cfg
+    peak, kind = tensor_peak()
     # the launcher's rule: 128-row tcgen05 tiles once a chunk fills one
     kernel = ("prefill_tc_kernel (tcgen05.mma, TMEM accumulators)"
-              if max_q * (cfg.num_heads // cfg.num_kv_heads) >= 128
+              if p["max_q"] * (cfg.num_heads // cfg.num_kv_heads) >= 128
               else "prefill_kernel (mma.sync m16n8k16)")
-    L = wl.seq_lens.numpy().astype(np.int64)
-    kv_bytes = int(L.sum()) * cfg.num_kv_heads * cfg.head_dim * 2 * 2
-    qo_bytes = 2 * q.numel() * 2
-    peak = 1686.0
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
-            peak = float(json.load(fh)["bf16_tflops"])
-        kind = "measured (bf16_tflops, cuBLAS burst)"
-    except Exception:
-        kind = "fallback"
-    tflops = flops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
-    achieved = flops / (kern_ms * 1e-3) / 1e12
+    achieved = p["flops"] / (p["kern_ms"] * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": kernel, "achieved": round(achieved, 2), "peak": peak,
+            "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "traffic": recorded_traffic(name), "launch_ms": round(p["kern_ms"], 5),
+            "flops_per_launch": p["flops"],
+            "hbm_gbs": round((p["kv_bytes"] + p["qo_bytes"]) / (p["kern_ms"] * 1e-3) / 1e9, 1)}
+
+
+def prefill_entry(name, p, steps, world):
+    roof = prefill_roofline(name, p)
+    return {"workload": f"{name}: {DESCR[name]}", "launch_ms": roof["launch_ms"],
+            "flops_per_launch": p["flops"], "achieved_tflops": roof["achieved"],
+            "frac": roof["frac"], "peak": roof["peak"], "peak_kind": roof["peak_kind"],
+            "traffic": roof["traffic"], "kernel": roof["kernel"],
+            "step_value": round(p["flops"] * world * steps / (p["elapsed_ms"] * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "ms_per_step": round(p["elapsed_ms"] / steps, 5), "steps": steps,
+            "gpu_launches": 2 * steps, "clocks": p["clocks"]}
+
+
+def run_prefill(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    p = prefill_case(args.config, dev, args, world, rank, with_e2e=True, with_cpu=(rank == 0))
+    if rank != 0:
+        return None
+    flops = p["flops"]
+    e2e_ms, e2e_steps, h2d, d2h = p["e2e"]
+    tflops = flops * world * args.steps / (p["elapsed_ms"] * 1e-3) / 1e12
     return {"metric": "paged multi-query attention (chunked prefill): TFLOP/s", "value":
             round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 5),
+            "warmup": args.warmup, "ms_per_step": round(p["elapsed_ms"] / args.steps, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": f"{args.config}: {DESCR[args.config]}",
-                       "query_tokens": int(wl.query_start[-1]), "flops_per_step": flops,
-                       "l2": f"KV read {kv_bytes / 1e6:.0f} MB per step, above the 126 MB L2"},
-            "roofline": {"bound": "tensor", "kernel": kernel,
-                         "achieved": round(achieved, 2), "peak": peak, "peak_kind": kind,
-                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                         "traffic": recorded_prefill_traffic(args.config),
-                         "launch_ms": round(kern_ms, 5),
-                         "hbm_gbs": round((kv_bytes + qo_bytes) / (kern_ms * 1e-3) / 1e9, 1)},
+                       "query_tokens": p["query_tokens"], "flops_per_step": flops,
+                       "l2": f"KV read {p['kv_bytes'] / 1e6:.0f} MB per step, above the 126 MB L2"},
+            "roofline": prefill_roofline(args.config, p),
             "e2e": {"value": round(flops * world * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2),
                     "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 5)},
-            "cpu_baseline": (None if args.no_cpu_baseline or world > 1
-                             else prefill_cpu_baseline(wl)),
+            "cpu_baseline": p.get("cpu_baseline"),
             "gpu_launches": 2 * args.steps,
-            "clocks": sampler.summary() if sampler else None}
+            "clocks": p["clocks"]}
 
 
 def run_reference(args, rank, world):
@@ -715,6 +960,8 @@ def main():
     ap.add_argument("--decode", default="auto", choices=["auto", "shared", "standard"],
                     help="copy-on-write workloads: shared-prefix decode (auto) or per sequence")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="default workload only: skip the `configs` map of the other workloads")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -258,13 +258,20 @@ int pa_copy_blocks(void* const* key_caches, void* const* value_caches, int num_l
  * Same arguments, layouts and results as pa_paged_attention_decode, minus the
  * workspace: the split-partition scratch lives in a fixed array of
  * PA_STATIC_WORKSPACE_BYTES in the library's own device memory, which every GPU
- * that loads the library's device code holds until the process exits.  This
- * function allocates nothing and calls no allocating routine.
+ * that uses it holds until the process exits.  This function allocates nothing
+ * and calls no allocating routine.
  *   - Sizes whose pa_paged_attention_workspace_size() exceeds
  *     PA_STATIC_WORKSPACE_BYTES are rejected with PA_ERR_WORKSPACE.
- *   - The first call on a device that needs scratch looks up the array's device
- *     address (cudaGetSymbolAddress, with that device current) and caches it;
- *     make that first call before any stream capture.
+ *   - Set-up: the first call on a device, whatever its sizes (num_seqs = 0
+ *     included), looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current) and caches it.  Under lazy module loading, the CUDA 12
+ *     default, that lookup is also when the driver reserves the array on the
+ *     device.  So make one call on each device before handing nearly all free
+ *     memory to a KV pool (or run with CUDA_MODULE_LOADING=EAGER), and before any
+ *     stream capture.  If the set-up fails the call returns PA_ERR_CUDA.
+ *   - The cached address belongs to the device's context of that moment: after
+ *     cudaDeviceReset it is stale, and this entry point must not be called on that
+ *     device again in the same process.
  *   - Every call on a device shares the one array and it keeps the last call's
  *     contents (nothing in it needs to start at zero).  Calls whose work overlaps
  *     on the GPU (other streams, other host threads) race on it: serialise them.

@@ -100,6 +100,8 @@ def _load():
             lib.oracle_to_f64.restype = I
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = I
+            lib.oracle_set_num_threads.argtypes = [I]
+            lib.oracle_set_num_threads.restype = I
             _lib = lib
     return _lib
 
@@ -134,6 +136,12 @@ def _ptr(a: np.ndarray) -> int:
 def num_threads() -> int:
     """OpenMP threads the oracle's decode loop uses."""
     return _load().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> int:
+    """Use n OpenMP threads in later calls (the bench's single-thread timing);
+    returns the count now in force."""
+    return _load().oracle_set_num_threads(int(n))
 
 
 def to_f64(a, dtype: str) -> np.ndarray:

@@ -509,6 +509,17 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Set the number of OpenMP threads later calls use (n >= 1); returns the new count. */
+int oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+  return omp_get_max_threads();
+#else
+  (void)n;
+  return 1;
+#endif
+}
+
 /* Convert n values of a format to fp64 (used by tests to read device outputs). */
 int oracle_to_f64(double* dst, const void* src, int64_t n, int dtype) {
   if (!elt_size(dtype)) return -1;

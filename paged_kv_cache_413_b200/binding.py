@@ -47,6 +47,39 @@ def library_path() -> str:
     return _LIB_PATH
 
 
+def declare(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Set the ctypes signatures of every entry point of a loaded libpa build."""
+    P, I, L, F, S = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                     ctypes.c_size_t)
+    lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, L, I, I, F, F, P]
+    lib.pa_reshape_and_cache.restype = I
+    lib.pa_paged_attention_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.pa_paged_attention_workspace_size.restype = S
+    lib.pa_paged_attention_partition_size.argtypes = [I, I, I, I, I]
+    lib.pa_paged_attention_partition_size.restype = I
+    lib.pa_paged_attention_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, I, L, F,
+                                              I, I, I, F, F, I, P, S, P]
+    lib.pa_paged_attention_decode.restype = I
+    lib.pa_paged_attention_decode_static_workspace.argtypes = [
+        P, P, P, P, P, I, P, I, I, I, I, I, I, L, F, I, I, I, F, F, I, P]
+    lib.pa_paged_attention_decode_static_workspace.restype = I
+    lib.pa_paged_attention_decode_shared_prefix.argtypes = [
+        P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, I, I, L, F, I, I, I, F, F, P]
+    lib.pa_paged_attention_decode_shared_prefix.restype = I
+    lib.pa_copy_blocks.argtypes = [P, P, I, P, I, S, L, P]
+    lib.pa_copy_blocks.restype = I
+    lib.pa_paged_attention_prefill.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I,
+                                               I, I, L, F, I, I, I, P]
+    lib.pa_paged_attention_prefill.restype = I
+    lib.pa_swap_blocks.argtypes = [P, P, P, P, I, P, I, S, L, L, P]
+    lib.pa_swap_blocks.restype = I
+    lib.pa_status_string.argtypes = [I]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), P]
+    lib.pa_get_device_error.restype = I
+    return lib
+
+
 def library() -> ctypes.CDLL:
     """Load libpa.so (once); raise if it has not been built."""
     global _lib
@@ -56,36 +89,7 @@ def library() -> ctypes.CDLL:
                 raise RuntimeError(
                     f"libpa.so not found at {_LIB_PATH}: build it with "
                     "`python -m paged_kv_cache_413_b200.build` (there is no fallback path)")
-            lib = ctypes.CDLL(_LIB_PATH)
-            P, I, L, F, S = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
-                             ctypes.c_size_t)
-            lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, L, I, I, F, F, P]
-            lib.pa_reshape_and_cache.restype = I
-            lib.pa_paged_attention_workspace_size.argtypes = [I, I, I, I, I, I]
-            lib.pa_paged_attention_workspace_size.restype = S
-            lib.pa_paged_attention_partition_size.argtypes = [I, I, I, I, I]
-            lib.pa_paged_attention_partition_size.restype = I
-            lib.pa_paged_attention_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, I, L, F,
-                                                      I, I, I, F, F, I, P, S, P]
-            lib.pa_paged_attention_decode.restype = I
-            lib.pa_paged_attention_decode_static_workspace.argtypes = [
-                P, P, P, P, P, I, P, I, I, I, I, I, I, L, F, I, I, I, F, F, I, P]
-            lib.pa_paged_attention_decode_static_workspace.restype = I
-            lib.pa_paged_attention_decode_shared_prefix.argtypes = [
-                P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, I, I, L, F, I, I, I, F, F, P]
-            lib.pa_paged_attention_decode_shared_prefix.restype = I
-            lib.pa_copy_blocks.argtypes = [P, P, I, P, I, S, L, P]
-            lib.pa_paged_attention_prefill.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I,
-                                                       I, I, L, F, I, I, I, P]
-            lib.pa_paged_attention_prefill.restype = I
-            lib.pa_swap_blocks.argtypes = [P, P, P, P, I, P, I, S, L, L, P]
-            lib.pa_swap_blocks.restype = I
-            lib.pa_copy_blocks.restype = I
-            lib.pa_status_string.argtypes = [I]
-            lib.pa_status_string.restype = ctypes.c_char_p
-            lib.pa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), P]
-            lib.pa_get_device_error.restype = I
-            _lib = lib
+            _lib = declare(ctypes.CDLL(_LIB_PATH))
     return _lib
 
 
@@ -100,6 +104,23 @@ def _stream(stream) -> int:
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+def _device_of(*tensors) -> torch.cuda.device:
+    """The device every CUDA tensor of a call lives on, as a context that makes it
+    current for the call (so the library launches there, on that device's current
+    stream).  Tensors on two different devices are rejected."""
+    idx = None
+    for t in tensors:
+        if isinstance(t, torch.Tensor) and t.device.type == "cuda":
+            i = t.device.index if t.device.index is not None else torch.cuda.current_device()
+            if idx is None:
+                idx = i
+            elif i != idx:
+                raise ValueError("all CUDA tensors of a call must be on the same device")
+    if idx is None:
+        raise ValueError("the call has no CUDA tensor")
+    return torch.cuda.device(idx)
 
 
 def _dev(t: torch.Tensor, name: str) -> int:
@@ -126,11 +147,12 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torc
     t = slot_mapping.shape[0]
     if key.shape != (t, hkv, d) or value.shape != key.shape or value_cache.shape != key_cache.shape:
         raise ValueError("shape mismatch between key/value and the caches")
-    _check("pa_reshape_and_cache", library().pa_reshape_and_cache(
-        _dev(key, "key"), _dev(value, "value"), _dev(key_cache, "key_cache"),
-        _dev(value_cache, "value_cache"), _dev(slot_mapping, "slot_mapping"), t, hkv, d, bs, nb,
-        _dt(key, "key"), _dt(key_cache, "key_cache"), float(k_scale), float(v_scale),
-        _stream(stream)))
+    with _device_of(key, value, key_cache, value_cache, slot_mapping):
+        _check("pa_reshape_and_cache", library().pa_reshape_and_cache(
+            _dev(key, "key"), _dev(value, "value"), _dev(key_cache, "key_cache"),
+            _dev(value_cache, "value_cache"), _dev(slot_mapping, "slot_mapping"), t, hkv, d, bs, nb,
+            _dt(key, "key"), _dt(key_cache, "key_cache"), float(k_scale), float(v_scale),
+            _stream(stream)))
 
 
 def pa_paged_attention_workspace_size(num_seqs: int, num_heads: int, num_kv_heads: int,
@@ -164,12 +186,13 @@ def pa_paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache:
     ws_ptr, ws_bytes = 0, 0
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
-    _check("pa_paged_attention_decode", library().pa_paged_attention_decode(
-        _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
-        _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
-        block_tables.shape[1], _dev(seq_lens, "seq_lens"), b, int(max_seq_len), h, hkv, d, bs,
-        nb, float(scale), _dt(query, "query"), _dt(key_cache, "key_cache"), _dt(out, "out"),
-        float(k_scale), float(v_scale), int(partition_size), ws_ptr, ws_bytes, _stream(stream)))
+    with _device_of(out, query, key_cache, value_cache, block_tables, seq_lens, workspace):
+        _check("pa_paged_attention_decode", library().pa_paged_attention_decode(
+            _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
+            _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+            block_tables.shape[1], _dev(seq_lens, "seq_lens"), b, int(max_seq_len), h, hkv, d, bs,
+            nb, float(scale), _dt(query, "query"), _dt(key_cache, "key_cache"), _dt(out, "out"),
+            float(k_scale), float(v_scale), int(partition_size), ws_ptr, ws_bytes, _stream(stream)))
 
 
 def pa_paged_attention_decode_static_workspace(out: torch.Tensor, query: torch.Tensor,
@@ -189,7 +212,8 @@ def pa_paged_attention_decode_static_workspace(out: torch.Tensor, query: torch.T
     if out.shape != query.shape or d2 != d or value_cache.shape != key_cache.shape or \
             block_tables.dim() != 2 or block_tables.shape[0] != b or seq_lens.shape != (b,):
         raise ValueError("shape mismatch")
-    status = library().pa_paged_attention_decode_static_workspace(
+    with _device_of(out, query, key_cache, value_cache, block_tables, seq_lens):
+        status = library().pa_paged_attention_decode_static_workspace(
         _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
         _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
         block_tables.shape[1], _dev(seq_lens, "seq_lens"), b, int(max_seq_len), h, hkv, d, bs,
@@ -222,15 +246,17 @@ def pa_paged_attention_decode_shared_prefix(out: torch.Tensor, query: torch.Tens
             block_tables.dim() != 2 or block_tables.shape[0] != b or seq_lens.shape != (b,) or \
             group_starts.shape != (ng + 1,):
         raise ValueError("shape mismatch")
-    _check("pa_paged_attention_decode_shared_prefix",
-           library().pa_paged_attention_decode_shared_prefix(
-               _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
-               _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
-               block_tables.shape[1], _dev(seq_lens, "seq_lens"), b, int(max_seq_len),
-               _dev(group_starts, "group_starts"), _dev(prefix_lens, "prefix_lens"), ng,
-               int(max_group_size), h, hkv, d, bs, nb, float(scale), _dt(query, "query"),
-               _dt(key_cache, "key_cache"), _dt(out, "out"), float(k_scale), float(v_scale),
-               _stream(stream)))
+    with _device_of(out, query, key_cache, value_cache, block_tables, seq_lens,
+                    group_starts, prefix_lens):
+        _check("pa_paged_attention_decode_shared_prefix",
+               library().pa_paged_attention_decode_shared_prefix(
+                   _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
+                   _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+                   block_tables.shape[1], _dev(seq_lens, "seq_lens"), b, int(max_seq_len),
+                   _dev(group_starts, "group_starts"), _dev(prefix_lens, "prefix_lens"), ng,
+                   int(max_group_size), h, hkv, d, bs, nb, float(scale), _dt(query, "query"),
+                   _dt(key_cache, "key_cache"), _dt(out, "out"), float(k_scale), float(v_scale),
+                   _stream(stream)))
 
 
 def pa_paged_attention_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
@@ -251,12 +277,14 @@ def pa_paged_attention_prefill(out: torch.Tensor, query: torch.Tensor, key_cache
             block_tables.dim() != 2 or block_tables.shape[0] != b or \
             query_start.shape != (b + 1,):
         raise ValueError("shape mismatch")
-    _check("pa_paged_attention_prefill", library().pa_paged_attention_prefill(
-        _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
-        _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
-        block_tables.shape[1], _dev(seq_lens, "seq_lens"), _dev(query_start, "query_start"), b,
-        int(max_query_len), int(max_seq_len), h, hkv, d, bs, nb, float(scale),
-        _dt(query, "query"), _dt(key_cache, "key_cache"), _dt(out, "out"), _stream(stream)))
+    with _device_of(out, query, key_cache, value_cache, block_tables, seq_lens,
+                    query_start):
+        _check("pa_paged_attention_prefill", library().pa_paged_attention_prefill(
+            _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
+            _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+            block_tables.shape[1], _dev(seq_lens, "seq_lens"), _dev(query_start, "query_start"), b,
+            int(max_query_len), int(max_seq_len), h, hkv, d, bs, nb, float(scale),
+            _dt(query, "query"), _dt(key_cache, "key_cache"), _dt(out, "out"), _stream(stream)))
 
 
 def pa_copy_blocks(key_caches: list, value_caches: list, block_mapping: torch.Tensor, *,
@@ -276,10 +304,11 @@ def pa_copy_blocks(key_caches: list, value_caches: list, block_mapping: torch.Te
             raise ValueError("all layers must share one shape and dtype")
     kp = (ctypes.c_void_p * n)(*[_dev(c, "key_caches[i]") for c in key_caches])
     vp = (ctypes.c_void_p * n)(*[_dev(c, "value_caches[i]") for c in value_caches])
-    _check("pa_copy_blocks", library().pa_copy_blocks(
-        ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), n,
-        _dev(block_mapping, "block_mapping"), block_mapping.shape[0], block_bytes, nb,
-        _stream(stream)))
+    with _device_of(*key_caches, *value_caches, block_mapping):
+        _check("pa_copy_blocks", library().pa_copy_blocks(
+            ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), n,
+            _dev(block_mapping, "block_mapping"), block_mapping.shape[0], block_bytes, nb,
+            _stream(stream)))
 
 
 def _dev_or_pinned(t: torch.Tensor, name: str) -> int:
@@ -312,11 +341,13 @@ def pa_swap_blocks(dst_key_caches: list, dst_value_caches: list, src_key_caches:
             raise ValueError("source layers must share one shape and dtype")
     arr = lambda xs, nm: ctypes.cast((ctypes.c_void_p * n)(*[_dev_or_pinned(c, nm) for c in xs]),
                                      ctypes.c_void_p)
-    _check("pa_swap_blocks", library().pa_swap_blocks(
-        arr(dst_key_caches, "dst_key_caches[i]"), arr(dst_value_caches, "dst_value_caches[i]"),
-        arr(src_key_caches, "src_key_caches[i]"), arr(src_value_caches, "src_value_caches[i]"),
-        n, _dev_or_pinned(block_mapping, "block_mapping"), block_mapping.shape[0], block_bytes,
-        s0.shape[0], d0.shape[0], _stream(stream)))
+    with _device_of(*dst_key_caches, *dst_value_caches, *src_key_caches,
+                    *src_value_caches, block_mapping):
+        _check("pa_swap_blocks", library().pa_swap_blocks(
+            arr(dst_key_caches, "dst_key_caches[i]"), arr(dst_value_caches, "dst_value_caches[i]"),
+            arr(src_key_caches, "src_key_caches[i]"), arr(src_value_caches, "src_value_caches[i]"),
+            n, _dev_or_pinned(block_mapping, "block_mapping"), block_mapping.shape[0], block_bytes,
+            s0.shape[0], d0.shape[0], _stream(stream)))
 
 
 def pa_status_string(status: int) -> str:

@@ -34,22 +34,31 @@ def _deps():
         os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+# The failure-detection test build: the same sources with pipeline waits that give
+# up after 2 ms instead of ~1 s, and a decode producer that never announces or
+# copies the 4th 16-token tile of a CTA (tile index 3), so the waits on that stage
+# must time out and report PA_DEVERR_PIPE_TIMEOUT.  Only the tests load it.
+TIMEOUT_TEST_LIB = os.path.join(PKG, "libpa_timeout_test.so")
+TIMEOUT_TEST_FLAGS = ["-DPA_WAIT_LIMIT_NS=2000000ull", "-DPA_TEST_STALL_TILE=3"]
+
+
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    """Compile every CUDA/C++ source and link libpa.so; returns its path."""
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None,
+          lib: str = LIB, build_dir: str = BUILD_DIR) -> str:
+    """Compile every CUDA/C++ source and link `lib` (libpa.so); returns its path."""
+    if not force and up_to_date(lib):
+        return lib
+    os.makedirs(build_dir, exist_ok=True)
     procs = []
     objs = []
     for src in _sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         objs.append(obj)
         cmd = [NVCC, *ARCH, *FLAGS, *(extra_flags or []), "-c", src, "-o", obj]
         if verbose:
@@ -65,12 +74,19 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
             failed.append(src)
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = lib + ".tmp.%d" % os.getpid()
     cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_timeout_test(force: bool = False, verbose: bool = False) -> str:
+    """Build the failure-detection test library (see TIMEOUT_TEST_FLAGS)."""
+    return build(force, verbose, extra_flags=TIMEOUT_TEST_FLAGS, lib=TIMEOUT_TEST_LIB,
+                 build_dir=os.path.join(BUILD_DIR, "timeout_test"))
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build_timeout_test(force="--force" in sys.argv, verbose="-v" in sys.argv))

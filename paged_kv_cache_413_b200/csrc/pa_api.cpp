@@ -319,6 +319,7 @@ int pa_get_device_error(int* host_flag, void* stream) {
   cudaError_t e = pa::read_and_clear_cache_errors(&bits, s);
   if (e == cudaSuccess) e = pa::read_and_clear_decode_errors(&bits, s);
   if (e == cudaSuccess) e = pa::read_and_clear_prefill_errors(&bits, s);
+  if (e == cudaSuccess) e = pa::read_and_clear_shared_errors(&bits, s);
   *host_flag = static_cast<int>(bits);
   return cuda_status(e);
 }

@@ -89,7 +89,7 @@ __device__ __forceinline__ void decode_unit(const Params& p, LptScratch& sc, int
   static_assert(kLptBuckets == 32 * kPer, "one scan slice of buckets per lane");
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x, n = p.num_seqs;
-    const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+    const int cap = p.cap;
     const int max_tiles = max(1, (cap + kBlockSize - 1) / kBlockSize);
     int bk[kPer];  // bucket of sequence lane + 32 k (0 = longest), -1 past the batch
 #pragma unroll
@@ -217,20 +217,6 @@ __device__ __forceinline__ void load_q_lane(const uint8_t* q, int lane, float mu
   }
 }
 
-// Combine region layout: per warp and head the max (log2 units) and the sum, then
-// the unnormalised accumulators with rows padded to D + 4 floats, which keeps the
-// fragment-order writes of the four column groups on distinct banks.
-template <int D>
-constexpr int combine_row() {
-  return D + 4;
-}
-template <int D, int GT>
-constexpr size_t combine_bytes() {
-  return (size_t(kConsumerWarps) * GT * 2 + size_t(kConsumerWarps) * GT * combine_row<D>() +
-          size_t(GT) * (kConsumerWarps + 1)) *
-         sizeof(float);
-}
-
 // Merge the consumer warps' softmax states (cm: max in log2 units, cl: sum,
 // cacc: unnormalised accumulators, all in shared memory) and store the result:
 // the output itself when the sequence has one partition, else this partition's
@@ -328,7 +314,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
     phys_first = table_row[(blk_begin + lane) / p.tiles_per_block];
   // Sequence length, range-checked against the launch bound and the table width.
   int L = p.seq_lens[seq];
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+  const int cap = p.cap;
   if (L < 0 || L > cap) {
     if (tid == 0 && part == 0 && hg == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
     L = L < 0 ? 0 : cap;
@@ -385,10 +371,18 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
             ok = false;
           }
           if (ok) {
-            mbar_arrive_expect_tx(&full[stage], 2 * TILE);
-            const size_t off = size_t(tl) * TILE;
-            bulk_copy_g2s(kbuf + stage * TILE, p.key_cache + off, TILE, &full[stage], policy);
-            bulk_copy_g2s(vbuf + stage * TILE, p.value_cache + off, TILE, &full[stage], policy);
+#ifdef PA_TEST_STALL_TILE
+            // Failure-detection test build only: tile PA_TEST_STALL_TILE of every CTA
+            // is neither announced nor copied, so its stage's phase never completes
+            // and every wait on it must give up and report PA_DEVERR_PIPE_TIMEOUT.
+            if (i != PA_TEST_STALL_TILE)
+#endif
+            {
+              mbar_arrive_expect_tx(&full[stage], 2 * TILE);
+              const size_t off = size_t(tl) * TILE;
+              bulk_copy_g2s(kbuf + stage * TILE, p.key_cache + off, TILE, &full[stage], policy);
+              bulk_copy_g2s(vbuf + stage * TILE, p.value_cache + off, TILE, &full[stage], policy);
+            }
             ++issued;
           }
         }
@@ -588,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, GT == 8 ? PA_MMA8_MIN_CTAS : 4) deco
   if (warp == kConsumerWarps && (blk_begin + lane) / p.tiles_per_block < p.max_blocks_per_seq)
     phys_first = table_row[(blk_begin + lane) / p.tiles_per_block];
   int L = p.seq_lens[seq];
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+  const int cap = p.cap;
   if (L < 0 || L > cap) {
     if (tid == 0 && part == 0 && hg == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
     L = L < 0 ? 0 : cap;
@@ -883,561 +877,6 @@ __global__ void __launch_bounds__(kThreads, GT == 8 ? PA_MMA8_MIN_CTAS : 4) deco
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// ---------------------------------------------------------------------------
-// Shared-prefix decode for copy-on-write groups (beams of one prompt, parallel
-// samples): sequences whose block tables point at the same physical blocks for
-// their first prefix_len tokens.  One CTA serves up to 16 query heads, i.e. the
-// kv head's query heads of up to 16 / G sequences of a group.  It streams each
-// shared prefix block once and applies it to all 16 heads (two n8 MMA tiles),
-// then each sequence's own blocks with the other sequences' heads masked.  The
-// online softmax of a head only ever sees its own sequence's tokens, so the
-// result equals per-sequence decode while the shared blocks cross HBM and the
-// SM once per group instead of once per sequence.
-// ---------------------------------------------------------------------------
-struct SharedParams {
-  CUtensorMap tmk;
-  CUtensorMap tmv;
-  Params p;
-  const int32_t* group_starts;  // [num_groups + 1]
-  const int32_t* prefix_lens;   // [num_groups]
-  int seqs_per_cta;             // SPB: sequences served by one CTA
-  int ctas_per_group;           // ceil(max_group_size / SPB)
-  int cluster;                  // CTAs splitting one unit's block stream (cluster size)
-};
-
-constexpr int kSharedCols = 16;  // query heads per CTA (two n8 tiles)
-constexpr float kSharedRescaleLog2 = 8.f;  // lazy running max: largest weight 2^8
-
-// 2^x by the MUFU approximation (inputs here are <= 8 or -inf; -inf gives 0)
-__device__ __forceinline__ float ex2_approx_ftz(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-#ifndef PA_SHARED_MIN_CHUNK
-#define PA_SHARED_MIN_CHUNK 128      // fewest blocks per CTA when a unit is split
-#endif
-
-template <typename CT, int kStages>
-constexpr size_t shared_smem_bytes() {
-  constexpr size_t tile = size_t(kBlockSize) * 128 * CacheTraits<CT>::bytes;
-  constexpr size_t pipe = 2 * kStages * tile;
-  constexpr size_t combine = combine_bytes<128, kSharedCols>();
-  constexpr size_t body = pipe > combine ? pipe : combine;
-  // + barriers, per-stage block info, Q^T fragments [8][2][32] x uint2, q multiplier
-  // + cluster exchange: per column the CTA's max, sum and accumulator row
-  return 1024 + body + 2 * kStages * sizeof(uint64_t) + kStages * sizeof(int) +
-         8 * 2 * 32 * sizeof(uint2) + 16 +
-         size_t(kSharedCols) * (2 + combine_row<128>()) * sizeof(float);
-}
-
-#ifndef PA_SHARED_MIN_CTAS
-#define PA_SHARED_MIN_CTAS 4  // resident CTAs per SM the register budget must allow
-#endif
-template <typename CT, typename QT, int kStages>
-__global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_prefix_kernel(
-    const __grid_constant__ SharedParams sp) {
-  constexpr int D = 128;
-  constexpr int NT = 2;
-  constexpr bool kFp8 = CacheTraits<CT>::bytes == 1;
-  constexpr int TILE = kBlockSize * D * CacheTraits<CT>::bytes;
-  using MT = typename std::conditional<kFp8, __half, CT>::type;
-  constexpr bool kSplitP = std::is_same<MT, __nv_bfloat16>::value;
-  static_assert(kStages % kConsumerWarps == 0, "each ring stage must belong to one warp");
-  const Params& p = sp.p;
-
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  constexpr size_t tile_region = 2 * kStages * size_t(TILE);
-  constexpr size_t combine_region = combine_bytes<D, kSharedCols>();
-  constexpr size_t body = tile_region > combine_region ? tile_region : combine_region;
-  uint8_t* kbuf = smem;
-  uint8_t* vbuf = smem + kStages * TILE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + body);
-  uint64_t* empty = full + kStages;
-  int* info = reinterpret_cast<int*>(empty + kStages);          // owner << 8 | valid tokens
-  uint2* qs = reinterpret_cast<uint2*>(info + kStages + (kStages & 1));  // [8][NT][32]
-  float* qmult_s = reinterpret_cast<float*>(qs + 8 * NT * 32);
-  float* xm = qmult_s + 4;                   // [16] this CTA's max per column (log2 units)
-  float* xl = xm + kSharedCols;              // [16] its sum
-  float* xo = xl + kSharedCols;              // [16][R] its accumulator rows
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // a cluster of `cluster` CTAs shares one (group part, kv head) unit and splits its
-  // block stream into contiguous chunks
-  const int unit = blockIdx.x / sp.cluster;
-  const int crank = int(cluster_ctarank());
-  const int grp = unit / sp.ctas_per_group;
-  const int sub = unit - grp * sp.ctas_per_group;
-  const int kvh = blockIdx.y;
-  const int G = p.group;
-  const int gs0 = sp.group_starts[grp], gs1 = sp.group_starts[grp + 1];
-  if (sub == 0 && threadIdx.x == 0 && blockIdx.y == 0 &&
-      (gs1 < gs0 || gs1 - gs0 > sp.ctas_per_group * sp.seqs_per_cta))
-    atomicOr(&g_decode_err, PA_DEVERR_PREFIX);  // a group the launch does not cover
-  const int s0 = gs0 + sub * sp.seqs_per_cta;
-  const int nseq = min(sp.seqs_per_cta, gs1 - s0);
-  if (nseq <= 0) return;
-
-  // lengths of the CTA's sequences and the shared prefix (device data: checked)
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
-  int Lmin = cap;
-  int Ls[kSharedCols];
-#pragma unroll
-  for (int j = 0; j < kSharedCols; ++j) {
-    int L = j < nseq ? p.seq_lens[s0 + j] : 0;
-    if (j < nseq && (L < 0 || L > cap)) {
-      if (tid == 0) atomicOr(&g_decode_err, PA_DEVERR_SEQ_LEN);
-      L = L < 0 ? 0 : cap;
-    }
-    Ls[j] = L;
-    if (j < nseq) Lmin = min(Lmin, L);
-  }
-  int P = sp.prefix_lens[grp];
-  if (P < 0 || P % p.block_size != 0 || P > Lmin) {
-    if (tid == 0 && sub == 0 && kvh == 0) atomicOr(&g_decode_err, PA_DEVERR_PREFIX);
-    P = P < 0 ? 0 : (min(P, Lmin) / p.block_size) * p.block_size;
-  }
-  const int pblk = P / kBlockSize;
-  int ntotal = pblk;
-#pragma unroll
-  for (int j = 0; j < kSharedCols; ++j)
-    if (j < nseq) ntotal += (Ls[j] + kBlockSize - 1) / kBlockSize - pblk;
-  // this CTA's chunk [lo, hi) of the stream: prefix blocks, then each member's own
-  const int chunk = (ntotal + sp.cluster - 1) / sp.cluster;
-  const int lo = min(ntotal, crank * chunk), hi = min(ntotal, lo + chunk);
-  const int nblk = hi - lo;
-
-  const int g = lane >> 2, c = lane & 3;
-  const int mi = lane >> 3, r = lane & 7;
-
-  if (tid == 0) {
-    for (int st = 0; st < kStages; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&empty[st], 1);
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();  // barriers initialised: the producer may start streaming
-
-  float acc[8][NT][4];
-  float m[NT][2], l[NT][2];
-
-  if (warp == kConsumerWarps) {
-    // ---------------- producer: prefix blocks, then every sequence's own blocks ------
-    const uint64_t policy = l2_policy_evict_first();
-    int issued = 0;
-    bool ok = true;
-    int gpos = 0;  // stream position of the current segment's first block
-    for (int seg = 0; seg <= nseq && ok; ++seg) {
-      const int owner = seg - 1;  // -1: the shared prefix
-      const int32_t* row = p.block_tables + int64_t(s0 + (owner < 0 ? 0 : owner)) * p.max_blocks_per_seq;
-      const int s_b0 = owner < 0 ? 0 : pblk;
-      const int s_b1 = owner < 0 ? pblk : (Ls[owner] + kBlockSize - 1) / kBlockSize;
-      const int Lown = owner < 0 ? P : Ls[owner];
-      // the part of this segment inside [lo, hi)
-      const int b0 = s_b0 + max(0, lo - gpos), b1 = s_b0 + min(s_b1 - s_b0, hi - gpos);
-      gpos += s_b1 - s_b0;
-      for (int base = b0; base < b1 && ok; base += 32) {
-        int tile = 0;
-        if (base + lane < b1) {
-          const int t = base + lane, e = t / p.tiles_per_block;
-          int32_t phys = row[e];
-          if (owner < 0) {  // the promise: every sequence of the group has these blocks
-            for (int j = 1; j < nseq; ++j)
-              if (p.block_tables[int64_t(s0 + j) * p.max_blocks_per_seq + e] != phys)
-                atomicOr(&g_decode_err, PA_DEVERR_PREFIX);
-          }
-          if (phys < 0 || phys >= p.num_blocks) {
-            atomicOr(&g_decode_err, PA_DEVERR_BLOCK_RANGE);
-            phys = 0;
-          }
-          tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
-        }
-        const int cnt = min(32, b1 - base);
-        for (int jj = 0; jj < cnt; ++jj) {
-          const int tl = __shfl_sync(kFullMask, tile, jj);
-          const int i = issued, stage = i % kStages;
-          if (lane == 0) {
-            if (i >= kStages && !mbar_wait_bounded(&empty[stage], ((i / kStages) - 1) & 1)) {
-              atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
-              ok = false;
-            }
-            if (ok) {
-              const int nvalid = min(kBlockSize, Lown - (base + jj) * kBlockSize);
-              info[stage] = ((owner + 1) << 8) | nvalid;
-              const int trow = tl * kBlockSize;
-              uint8_t* kd = kbuf + stage * TILE;
-              uint8_t* vd = vbuf + stage * TILE;
-              mbar_arrive_expect_tx(&full[stage], 2 * TILE);
-              if constexpr (kFp8) {
-                tma_load_2d(kd, &sp.tmk, 0, trow, &full[stage], policy);
-                tma_load_2d(vd, &sp.tmv, 0, trow, &full[stage], policy);
-              } else {
-                tma_load_2d(kd, &sp.tmk, 0, trow, &full[stage], policy);
-                tma_load_2d(kd + TILE / 2, &sp.tmk, 64, trow, &full[stage], policy);
-                tma_load_2d(vd, &sp.tmv, 0, trow, &full[stage], policy);
-                tma_load_2d(vd + TILE / 2, &sp.tmv, 64, trow, &full[stage], policy);
-              }
-            }
-          }
-          ok = __shfl_sync(kFullMask, ok, 0);
-          if (!ok) break;
-          ++issued;
-        }
-      }
-    }
-    if (lane == 0) {
-      const int first = issued > kStages ? issued - kStages : 0;
-      for (int i = first; i < issued; ++i)
-        if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1))
-          atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
-    }
-    __syncwarp();
-  } else {
-    // ---------------- consumers ----------------
-  // Q^T fragments of the CTA's 16 columns (column n = j * G + head-in-group),
-    // prepared once by warp 0 into shared memory.
-    if (warp == 0) {
-      float mult = p.q_mult;
-      uint32_t frag[8][NT][2];
-      float qmax = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int n = nt * 8 + g, j = n / G, hi = n - j * G;
-        const bool ok = n < nseq * G;
-        const uint8_t* qrow =
-            p.query + (int64_t(s0 + (ok ? j : 0)) * p.num_heads + kvh * G + (ok ? hi : 0)) * D * 2;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          if constexpr (!kFp8) {
-            frag[ks][nt][0] = ok ? *reinterpret_cast<const uint32_t*>(qrow + (16 * ks + 2 * c) * 2) : 0u;
-            frag[ks][nt][1] = ok ? *reinterpret_cast<const uint32_t*>(qrow + (16 * ks + 2 * c + 8) * 2) : 0u;
-          } else {
-            const uint2 w = ok ? *reinterpret_cast<const uint2*>(qrow + (16 * ks + 4 * c) * 2)
-                               : make_uint2(0u, 0u);
-            frag[ks][nt][0] = w.x;
-            frag[ks][nt][1] = w.y;
-            if constexpr (!std::is_same<QT, __half>::value) {
-              const float2 a = unpack2(w.x, QT{}), b = unpack2(w.y, QT{});
-              qmax = fmaxf(qmax, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y))));
-            }
-          }
-        }
-      }
-      if constexpr (kFp8 && !std::is_same<QT, __half>::value) {
-        // bf16 -> f16 with a power-of-two scale (see decode_mma_kernel)
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(kFullMask, qmax, o));
-        int e = 0;
-        if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &e);
-        const int sq = min(max(15 - e, -100), 100);
-        mult = ldexpf(mult, -sq);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const float2 a = unpack2(frag[ks][nt][0], QT{}), b = unpack2(frag[ks][nt][1], QT{});
-            frag[ks][nt][0] = pack2(ldexpf(a.x, sq), ldexpf(a.y, sq), __half{});
-            frag[ks][nt][1] = pack2(ldexpf(b.x, sq), ldexpf(b.y, sq), __half{});
-          }
-      }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          qs[(ks * NT + nt) * 32 + lane] = make_uint2(frag[ks][nt][0], frag[ks][nt][1]);
-      if (lane == 0) *qmult_s = mult;
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");  // consumers only
-    const float mult = *qmult_s;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      m[nt][0] = m[nt][1] = -INFINITY;
-      l[nt][0] = l[nt][1] = 0.f;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) acc[t][nt][0] = acc[t][nt][1] = acc[t][nt][2] = acc[t][nt][3] = 0.f;
-    }
-    for (int i = warp; i < nblk; i += kConsumerWarps) {
-      const int stage = i % kStages;
-      if (!__all_sync(kFullMask, mbar_wait_bounded(&full[stage], (i / kStages) & 1))) {
-        if (lane == 0) atomicOr(&g_decode_err, PA_DEVERR_PIPE_TIMEOUT);
-        break;
-      }
-      const int inf = info[stage];
-      const int owner = (inf >> 8) - 1, nvalid = inf & 0xff;
-      const uint32_t kt = smem_u32(kbuf + stage * TILE);
-      const uint32_t vt = smem_u32(vbuf + stage * TILE);
-
-      float sc[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-      if constexpr (!kFp8) {
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const int tok = r + 8 * (mi & 1), j = 2 * ks + (mi >> 1);
-          uint32_t a[4];
-          ldsm_x4(kt + (j >> 3) * (TILE / 2) + tok * 128 + (((j & 7) ^ r) << 4), a);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const uint2 b = qs[(ks * NT + nt) * 32 + lane];
-            mma_16816(sc[nt], a, b.x, b.y, MT{});
-          }
-        }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int tok = r + 8 * (mi & 1), j = 2 * u + (mi >> 1);
-          uint32_t R[4];
-          ldsm_x4(kt + tok * 128 + ((j ^ r) << 4), R);
-          const uint32_t a0[4] = {e4m3x2_to_f16x2(R[0]), e4m3x2_to_f16x2(R[1]),
-                                  e4m3x2_to_f16x2(R[0] >> 16), e4m3x2_to_f16x2(R[1] >> 16)};
-          const uint32_t a1[4] = {e4m3x2_to_f16x2(R[2]), e4m3x2_to_f16x2(R[3]),
-                                  e4m3x2_to_f16x2(R[2] >> 16), e4m3x2_to_f16x2(R[3] >> 16)};
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const uint2 b0 = qs[((2 * u) * NT + nt) * 32 + lane];
-            const uint2 b1 = qs[((2 * u + 1) * NT + nt) * 32 + lane];
-            mma_16816(sc[nt], a0, b0.x, b0.y, MT{});
-            mma_16816(sc[nt], a1, b1.x, b1.y, MT{});
-          }
-        }
-      }
-      const bool v0 = g < nvalid, v8 = g + 8 < nvalid;
-      uint32_t bh0[NT], bh1[NT], bl0[NT], bl1[NT];
-      float al[NT][2];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        // columns of this thread and whether the block belongs to them
-        const int n0 = nt * 8 + 2 * c, n1 = n0 + 1;
-        const bool a0 = owner < 0 || n0 / G == owner;
-        const bool a1 = owner < 0 || n1 / G == owner;
-        sc[nt][0] = (v0 && a0) ? sc[nt][0] * mult : -INFINITY;
-        sc[nt][1] = (v0 && a1) ? sc[nt][1] * mult : -INFINITY;
-        sc[nt][2] = (v8 && a0) ? sc[nt][2] * mult : -INFINITY;
-        sc[nt][3] = (v8 && a1) ? sc[nt][3] * mult : -INFINITY;
-        float mx0 = fmaxf(sc[nt][0], sc[nt][2]), mx1 = fmaxf(sc[nt][1], sc[nt][3]);
-#pragma unroll
-        for (int o = 4; o <= 16; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
-        }
-        // lazy running max: it moves only when a tile's max passes it by more than
-        // 2^8, so weights stay <= 256 and most tiles skip the accumulator rescale;
-        // O and l are always relative to the same max, so the result is unchanged
-        const float mn0 = mx0 > m[nt][0] + kSharedRescaleLog2 ? mx0 : m[nt][0];
-        const float mn1 = mx1 > m[nt][1] + kSharedRescaleLog2 ? mx1 : m[nt][1];
-        // a column that has seen no token yet keeps m = -inf: scale 1, weights 0
-        al[nt][0] = mn0 == -INFINITY ? 1.f : ex2_approx_ftz(m[nt][0] - mn0);
-        al[nt][1] = mn1 == -INFINITY ? 1.f : ex2_approx_ftz(m[nt][1] - mn1);
-        m[nt][0] = mn0;
-        m[nt][1] = mn1;
-        const float p0 = mn0 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][0] - mn0);
-        const float p1 = mn1 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][1] - mn1);
-        const float p2 = mn0 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][2] - mn0);
-        const float p3 = mn1 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][3] - mn1);
-        l[nt][0] = l[nt][0] * al[nt][0] + (p0 + p2);
-        l[nt][1] = l[nt][1] * al[nt][1] + (p1 + p3);
-        const uint32_t x0 = pack2(p0, p1, MT{}), x1 = pack2(p2, p3, MT{});
-        bh0[nt] = movmatrix_trans(x0);
-        bh1[nt] = movmatrix_trans(x1);
-        bl0[nt] = bl1[nt] = 0;
-        if constexpr (kSplitP) {
-          const float2 h0 = unpack2(x0, MT{}), h1 = unpack2(x1, MT{});
-          bl0[nt] = movmatrix_trans(pack2(p0 - h0.x, p1 - h0.y, MT{}));
-          bl1[nt] = movmatrix_trans(pack2(p2 - h1.x, p3 - h1.y, MT{}));
-        }
-      }
-      if (__any_sync(kFullMask, al[0][0] != 1.f || al[0][1] != 1.f || al[1][0] != 1.f ||
-                                    al[1][1] != 1.f))
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            acc[t][nt][0] *= al[nt][0];
-            acc[t][nt][1] *= al[nt][1];
-            acc[t][nt][2] *= al[nt][0];
-            acc[t][nt][3] *= al[nt][1];
-          }
-      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-      if (nvalid < kBlockSize) {
-        mlo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
-        mhi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
-      }
-      if constexpr (!kFp8) {
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int tok = r + 8 * (mi >> 1), j = 2 * t + (mi & 1);
-          uint32_t a[4];
-          ldsm_x4_trans(vt + (j >> 3) * (TILE / 2) + tok * 128 + (((j & 7) ^ r) << 4), a);
-          a[0] &= mlo;
-          a[1] &= mlo;
-          a[2] &= mhi;
-          a[3] &= mhi;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_16816(acc[t][nt], a, bh0[nt], bh1[nt], MT{});
-            if constexpr (kSplitP) mma_16816(acc[t][nt], a, bl0[nt], bl1[nt], MT{});
-          }
-        }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int tok = r + 8 * (mi & 1), j = 2 * u + (mi >> 1);
-          uint32_t R[4];
-          ldsm_x4_trans(vt + tok * 128 + ((j ^ r) << 4), R);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t lo = R[2 * h], hi8 = R[2 * h + 1];
-            uint32_t a[4] = {e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x20)) & mlo,
-                             e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x31)) & mlo,
-                             e4m3x2_to_f16x2(__byte_perm(hi8, 0, 0x20)) & mhi,
-                             e4m3x2_to_f16x2(__byte_perm(hi8, 0, 0x31)) & mhi};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_16816(acc[2 * u + h][nt], a, bh0[nt], bh1[nt], MT{});
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int o = 4; o <= 16; o <<= 1) {
-        l[nt][0] += __shfl_xor_sync(kFullMask, l[nt][0], o);
-        l[nt][1] += __shfl_xor_sync(kFullMask, l[nt][1], o);
-      }
-  }
-
-  __syncthreads();  // pipeline finished: the tile region becomes the combine region
-  constexpr int GC = kSharedCols;
-  constexpr int R = combine_row<D>();
-  float* cm = reinterpret_cast<float*>(smem);
-  float* cl = cm + kConsumerWarps * GC;
-  float* cacc = cl + kConsumerWarps * GC;
-  float* cf = cacc + kConsumerWarps * GC * R;
-  if (warp < kConsumerWarps) {
-    if (g == 0) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        cm[warp * GC + nt * 8 + 2 * c] = m[nt][0];
-        cl[warp * GC + nt * 8 + 2 * c] = l[nt][0];
-        cm[warp * GC + nt * 8 + 2 * c + 1] = m[nt][1];
-        cl[warp * GC + nt * 8 + 2 * c + 1] = l[nt][1];
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int d0 = kFp8 ? 16 * t + 2 * g : 16 * t + g;
-      const int d1 = kFp8 ? d0 + 1 : d0 + 8;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int n0 = nt * 8 + 2 * c;
-        cacc[(warp * GC + n0) * R + d0] = acc[t][nt][0];
-        cacc[(warp * GC + n0) * R + d1] = acc[t][nt][2];
-        cacc[(warp * GC + n0 + 1) * R + d0] = acc[t][nt][1];
-        cacc[(warp * GC + n0 + 1) * R + d1] = acc[t][nt][3];
-      }
-    }
-  }
-  __syncthreads();
-  if (sp.cluster == 1) {  // the whole unit in this CTA: finish the columns directly
-    if (tid < GC) {
-      const int n = tid;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * GC + n]);
-      float f[kConsumerWarps];
-      float Lsum = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float mw = cm[w * GC + n];
-        f[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
-        Lsum += cl[w * GC + n] * f[w];
-      }
-      const float inv = Lsum > 0.f ? p.v_mult / Lsum : 0.f;  // an empty context gives zeros
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) cf[n * (kConsumerWarps + 1) + w] = f[w] * inv;
-    }
-    __syncthreads();
-    for (int e = tid; e < nseq * G * D; e += kThreads) {
-      const int n = e / D, d = e - n * D;
-      float o = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w)
-        o = fmaf(cacc[(w * GC + n) * R + d], cf[n * (kConsumerWarps + 1) + w], o);
-      const int jseq = n / G, hi = n - jseq * G;
-      store_out(p.out, (int64_t(s0 + jseq) * p.num_heads + kvh * G + hi) * D + d, o,
-                p.out_dtype);
-    }
-    return;
-  }
-  // This CTA's state per column: max over its warps, sum and accumulator scaled to it.
-  if (tid < GC) {
-    const int n = tid;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * GC + n]);
-    float Lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const float mw = cm[w * GC + n];
-      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);  // a warp that saw no block
-      cf[n * (kConsumerWarps + 1) + w] = f;
-      Lsum += cl[w * GC + n] * f;
-    }
-    xm[n] = M;
-    xl[n] = Lsum;
-  }
-  __syncthreads();
-  for (int e = tid; e < GC * D; e += kThreads) {
-    const int n = e / D, d = e - n * D;
-    float o = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w)
-      o = fmaf(cacc[(w * GC + n) * R + d], cf[n * (kConsumerWarps + 1) + w], o);
-    xo[n * R + d] = o;
-  }
-  // Merge across the cluster: CTA `crank` finishes the columns n = crank mod cluster,
-  // one output element per thread, reading every CTA's state for it through
-  // distributed shared memory (independent reads, issued together).
-  cluster_sync();
-  const int ncols = nseq * G;
-  const int mycols = (ncols - crank + sp.cluster - 1) / sp.cluster;
-  for (int e = tid; e < mycols * D; e += kThreads) {
-    const int k = e / D, d = e - k * D;
-    const int n = crank + k * sp.cluster;
-    float mq[8], lq[8], oq[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (q < sp.cluster) {
-        mq[q] = ld_dsmem_f32(xm + n, q);
-        lq[q] = ld_dsmem_f32(xl + n, q);
-        oq[q] = ld_dsmem_f32(xo + n * R + d, q);
-      }
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q < sp.cluster) M = fmaxf(M, mq[q]);
-    float Lsum = 0.f, o = 0.f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (q < sp.cluster && mq[q] != -INFINITY) {
-        const float f = exp2f(mq[q] - M);
-        Lsum = fmaf(lq[q], f, Lsum);
-        o = fmaf(oq[q], f, o);
-      }
-    }
-    const float inv = Lsum > 0.f ? p.v_mult / Lsum : 0.f;  // an empty context gives zeros
-    const int jseq = n / G, hi = n - jseq * G;
-    store_out(p.out, (int64_t(s0 + jseq) * p.num_heads + kvh * G + hi) * D + d, o * inv,
-              p.out_dtype);
-  }
-  cluster_sync();  // keep every CTA's shared memory alive until all reads are done
-}
-
 // Log-sum-exp merge of the partitions of sequences with more than one:
 // M = max m_p, w_p = l_p exp(m_p - M), out = sum w_p o_p / sum w_p.
 // One CTA of kReduceWarps warps per (sequence, head) row.  Warp w takes the
@@ -1523,18 +962,8 @@ template <int D, int GT, typename CT, typename QT>
 int launch_typed(const Params& p, int num_seqs, cudaStream_t stream) {
   constexpr size_t smem = smem_bytes<D, GT, CT, kStagesSimt>();
   auto kern = decode_kernel<D, GT, CT, QT, kStagesSimt>;
-  // The shared-memory opt-in is set once per device and instantiation; a race
-  // only repeats an idempotent call.
-  static unsigned long long attr_set_mask = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_set_mask & bit)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-      return PA_ERR_CUDA;
-    attr_set_mask |= bit;
-  }
+  static std::atomic<unsigned long long> smem_set{0};
+  if (set_smem_once(kern, smem, smem_set) != PA_OK) return PA_ERR_CUDA;
   const dim3 grid(unsigned(num_seqs) * unsigned(p.max_parts),
                   unsigned(p.num_kv_heads * p.head_groups));
   kern<<<grid, kThreads, smem, stream>>>(p);
@@ -1566,16 +995,8 @@ int launch_mma_typed(const Params& p, const void* kc, const void* vc, int64_t ro
   constexpr int stages = fp8 ? kStagesMmaFp8 : kStagesMma16;
   constexpr size_t smem = mma_smem_bytes<CT, stages>();
   auto kern = decode_mma_kernel<GT, CT, QT, stages>;
-  static unsigned long long attr_set_mask = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_set_mask & bit)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-      return PA_ERR_CUDA;
-    attr_set_mask |= bit;
-  }
+  static std::atomic<unsigned long long> smem_set{0};
+  if (set_smem_once(kern, smem, smem_set) != PA_OK) return PA_ERR_CUDA;
   TmaParams tp;
   memset(&tp, 0, sizeof tp);
   tp.p = p;
@@ -1594,99 +1015,7 @@ int dispatch_mma(const Params& p, int gt, const void* kc, const void* vc, int64_
   return launch_mma_typed<4, CT, QT>(p, kc, vc, rows, num_seqs, s);
 }
 
-template <typename CT, typename QT>
-int launch_shared_typed(const SharedParams& base, int grid_x, cudaStream_t stream) {
-  constexpr bool fp8 = CacheTraits<CT>::bytes == 1;
-  constexpr int stages = fp8 ? kStagesMmaFp8 : kStagesMma16;
-  constexpr size_t smem = shared_smem_bytes<CT, stages>();
-  auto kern = decode_shared_prefix_kernel<CT, QT, stages>;
-  static unsigned long long attr_set_mask = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_set_mask & bit)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-      return PA_ERR_CUDA;
-    attr_set_mask |= bit;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(grid_x) * unsigned(base.cluster), unsigned(base.p.num_kv_heads));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(base.cluster);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, base);
-  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
 }  // namespace
-
-int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts,
-                                const int32_t* prefix_lens, int num_groups, int max_group_size,
-                                cudaStream_t stream) {
-  const int group = a.num_heads / a.num_kv_heads;
-  const int64_t rows = a.num_blocks * a.num_kv_heads * a.block_size;
-  if (a.head_dim != 128 || group > kSharedCols || rows >= (int64_t(1) << 31) ||
-      encode_fn() == nullptr)
-    return PA_ERR_UNSUPPORTED;
-  SharedParams sp;
-  memset(&sp, 0, sizeof sp);
-  Params& p = sp.p;
-  p.out = a.out;
-  p.query = static_cast<const uint8_t*>(a.query);
-  p.block_tables = a.block_tables;
-  p.seq_lens = a.seq_lens;
-  p.max_blocks_per_seq = a.max_blocks_per_seq;
-  p.block_size = a.block_size;
-  p.tiles_per_block = a.block_size / kBlockSize;
-  p.max_seq_len = a.max_seq_len;
-  p.num_heads = a.num_heads;
-  p.num_kv_heads = a.num_kv_heads;
-  p.group = group;
-  p.head_groups = 1;
-  p.partition = a.max_seq_len > 0 ? a.max_seq_len : 1;
-  p.max_parts = 1;
-  p.out_dtype = a.out_dtype;
-  p.num_blocks = a.num_blocks;
-  p.num_seqs = a.num_seqs;
-  const bool fp8 = a.cache_dtype == PA_FP8_E4M3;
-  p.q_mult = a.scale * kLog2e * (fp8 ? a.k_scale : 1.f);
-  p.v_mult = fp8 ? a.v_scale : 1.f;
-  sp.group_starts = group_starts;
-  sp.prefix_lens = prefix_lens;
-  sp.seqs_per_cta = kSharedCols / group;
-  sp.ctas_per_group = (max_group_size + sp.seqs_per_cta - 1) / sp.seqs_per_cta;
-  const int64_t grid_x = int64_t(num_groups) * sp.ctas_per_group;
-  // Split each unit's block stream over a cluster of up to 8 CTAs when there are
-  // too few units to keep the GPU streaming, keeping chunks of at least
-  // PA_SHARED_MIN_CHUNK blocks.
-  {
-    const int64_t units = grid_x * a.num_kv_heads;
-    int c = int((kAutoTargetCtas + units - 1) / (units > 0 ? units : 1));
-    const int est_blocks = (a.max_seq_len + kBlockSize - 1) / kBlockSize;
-    c = min(c, max(1, est_blocks / PA_SHARED_MIN_CHUNK));
-    sp.cluster = max(1, min(c, 8));
-  }
-  if (grid_x * sp.cluster > INT32_MAX) return PA_ERR_UNSUPPORTED;
-  if (!encode_pool_map(&sp.tmk, a.key_cache, rows, fp8) ||
-      !encode_pool_map(&sp.tmv, a.value_cache, rows, fp8))
-    return PA_ERR_CUDA;
-  if (a.cache_dtype == PA_F16 && a.q_dtype == PA_F16)
-    return launch_shared_typed<__half, __half>(sp, int(grid_x), stream);
-  if (a.cache_dtype == PA_BF16 && a.q_dtype == PA_BF16)
-    return launch_shared_typed<__nv_bfloat16, __nv_bfloat16>(sp, int(grid_x), stream);
-  if (fp8 && a.q_dtype == PA_F16) return launch_shared_typed<fp8_e4m3, __half>(sp, int(grid_x), stream);
-  if (fp8 && a.q_dtype == PA_BF16)
-    return launch_shared_typed<fp8_e4m3, __nv_bfloat16>(sp, int(grid_x), stream);
-  return PA_ERR_UNSUPPORTED;
-}
 
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int group = a.num_heads / a.num_kv_heads;
@@ -1702,6 +1031,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.block_size = a.block_size;
   p.tiles_per_block = a.block_size / kBlockSize;
   p.max_seq_len = a.max_seq_len;
+  p.cap = context_cap(a.max_seq_len, a.max_blocks_per_seq, a.block_size);
   p.num_heads = a.num_heads;
   p.num_kv_heads = a.num_kv_heads;
   p.group = group;
@@ -1749,9 +1079,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   else
     rc = PA_ERR_UNSUPPORTED;
   if (rc != PA_OK || a.ws.max_parts <= 1) return rc;
-  const int cap = a.max_seq_len < a.max_blocks_per_seq * a.block_size
-                      ? a.max_seq_len
-                      : a.max_blocks_per_seq * a.block_size;
+  const int cap = p.cap;
   const int out_rows = a.num_seqs * a.num_heads;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(out_rows));

@@ -1,0 +1,1175 @@
+// pa_decode_shared.cu -- shared-prefix paged decode for copy-on-write groups.
+//
+// Sequences forked from one prompt (beams, parallel samples) share the physical
+// blocks of their prefix ("vLLM推理引擎PagedAttention原理与性能优化实战" sec 3.2:
+// sharers' block tables point at the same blocks, reference-counted).  Attention
+// over such a group reads each shared block once for all of its members; the result
+// is the per-sequence decode's ("vLLM 推理优化技术深度调研报告" sec 3 formulas 3, 4).
+
+#include "pa_kernels.cuh"
+#include "pa_tcgen05.cuh"
+
+namespace pa {
+namespace {
+
+__device__ unsigned int g_shared_err;
+
+// Ring depths of the mma.sync kernel: 8 KB per stage for 16-bit caches, 4 KB for
+// E4M3; a multiple of the consumer-warp count, so each stage has one owning warp.
+constexpr int kSharedStages16 = 4;
+constexpr int kSharedStagesFp8 = 8;
+
+// ---------------------------------------------------------------------------
+// Shared-prefix decode for copy-on-write groups (beams of one prompt, parallel
+// samples): sequences whose block tables point at the same physical blocks for
+// their first prefix_len tokens.  One CTA serves up to 16 query heads, i.e. the
+// kv head's query heads of up to 16 / G sequences of a group.  It streams each
+// shared prefix block once and applies it to all 16 heads (two n8 MMA tiles),
+// then each sequence's own blocks with the other sequences' heads masked.  The
+// online softmax of a head only ever sees its own sequence's tokens, so the
+// result equals per-sequence decode while the shared blocks cross HBM and the
+// SM once per group instead of once per sequence.
+// ---------------------------------------------------------------------------
+struct SharedParams {
+  CUtensorMap tmk;
+  CUtensorMap tmv;
+  Params p;
+  const int32_t* group_starts;  // [num_groups + 1]
+  const int32_t* prefix_lens;   // [num_groups]
+  int seqs_per_cta;             // SPB: sequences served by one CTA
+  int ctas_per_group;           // ceil(max_group_size / SPB)
+  int cluster;                  // CTAs splitting one unit's block stream (cluster size)
+};
+
+constexpr int kSharedCols = 16;  // query heads per CTA (two n8 tiles)
+constexpr float kSharedRescaleLog2 = 8.f;  // lazy running max: largest weight 2^8
+
+// 2^x by the MUFU approximation (inputs here are <= 8 or -inf; -inf gives 0)
+__device__ __forceinline__ float ex2_approx_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+#ifndef PA_SHARED_MIN_CHUNK
+#define PA_SHARED_MIN_CHUNK 128      // fewest blocks per CTA when a unit is split
+#endif
+
+template <typename CT, int kStages>
+constexpr size_t shared_smem_bytes() {
+  constexpr size_t tile = size_t(kBlockSize) * 128 * CacheTraits<CT>::bytes;
+  constexpr size_t pipe = 2 * kStages * tile;
+  constexpr size_t combine = combine_bytes<128, kSharedCols>();
+  constexpr size_t body = pipe > combine ? pipe : combine;
+  // + barriers, per-stage block info, Q^T fragments [8][2][32] x uint2, q multiplier
+  // + cluster exchange: per column the CTA's max, sum and accumulator row
+  return 1024 + body + 2 * kStages * sizeof(uint64_t) + kStages * sizeof(int) +
+         8 * 2 * 32 * sizeof(uint2) + 16 +
+         size_t(kSharedCols) * (2 + combine_row<128>()) * sizeof(float);
+}
+
+#ifndef PA_SHARED_MIN_CTAS
+#define PA_SHARED_MIN_CTAS 4  // resident CTAs per SM the register budget must allow
+#endif
+template <typename CT, typename QT, int kStages>
+__global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_prefix_kernel(
+    const __grid_constant__ SharedParams sp) {
+  constexpr int D = 128;
+  constexpr int NT = 2;
+  constexpr bool kFp8 = CacheTraits<CT>::bytes == 1;
+  constexpr int TILE = kBlockSize * D * CacheTraits<CT>::bytes;
+  using MT = typename std::conditional<kFp8, __half, CT>::type;
+  constexpr bool kSplitP = std::is_same<MT, __nv_bfloat16>::value;
+  static_assert(kStages % kConsumerWarps == 0, "each ring stage must belong to one warp");
+  const Params& p = sp.p;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  constexpr size_t tile_region = 2 * kStages * size_t(TILE);
+  constexpr size_t combine_region = combine_bytes<D, kSharedCols>();
+  constexpr size_t body = tile_region > combine_region ? tile_region : combine_region;
+  uint8_t* kbuf = smem;
+  uint8_t* vbuf = smem + kStages * TILE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + body);
+  uint64_t* empty = full + kStages;
+  int* info = reinterpret_cast<int*>(empty + kStages);          // owner << 8 | valid tokens
+  uint2* qs = reinterpret_cast<uint2*>(info + kStages + (kStages & 1));  // [8][NT][32]
+  float* qmult_s = reinterpret_cast<float*>(qs + 8 * NT * 32);
+  float* xm = qmult_s + 4;                   // [16] this CTA's max per column (log2 units)
+  float* xl = xm + kSharedCols;              // [16] its sum
+  float* xo = xl + kSharedCols;              // [16][R] its accumulator rows
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // a cluster of `cluster` CTAs shares one (group part, kv head) unit and splits its
+  // block stream into contiguous chunks
+  const int unit = blockIdx.x / sp.cluster;
+  const int crank = int(cluster_ctarank());
+  const int grp = unit / sp.ctas_per_group;
+  const int sub = unit - grp * sp.ctas_per_group;
+  const int kvh = blockIdx.y;
+  const int G = p.group;
+  int gs0 = sp.group_starts[grp], gs1 = sp.group_starts[grp + 1];
+  if (gs0 < 0 || gs1 > p.num_seqs || gs1 < gs0) {  // outside the batch: skip the group
+    if (sub == 0 && threadIdx.x == 0 && blockIdx.y == 0) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+    gs0 = gs1 = 0;
+  }
+  if (sub == 0 && threadIdx.x == 0 && blockIdx.y == 0 &&
+      gs1 - gs0 > sp.ctas_per_group * sp.seqs_per_cta)
+    atomicOr(&g_shared_err, PA_DEVERR_PREFIX);  // a group the launch does not cover
+  const int s0 = gs0 + sub * sp.seqs_per_cta;
+  const int nseq = min(sp.seqs_per_cta, gs1 - s0);
+  if (nseq <= 0) return;
+
+  // lengths of the CTA's sequences and the shared prefix (device data: checked)
+  const int cap = p.cap;
+  int Lmin = cap;
+  int Ls[kSharedCols];
+#pragma unroll
+  for (int j = 0; j < kSharedCols; ++j) {
+    int L = j < nseq ? p.seq_lens[s0 + j] : 0;
+    if (j < nseq && (L < 0 || L > cap)) {
+      if (tid == 0) atomicOr(&g_shared_err, PA_DEVERR_SEQ_LEN);
+      L = L < 0 ? 0 : cap;
+    }
+    Ls[j] = L;
+    if (j < nseq) Lmin = min(Lmin, L);
+  }
+  int P = sp.prefix_lens[grp];
+  if (P < 0 || P % p.block_size != 0 || P > Lmin) {
+    if (tid == 0 && sub == 0 && kvh == 0) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+    P = P < 0 ? 0 : (min(P, Lmin) / p.block_size) * p.block_size;
+  }
+  const int pblk = P / kBlockSize;
+  int ntotal = pblk;
+#pragma unroll
+  for (int j = 0; j < kSharedCols; ++j)
+    if (j < nseq) ntotal += (Ls[j] + kBlockSize - 1) / kBlockSize - pblk;
+  // this CTA's chunk [lo, hi) of the stream: prefix blocks, then each member's own
+  const int chunk = (ntotal + sp.cluster - 1) / sp.cluster;
+  const int lo = min(ntotal, crank * chunk), hi = min(ntotal, lo + chunk);
+  const int nblk = hi - lo;
+
+  const int g = lane >> 2, c = lane & 3;
+  const int mi = lane >> 3, r = lane & 7;
+
+  if (tid == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();  // barriers initialised: the producer may start streaming
+
+  float acc[8][NT][4];
+  float m[NT][2], l[NT][2];
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: prefix blocks, then every sequence's own blocks ------
+    const uint64_t policy = l2_policy_evict_first();
+    int issued = 0;
+    bool ok = true;
+    int gpos = 0;  // stream position of the current segment's first block
+    for (int seg = 0; seg <= nseq && ok; ++seg) {
+      const int owner = seg - 1;  // -1: the shared prefix
+      const int32_t* row = p.block_tables + int64_t(s0 + (owner < 0 ? 0 : owner)) * p.max_blocks_per_seq;
+      const int s_b0 = owner < 0 ? 0 : pblk;
+      const int s_b1 = owner < 0 ? pblk : (Ls[owner] + kBlockSize - 1) / kBlockSize;
+      const int Lown = owner < 0 ? P : Ls[owner];
+      // the part of this segment inside [lo, hi)
+      const int b0 = s_b0 + max(0, lo - gpos), b1 = s_b0 + min(s_b1 - s_b0, hi - gpos);
+      gpos += s_b1 - s_b0;
+      for (int base = b0; base < b1 && ok; base += 32) {
+        int tile = 0;
+        if (base + lane < b1) {
+          const int t = base + lane, e = t / p.tiles_per_block;
+          int32_t phys = row[e];
+          if (owner < 0) {  // the promise: every sequence of the group has these blocks
+            for (int j = 1; j < nseq; ++j)
+              if (p.block_tables[int64_t(s0 + j) * p.max_blocks_per_seq + e] != phys)
+                atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+          }
+          if (phys < 0 || phys >= p.num_blocks) {
+            atomicOr(&g_shared_err, PA_DEVERR_BLOCK_RANGE);
+            phys = 0;
+          }
+          tile = (phys * p.num_kv_heads + kvh) * p.tiles_per_block + (t - e * p.tiles_per_block);
+        }
+        const int cnt = min(32, b1 - base);
+        for (int jj = 0; jj < cnt; ++jj) {
+          const int tl = __shfl_sync(kFullMask, tile, jj);
+          const int i = issued, stage = i % kStages;
+          if (lane == 0) {
+            if (i >= kStages && !mbar_wait_bounded(&empty[stage], ((i / kStages) - 1) & 1)) {
+              atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+              ok = false;
+            }
+            if (ok) {
+              const int nvalid = min(kBlockSize, Lown - (base + jj) * kBlockSize);
+              info[stage] = ((owner + 1) << 8) | nvalid;
+              const int trow = tl * kBlockSize;
+              uint8_t* kd = kbuf + stage * TILE;
+              uint8_t* vd = vbuf + stage * TILE;
+              mbar_arrive_expect_tx(&full[stage], 2 * TILE);
+              if constexpr (kFp8) {
+                tma_load_2d(kd, &sp.tmk, 0, trow, &full[stage], policy);
+                tma_load_2d(vd, &sp.tmv, 0, trow, &full[stage], policy);
+              } else {
+                tma_load_2d(kd, &sp.tmk, 0, trow, &full[stage], policy);
+                tma_load_2d(kd + TILE / 2, &sp.tmk, 64, trow, &full[stage], policy);
+                tma_load_2d(vd, &sp.tmv, 0, trow, &full[stage], policy);
+                tma_load_2d(vd + TILE / 2, &sp.tmv, 64, trow, &full[stage], policy);
+              }
+            }
+          }
+          ok = __shfl_sync(kFullMask, ok, 0);
+          if (!ok) break;
+          ++issued;
+        }
+      }
+    }
+    if (lane == 0) {
+      const int first = issued > kStages ? issued - kStages : 0;
+      for (int i = first; i < issued; ++i)
+        if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1))
+          atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- consumers ----------------
+  // Q^T fragments of the CTA's 16 columns (column n = j * G + head-in-group),
+    // prepared once by warp 0 into shared memory.
+    if (warp == 0) {
+      float mult = p.q_mult;
+      uint32_t frag[8][NT][2];
+      float qmax = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n = nt * 8 + g, j = n / G, hi = n - j * G;
+        const bool ok = n < nseq * G;
+        const uint8_t* qrow =
+            p.query + (int64_t(s0 + (ok ? j : 0)) * p.num_heads + kvh * G + (ok ? hi : 0)) * D * 2;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          if constexpr (!kFp8) {
+            frag[ks][nt][0] = ok ? *reinterpret_cast<const uint32_t*>(qrow + (16 * ks + 2 * c) * 2) : 0u;
+            frag[ks][nt][1] = ok ? *reinterpret_cast<const uint32_t*>(qrow + (16 * ks + 2 * c + 8) * 2) : 0u;
+          } else {
+            const uint2 w = ok ? *reinterpret_cast<const uint2*>(qrow + (16 * ks + 4 * c) * 2)
+                               : make_uint2(0u, 0u);
+            frag[ks][nt][0] = w.x;
+            frag[ks][nt][1] = w.y;
+            if constexpr (!std::is_same<QT, __half>::value) {
+              const float2 a = unpack2(w.x, QT{}), b = unpack2(w.y, QT{});
+              qmax = fmaxf(qmax, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y))));
+            }
+          }
+        }
+      }
+      if constexpr (kFp8 && !std::is_same<QT, __half>::value) {
+        // bf16 -> f16 with a power-of-two scale (see decode_mma_kernel)
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(kFullMask, qmax, o));
+        int e = 0;
+        if (qmax > 0.f && isfinite(qmax)) frexpf(qmax, &e);
+        const int sq = min(max(15 - e, -100), 100);
+        mult = ldexpf(mult, -sq);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const float2 a = unpack2(frag[ks][nt][0], QT{}), b = unpack2(frag[ks][nt][1], QT{});
+            frag[ks][nt][0] = pack2(ldexpf(a.x, sq), ldexpf(a.y, sq), __half{});
+            frag[ks][nt][1] = pack2(ldexpf(b.x, sq), ldexpf(b.y, sq), __half{});
+          }
+      }
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          qs[(ks * NT + nt) * 32 + lane] = make_uint2(frag[ks][nt][0], frag[ks][nt][1]);
+      if (lane == 0) *qmult_s = mult;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");  // consumers only
+    const float mult = *qmult_s;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) acc[t][nt][0] = acc[t][nt][1] = acc[t][nt][2] = acc[t][nt][3] = 0.f;
+    }
+    for (int i = warp; i < nblk; i += kConsumerWarps) {
+      const int stage = i % kStages;
+      if (!__all_sync(kFullMask, mbar_wait_bounded(&full[stage], (i / kStages) & 1))) {
+        if (lane == 0) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+        break;
+      }
+      const int inf = info[stage];
+      const int owner = (inf >> 8) - 1, nvalid = inf & 0xff;
+      const uint32_t kt = smem_u32(kbuf + stage * TILE);
+      const uint32_t vt = smem_u32(vbuf + stage * TILE);
+
+      float sc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      if constexpr (!kFp8) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const int tok = r + 8 * (mi & 1), j = 2 * ks + (mi >> 1);
+          uint32_t a[4];
+          ldsm_x4(kt + (j >> 3) * (TILE / 2) + tok * 128 + (((j & 7) ^ r) << 4), a);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint2 b = qs[(ks * NT + nt) * 32 + lane];
+            mma_16816(sc[nt], a, b.x, b.y, MT{});
+          }
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tok = r + 8 * (mi & 1), j = 2 * u + (mi >> 1);
+          uint32_t R[4];
+          ldsm_x4(kt + tok * 128 + ((j ^ r) << 4), R);
+          const uint32_t a0[4] = {e4m3x2_to_f16x2(R[0]), e4m3x2_to_f16x2(R[1]),
+                                  e4m3x2_to_f16x2(R[0] >> 16), e4m3x2_to_f16x2(R[1] >> 16)};
+          const uint32_t a1[4] = {e4m3x2_to_f16x2(R[2]), e4m3x2_to_f16x2(R[3]),
+                                  e4m3x2_to_f16x2(R[2] >> 16), e4m3x2_to_f16x2(R[3] >> 16)};
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint2 b0 = qs[((2 * u) * NT + nt) * 32 + lane];
+            const uint2 b1 = qs[((2 * u + 1) * NT + nt) * 32 + lane];
+            mma_16816(sc[nt], a0, b0.x, b0.y, MT{});
+            mma_16816(sc[nt], a1, b1.x, b1.y, MT{});
+          }
+        }
+      }
+      const bool v0 = g < nvalid, v8 = g + 8 < nvalid;
+      uint32_t bh0[NT], bh1[NT], bl0[NT], bl1[NT];
+      float al[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        // columns of this thread and whether the block belongs to them
+        const int n0 = nt * 8 + 2 * c, n1 = n0 + 1;
+        const bool a0 = owner < 0 || n0 / G == owner;
+        const bool a1 = owner < 0 || n1 / G == owner;
+        sc[nt][0] = (v0 && a0) ? sc[nt][0] * mult : -INFINITY;
+        sc[nt][1] = (v0 && a1) ? sc[nt][1] * mult : -INFINITY;
+        sc[nt][2] = (v8 && a0) ? sc[nt][2] * mult : -INFINITY;
+        sc[nt][3] = (v8 && a1) ? sc[nt][3] * mult : -INFINITY;
+        float mx0 = fmaxf(sc[nt][0], sc[nt][2]), mx1 = fmaxf(sc[nt][1], sc[nt][3]);
+#pragma unroll
+        for (int o = 4; o <= 16; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
+        }
+        // lazy running max: it moves only when a tile's max passes it by more than
+        // 2^8, so weights stay <= 256 and most tiles skip the accumulator rescale;
+        // O and l are always relative to the same max, so the result is unchanged
+        const float mn0 = mx0 > m[nt][0] + kSharedRescaleLog2 ? mx0 : m[nt][0];
+        const float mn1 = mx1 > m[nt][1] + kSharedRescaleLog2 ? mx1 : m[nt][1];
+        // a column that has seen no token yet keeps m = -inf: scale 1, weights 0
+        al[nt][0] = mn0 == -INFINITY ? 1.f : ex2_approx_ftz(m[nt][0] - mn0);
+        al[nt][1] = mn1 == -INFINITY ? 1.f : ex2_approx_ftz(m[nt][1] - mn1);
+        m[nt][0] = mn0;
+        m[nt][1] = mn1;
+        const float p0 = mn0 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][0] - mn0);
+        const float p1 = mn1 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][1] - mn1);
+        const float p2 = mn0 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][2] - mn0);
+        const float p3 = mn1 == -INFINITY ? 0.f : ex2_approx_ftz(sc[nt][3] - mn1);
+        l[nt][0] = l[nt][0] * al[nt][0] + (p0 + p2);
+        l[nt][1] = l[nt][1] * al[nt][1] + (p1 + p3);
+        const uint32_t x0 = pack2(p0, p1, MT{}), x1 = pack2(p2, p3, MT{});
+        bh0[nt] = movmatrix_trans(x0);
+        bh1[nt] = movmatrix_trans(x1);
+        bl0[nt] = bl1[nt] = 0;
+        if constexpr (kSplitP) {
+          const float2 h0 = unpack2(x0, MT{}), h1 = unpack2(x1, MT{});
+          bl0[nt] = movmatrix_trans(pack2(p0 - h0.x, p1 - h0.y, MT{}));
+          bl1[nt] = movmatrix_trans(pack2(p2 - h1.x, p3 - h1.y, MT{}));
+        }
+      }
+      if (__any_sync(kFullMask, al[0][0] != 1.f || al[0][1] != 1.f || al[1][0] != 1.f ||
+                                    al[1][1] != 1.f))
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[t][nt][0] *= al[nt][0];
+            acc[t][nt][1] *= al[nt][1];
+            acc[t][nt][2] *= al[nt][0];
+            acc[t][nt][3] *= al[nt][1];
+          }
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (nvalid < kBlockSize) {
+        mlo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+        mhi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+      }
+      if constexpr (!kFp8) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int tok = r + 8 * (mi >> 1), j = 2 * t + (mi & 1);
+          uint32_t a[4];
+          ldsm_x4_trans(vt + (j >> 3) * (TILE / 2) + tok * 128 + (((j & 7) ^ r) << 4), a);
+          a[0] &= mlo;
+          a[1] &= mlo;
+          a[2] &= mhi;
+          a[3] &= mhi;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_16816(acc[t][nt], a, bh0[nt], bh1[nt], MT{});
+            if constexpr (kSplitP) mma_16816(acc[t][nt], a, bl0[nt], bl1[nt], MT{});
+          }
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tok = r + 8 * (mi & 1), j = 2 * u + (mi >> 1);
+          uint32_t R[4];
+          ldsm_x4_trans(vt + tok * 128 + ((j ^ r) << 4), R);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t lo = R[2 * h], hi8 = R[2 * h + 1];
+            uint32_t a[4] = {e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x20)) & mlo,
+                             e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x31)) & mlo,
+                             e4m3x2_to_f16x2(__byte_perm(hi8, 0, 0x20)) & mhi,
+                             e4m3x2_to_f16x2(__byte_perm(hi8, 0, 0x31)) & mhi};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_16816(acc[2 * u + h][nt], a, bh0[nt], bh1[nt], MT{});
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int o = 4; o <= 16; o <<= 1) {
+        l[nt][0] += __shfl_xor_sync(kFullMask, l[nt][0], o);
+        l[nt][1] += __shfl_xor_sync(kFullMask, l[nt][1], o);
+      }
+  }
+
+  __syncthreads();  // pipeline finished: the tile region becomes the combine region
+  constexpr int GC = kSharedCols;
+  constexpr int R = combine_row<D>();
+  float* cm = reinterpret_cast<float*>(smem);
+  float* cl = cm + kConsumerWarps * GC;
+  float* cacc = cl + kConsumerWarps * GC;
+  float* cf = cacc + kConsumerWarps * GC * R;
+  if (warp < kConsumerWarps) {
+    if (g == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        cm[warp * GC + nt * 8 + 2 * c] = m[nt][0];
+        cl[warp * GC + nt * 8 + 2 * c] = l[nt][0];
+        cm[warp * GC + nt * 8 + 2 * c + 1] = m[nt][1];
+        cl[warp * GC + nt * 8 + 2 * c + 1] = l[nt][1];
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int d0 = kFp8 ? 16 * t + 2 * g : 16 * t + g;
+      const int d1 = kFp8 ? d0 + 1 : d0 + 8;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n0 = nt * 8 + 2 * c;
+        cacc[(warp * GC + n0) * R + d0] = acc[t][nt][0];
+        cacc[(warp * GC + n0) * R + d1] = acc[t][nt][2];
+        cacc[(warp * GC + n0 + 1) * R + d0] = acc[t][nt][1];
+        cacc[(warp * GC + n0 + 1) * R + d1] = acc[t][nt][3];
+      }
+    }
+  }
+  __syncthreads();
+  if (sp.cluster == 1) {  // the whole unit in this CTA: finish the columns directly
+    if (tid < GC) {
+      const int n = tid;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * GC + n]);
+      float f[kConsumerWarps];
+      float Lsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float mw = cm[w * GC + n];
+        f[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+        Lsum += cl[w * GC + n] * f[w];
+      }
+      const float inv = Lsum > 0.f ? p.v_mult / Lsum : 0.f;  // an empty context gives zeros
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) cf[n * (kConsumerWarps + 1) + w] = f[w] * inv;
+    }
+    __syncthreads();
+    for (int e = tid; e < nseq * G * D; e += kThreads) {
+      const int n = e / D, d = e - n * D;
+      float o = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w)
+        o = fmaf(cacc[(w * GC + n) * R + d], cf[n * (kConsumerWarps + 1) + w], o);
+      const int jseq = n / G, hi = n - jseq * G;
+      store_out(p.out, (int64_t(s0 + jseq) * p.num_heads + kvh * G + hi) * D + d, o,
+                p.out_dtype);
+    }
+    return;
+  }
+  // This CTA's state per column: max over its warps, sum and accumulator scaled to it.
+  if (tid < GC) {
+    const int n = tid;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * GC + n]);
+    float Lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float mw = cm[w * GC + n];
+      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);  // a warp that saw no block
+      cf[n * (kConsumerWarps + 1) + w] = f;
+      Lsum += cl[w * GC + n] * f;
+    }
+    xm[n] = M;
+    xl[n] = Lsum;
+  }
+  __syncthreads();
+  for (int e = tid; e < GC * D; e += kThreads) {
+    const int n = e / D, d = e - n * D;
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w)
+      o = fmaf(cacc[(w * GC + n) * R + d], cf[n * (kConsumerWarps + 1) + w], o);
+    xo[n * R + d] = o;
+  }
+  // Merge across the cluster: CTA `crank` finishes the columns n = crank mod cluster,
+  // one output element per thread, reading every CTA's state for it through
+  // distributed shared memory (independent reads, issued together).
+  cluster_sync();
+  const int ncols = nseq * G;
+  const int mycols = (ncols - crank + sp.cluster - 1) / sp.cluster;
+  for (int e = tid; e < mycols * D; e += kThreads) {
+    const int k = e / D, d = e - k * D;
+    const int n = crank + k * sp.cluster;
+    float mq[8], lq[8], oq[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < sp.cluster) {
+        mq[q] = ld_dsmem_f32(xm + n, q);
+        lq[q] = ld_dsmem_f32(xl + n, q);
+        oq[q] = ld_dsmem_f32(xo + n * R + d, q);
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < sp.cluster) M = fmaxf(M, mq[q]);
+    float Lsum = 0.f, o = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < sp.cluster && mq[q] != -INFINITY) {
+        const float f = exp2f(mq[q] - M);
+        Lsum = fmaf(lq[q], f, Lsum);
+        o = fmaf(oq[q], f, o);
+      }
+    }
+    const float inv = Lsum > 0.f ? p.v_mult / Lsum : 0.f;  // an empty context gives zeros
+    const int jseq = n / G, hi = n - jseq * G;
+    store_out(p.out, (int64_t(s0 + jseq) * p.num_heads + kvh * G + hi) * D + d, o * inv,
+              p.out_dtype);
+  }
+  cluster_sync();  // keep every CTA's shared memory alive until all reads are done
+}
+
+
+// ---------------------------------------------------------------------------
+// Shared-prefix decode on the 5th-generation tensor cores, for E4M3 caches.
+//
+// The same work unit as above (one CTA per group part and kv head, up to 16
+// columns = the kv head's query heads of up to 16 / G members), but the stream
+// of 16-token tiles -- the shared prefix first, then each member's own tiles --
+// is cut into stages of 128 tokens with the tokens on the M axis:
+//   S^T[128 tokens x 16 columns]  = K[128 x 128 dims] . Q^T     A = K from TMEM,
+//                                                               B = Q^T from smem
+//   O^T[128 dims x 16 columns]   += V^T[128 dims x 128] . P^T   A = V^T from smem
+//                                                               (MN-major), B = P^T
+// One thread issues the 16 MMAs of a stage.  Four worker warps own one TMEM lane
+// quadrant each: thread t widens token t's K row (E4M3 -> f16, exact) into TMEM
+// and its V row into the f16 operand in shared memory, reads its row of S^T,
+// applies the masks (context length, and for a member's own tiles the other
+// members' columns), and writes its P row.  The softmax needs no reduction across
+// threads per stage: every column keeps one reference maximum shared by all
+// threads, moved (with a rescale of l and of O^T's column in TMEM) only when some
+// score passes it by more than 2^8, which a vote and a named barrier detect; each
+// thread sums its own l and the sums meet once, at the end.  P <= 2^8 is exact
+// enough in f16 (relative 2^-11); softmax and accumulation are fp32.  A producer
+// warp streams the raw E4M3 tiles (tiled TMA, 128-byte swizzle, no multicast)
+// into a ring of kStRing stages.  All waits are bounded; after a failure the
+// waits are skipped but every named barrier is still reached.
+// ---------------------------------------------------------------------------
+constexpr int kStTokens = 128;                          // tokens per stage (M of S^T)
+constexpr int kStTiles = kStTokens / kBlockSize;        // pool tiles per stage
+constexpr int kStWorkers = 4;                           // worker warps, one per lane quadrant
+constexpr int kStProducerWarp = kStWorkers;
+constexpr int kStMmaWarp = kStWorkers + 1;
+constexpr int kStThreads = (kStWorkers + 2) * 32;
+#ifndef PA_SHARED_TC_RING
+#define PA_SHARED_TC_RING 2
+#endif
+constexpr int kStRing = PA_SHARED_TC_RING;              // raw stages in flight
+constexpr int kStRawTile = kBlockSize * 128;            // one E4M3 tile of K or V: 2 KB
+constexpr int kStRawStage = 2 * kStTiles * kStRawTile;  // K tiles, then V tiles: 32 KB
+constexpr int kStVBytes = kStTokens * 128 * 2;          // V of a stage in f16: 32 KB
+constexpr int kStOpBytes = kSharedCols * 128 * 2;       // Q^T or P^T operand: 4 KB
+constexpr int kStOpHalf = kSharedCols * 128;            // one 64-element K half of it
+constexpr uint32_t kStTmemCols = 128;
+constexpr uint32_t kStTmemK = 0;   // K of the stage: 64 columns of f16 pairs (A operand)
+constexpr uint32_t kStTmemS = 64;  // S^T: 16 fp32 columns
+constexpr uint32_t kStTmemO = 80;  // O^T: 16 fp32 columns
+constexpr uint32_t kStIdescS = umma_idesc_f16(0, 0, kStTokens, kSharedCols);
+constexpr uint32_t kStIdescPV = umma_idesc_f16_ab(0, 1, 0, 128, kSharedCols);
+static_assert(kStTmemO + kSharedCols <= kStTmemCols, "TMEM budget");
+
+constexpr size_t shared_tc_smem_bytes() {
+  return 1024 + size_t(kStRing) * kStRawStage + kStVBytes + 2 * kStOpBytes +
+         (2 * kStRing + 5) * sizeof(uint64_t) +
+         (8 + 2 * kStWorkers * kSharedCols + kStWorkers * kSharedCols + kStWorkers) * 4 +
+         (2 * (kSharedCols + 1) + 2) * 4;
+}
+static_assert(2 * (shared_tc_smem_bytes() + 1024) <= 228 * 1024, "two CTAs per SM");
+
+// Four E4M3 bytes (byte 0 = element 0) to four f16: lo = elements 0, 1, hi = 2, 3.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// 16 32-bit words into this warp's 32 TMEM lanes, columns taddr .. taddr + 15.
+__device__ __forceinline__ void tmem_st16_f(uint32_t taddr, const float (&v)[16]) {
+  uint32_t u[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
+  tmem_st16(taddr, u);
+}
+
+template <typename QT>
+__global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
+    const __grid_constant__ SharedParams sp) {
+  constexpr int D = 128;
+  const Params& p = sp.p;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* raw = smem;                                  // [kStRing][K tiles, V tiles]
+  uint8_t* vf = raw + kStRing * kStRawStage;            // V f16: [2 halves][128 rows][128 B]
+  uint8_t* qop = vf + kStVBytes;                        // Q^T: [2 halves][16 rows][128 B]
+  uint8_t* pop = qop + kStOpBytes;                      // P^T: [2 halves][16 rows][128 B]
+  uint64_t* full = reinterpret_cast<uint64_t*>(pop + kStOpBytes);
+  uint64_t* empty = full + kStRing;
+  uint64_t* kready = empty + kStRing;                   // K of stage st in TMEM (4 warps)
+  uint64_t* pready = kready + 1;                        // V and P of stage st in smem (4 warps)
+  uint64_t* sdone = pready + 1;                         // S^T of stage st written
+  uint64_t* odone = sdone + 1;                          // P.V of stage st done
+  uint64_t* done = odone + 1;                           // every MMA done
+  int* flags = reinterpret_cast<int*>(done + 1);        // [2][4] rescale votes
+  float* wmax = reinterpret_cast<float*>(flags + 8);    // [2][4][16] warp column maxima
+  float* lsum = wmax + 2 * kStWorkers * kSharedCols;    // [4][16] warp column sums
+  float* qmax_w = lsum + kStWorkers * kSharedCols;      // [4]
+  int* own_start = reinterpret_cast<int*>(qmax_w + kStWorkers);  // [17] stream position
+  int* own_len = own_start + kSharedCols + 1;           // [16] member lengths
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(own_len + kSharedCols + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int unit = blockIdx.x;
+  const int grp = unit / sp.ctas_per_group;
+  const int sub = unit - grp * sp.ctas_per_group;
+  const int kvh = blockIdx.y;
+  const int G = p.group;
+  int gs0 = sp.group_starts[grp], gs1 = sp.group_starts[grp + 1];
+  if (gs0 < 0 || gs1 > p.num_seqs || gs1 < gs0) {  // outside the batch: skip the group
+    if (sub == 0 && tid == 0 && kvh == 0) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+    gs0 = gs1 = 0;
+  }
+  if (sub == 0 && tid == 0 && kvh == 0 && gs1 - gs0 > sp.ctas_per_group * sp.seqs_per_cta)
+    atomicOr(&g_shared_err, PA_DEVERR_PREFIX);  // a group the launch does not cover
+  const int s0 = gs0 + sub * sp.seqs_per_cta;
+  const int nseq = min(sp.seqs_per_cta, gs1 - s0);
+  if (nseq <= 0) return;  // uniform over the CTA, before any barrier or TMEM
+  const int ncols = nseq * G;
+
+  // lengths and the shared prefix (device data: checked), as the mma.sync kernel
+  const int cap = p.cap;
+  int Lmin = cap, ntotal = 0;
+  if (tid == 0) {
+    for (int j = 0; j < kSharedCols; ++j) {
+      int L = j < nseq ? p.seq_lens[s0 + j] : 0;
+      if (j < nseq && (L < 0 || L > cap)) {
+        atomicOr(&g_shared_err, PA_DEVERR_SEQ_LEN);
+        L = L < 0 ? 0 : cap;
+      }
+      own_len[j] = L;
+      if (j < nseq) Lmin = min(Lmin, L);
+    }
+    int P = sp.prefix_lens[grp];
+    if (P < 0 || P % p.block_size != 0 || P > Lmin) {
+      if (sub == 0 && kvh == 0) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+      P = P < 0 ? 0 : (min(P, Lmin) / p.block_size) * p.block_size;
+    }
+    const int pblk = P / kBlockSize;
+    int pos = pblk;
+    for (int j = 0; j < kSharedCols; ++j) {
+      own_start[j] = pos;
+      if (j < nseq) pos += (own_len[j] + kBlockSize - 1) / kBlockSize - pblk;
+    }
+    own_start[kSharedCols] = pos;
+    for (int st = 0; st < kStRing; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kStWorkers);
+    }
+    mbar_init(kready, kStWorkers);
+    mbar_init(pready, kStWorkers);
+    mbar_init(sdone, 1);
+    mbar_init(odone, 1);
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == kStMmaWarp) {  // the MMA warp owns the TMEM allocation
+    tmem_alloc(tmem_slot, kStTmemCols);
+    tmem_relinquish();
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  tcgen05_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int pblk = own_start[0];
+  ntotal = own_start[kSharedCols];
+  const int nstages = (ntotal + kStTiles - 1) / kStTiles;
+
+  if (warp == kStProducerWarp) {
+    // ---------------- producer: raw E4M3 tiles of each stage ----------------
+    const uint64_t policy = l2_policy_evict_first();
+    int issued = 0, ent = -1;
+    bool ok = true;
+    for (int st = 0; st < nstages && ok; ++st) {
+      // one table read per lane covers 4 stages: lane l takes stream tile 8 st + l
+      if ((st & 3) == 0) {
+        const int T = st * kStTiles + lane;
+        ent = -1;
+        if (T < ntotal) {
+          int j = 0, lt = T;  // member whose table holds the tile, logical tile there
+          if (T >= pblk) {
+            while (j + 1 < nseq && own_start[j + 1] <= T) ++j;
+            lt = pblk + (T - own_start[j]);
+          }
+          const int e = lt / p.tiles_per_block;
+          int32_t phys = p.block_tables[int64_t(s0 + j) * p.max_blocks_per_seq + e];
+          if (T < pblk) {  // the promise: every member has these blocks
+            for (int jj = 1; jj < nseq; ++jj)
+              if (p.block_tables[int64_t(s0 + jj) * p.max_blocks_per_seq + e] != phys)
+                atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+          }
+          if (phys < 0 || phys >= p.num_blocks) {
+            atomicOr(&g_shared_err, PA_DEVERR_BLOCK_RANGE);
+            phys = 0;
+          }
+          ent = ((phys * p.num_kv_heads + kvh) * p.tiles_per_block + (lt - e * p.tiles_per_block)) *
+                kBlockSize;
+        }
+      }
+      int rows[kStTiles];
+#pragma unroll
+      for (int i = 0; i < kStTiles; ++i) rows[i] = __shfl_sync(kFullMask, ent, (st & 3) * kStTiles + i);
+      const int slot = st % kStRing;
+      if (lane == 0) {
+        if (st >= kStRing && !mbar_wait_bounded(&empty[slot], ((st / kStRing) - 1) & 1)) {
+          atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+          ok = false;
+        }
+        if (ok) {
+          const int n = min(kStTiles, ntotal - st * kStTiles);
+          uint8_t* dst = raw + slot * kStRawStage;
+          mbar_arrive_expect_tx(&full[slot], uint32_t(n) * 2 * kStRawTile);
+          for (int i = 0; i < n; ++i) {
+            tma_load_2d(dst + i * kStRawTile, &sp.tmk, 0, rows[i], &full[slot], policy);
+            tma_load_2d(dst + (kStTiles + i) * kStRawTile, &sp.tmv, 0, rows[i], &full[slot],
+                        policy);
+          }
+          ++issued;
+        }
+      }
+      ok = __shfl_sync(kFullMask, ok, 0);
+    }
+    if (lane == 0) {  // no copy may still be landing when the CTA exits
+      for (int i = max(0, issued - kStRing); i < issued; ++i)
+        if (!mbar_wait_bounded(&full[i % kStRing], (i / kStRing) & 1))
+          atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp == kStMmaWarp) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      const uint64_t qdesc = umma_smem_desc(smem_u32(qop), 16, 1024, kUmmaSwizzle128B);
+      const uint64_t pdesc = umma_smem_desc(smem_u32(pop), 16, 1024, kUmmaSwizzle128B);
+      const uint64_t vdesc = umma_smem_desc(smem_u32(vf), kStVBytes / 2, 1024, kUmmaSwizzle128B);
+      bool ok = true;
+      for (int st = 0; st < nstages && ok; ++st) {
+        if (!(ok = mbar_wait_bounded(kready, st & 1))) break;
+        tcgen05_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)  // 16 dims per step: K columns 8 ks.., Q^T k-step ks
+          umma_f16_ts(tmem + kStTmemS, tmem + kStTmemK + uint32_t(8 * ks),
+                      qdesc + uint64_t(((ks >> 2) * kStOpHalf + (ks & 3) * 32) >> 4), kStIdescS,
+                      ks > 0 ? 1u : 0u);
+        umma_commit(sdone);
+        if (!(ok = mbar_wait_bounded(pready, st & 1))) break;
+        tcgen05_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)  // 16 tokens per step
+          umma_f16_ss(tmem + kStTmemO, vdesc + uint64_t((ks * 2048) >> 4),
+                      pdesc + uint64_t(((ks >> 2) * kStOpHalf + (ks & 3) * 32) >> 4), kStIdescPV,
+                      (st > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(odone);
+      }
+      if (!ok) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+      umma_commit(done);  // fires once every MMA issued above has completed
+      if (!mbar_wait_bounded(done, 0)) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- workers: thread = token row of S^T / dim row of O^T ----------------
+    const int r = tid;                                       // 0..127
+    const uint32_t tl = tmem + (uint32_t(32 * warp) << 16);  // this warp's lane quadrant
+    bool ok = true;  // warp-uniform; after a failure waits are skipped, barriers still met
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
+    };
+    auto arrive = [&](uint64_t* bar) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+    // ---- Q^T: thread t writes column n = t / 8, dims 16 (t % 8) .. + 15 (f16) ----
+    float mult = p.q_mult;
+    {
+      const int n = r >> 3, dc = r & 7;
+      const int j = n / G, hi = n - j * G;
+      const bool has = n < ncols;
+      uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+      if (has) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.query + (int64_t(s0 + j) * p.num_heads + kvh * G + hi) * D * 2 + dc * 32);
+        w0 = src[0];
+        w1 = src[1];
+      }
+      uint32_t q[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      if constexpr (!std::is_same<QT, __half>::value) {
+        // bf16 -> f16 with one power of two for the CTA: its largest |q| lands in
+        // [2^14, 2^15); the score multiplier takes the inverse
+        float qm = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 a = unpack2(q[i], QT{});
+          qm = fmaxf(qm, fmaxf(fabsf(a.x), fabsf(a.y)));
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(kFullMask, qm, o));
+        if (lane == 0) qmax_w[warp] = qm;
+        named_bar_sync(1, kStWorkers * 32);
+        qm = fmaxf(fmaxf(qmax_w[0], qmax_w[1]), fmaxf(qmax_w[2], qmax_w[3]));
+        int e = 0;
+        if (qm > 0.f && isfinite(qm)) frexpf(qm, &e);
+        const int sq = min(max(15 - e, -100), 100);
+        mult = ldexpf(mult, -sq);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 a = unpack2(q[i], QT{});
+          q[i] = pack2(ldexpf(a.x, sq), ldexpf(a.y, sq), __half{});
+        }
+      }
+      // K-major, 128-byte swizzle: dim d of row n in half d / 64, 16-byte chunk
+      // (d % 64) / 8 stored at chunk ^ (n % 8)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int d0 = 16 * dc + 8 * c, h = d0 >> 6, ch = (d0 & 63) >> 3;
+        *reinterpret_cast<uint4*>(qop + h * kStOpHalf + n * 128 + ((ch ^ (n & 7)) << 4)) =
+            make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
+      }
+      fence_proxy_async_smem();  // the MMA reads it through the async proxy
+    }
+
+    float mref[kSharedCols], lacc[kSharedCols];
+#pragma unroll
+    for (int n = 0; n < kSharedCols; ++n) {
+      mref[n] = -INFINITY;
+      lacc[n] = 0.f;
+    }
+    const int rr = r & 15;             // row within its pool tile
+    const int sw = (rr & 7);           // the TMA's 128-byte swizzle of that row
+    for (int st = 0; st < nstages; ++st) {
+      const int slot = st % kStRing;
+      // this row's token: stream tile T, its member (-1: prefix) and validity
+      const int T = st * kStTiles + (r >> 4);
+      int owner = -1;
+      bool valid = T < ntotal;
+      if (valid && T >= pblk) {
+        owner = 0;
+        while (owner + 1 < nseq && own_start[owner + 1] <= T) ++owner;
+        valid = (pblk + (T - own_start[owner])) * kBlockSize + rr < own_len[owner];
+      }
+      const int lo = owner < 0 ? 0 : owner * G, hi = owner < 0 ? ncols : lo + G;
+      wait(&full[slot], (st / kStRing) & 1);
+      const uint8_t* rk = raw + slot * kStRawStage + (r >> 4) * kStRawTile + rr * 128;
+      const uint8_t* rv = rk + kStTiles * kStRawTile;
+      // ---- K row -> TMEM (A operand), f16 pairs: column c holds dims 2c, 2c + 1 ----
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float kw[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(rk + (((4 * h + c) ^ sw) << 4));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t a, b;
+            e4m3x4_to_f16x4(ww[i], a, b);
+            kw[8 * c + 2 * i] = __uint_as_float(a);
+            kw[8 * c + 2 * i + 1] = __uint_as_float(b);
+          }
+        }
+        tmem_st32(tl + kStTmemK + 32 * h, kw);
+      }
+      tmem_wait_st();
+      tcgen05_fence_before();
+      arrive(kready);
+      // ---- V row -> f16 operand (MN-major, 128-byte swizzle), once P.V(st - 1) is done ----
+      if (st > 0) wait(odone, (st - 1) & 1);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) w = *reinterpret_cast<const uint4*>(rv + ((c ^ sw) << 4));
+        uint32_t f[8];
+        e4m3x4_to_f16x4(w.x, f[0], f[1]);
+        e4m3x4_to_f16x4(w.y, f[2], f[3]);
+        e4m3x4_to_f16x4(w.z, f[4], f[5]);
+        e4m3x4_to_f16x4(w.w, f[6], f[7]);
+        // dims 16c .. 16c + 15: chunks 2c and 2c + 1 of the row, half c / 4
+        uint8_t* vrow = vf + (c >> 2) * (kStVBytes / 2) + r * 128;
+        const int c0 = (2 * c) & 7;
+        *reinterpret_cast<uint4*>(vrow + ((c0 ^ (r & 7)) << 4)) = make_uint4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<uint4*>(vrow + (((c0 + 1) ^ (r & 7)) << 4)) =
+            make_uint4(f[4], f[5], f[6], f[7]);
+      }
+      arrive(&empty[slot]);  // the raw stage is read (K and V)
+      // ---- scores of this row, masked, in log2 units ----
+      wait(sdone, st & 1);
+      tcgen05_fence_after();
+      float x[kSharedCols];
+      tmem_ld16(tl + kStTmemS, x);
+      tmem_wait_ld();
+      bool up = false;
+#pragma unroll
+      for (int n = 0; n < kSharedCols; ++n) {
+        x[n] = (valid && n >= lo && n < hi) ? x[n] * mult : -INFINITY;
+        up |= x[n] > mref[n] + kSharedRescaleLog2;
+      }
+      // ---- does any column's reference maximum move?  (vote, 128 threads) ----
+      const int fb = (st & 1) * kStWorkers;
+      const unsigned vote = __ballot_sync(kFullMask, up);
+      if (lane == 0) flags[fb + warp] = vote != 0u;
+      named_bar_sync(1, kStWorkers * 32);
+      if (flags[fb] | flags[fb + 1] | flags[fb + 2] | flags[fb + 3]) {  // uniform
+#pragma unroll
+        for (int n = 0; n < kSharedCols; ++n) {
+          float m = x[n];
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+          if (lane == 0) wmax[(fb + warp) * kSharedCols + n] = m;
+        }
+        named_bar_sync(1, kStWorkers * 32);
+        float alpha[kSharedCols];
+        bool moved = false;
+#pragma unroll
+        for (int n = 0; n < kSharedCols; ++n) {
+          const float* wm = wmax + fb * kSharedCols + n;
+          const float cm = fmaxf(fmaxf(wm[0], wm[kSharedCols]),
+                                 fmaxf(wm[2 * kSharedCols], wm[3 * kSharedCols]));
+          const float mn = cm > mref[n] + kSharedRescaleLog2 ? cm : mref[n];
+          alpha[n] = mn == mref[n] ? 1.f : ex2_approx_ftz(mref[n] - mn);  // -inf -> 0
+          moved |= mn != mref[n];
+          mref[n] = mn;
+          lacc[n] *= alpha[n];
+        }
+        if (st > 0 && moved) {  // O^T columns (this thread's dim row) follow
+          float o[kSharedCols];
+          tmem_ld16(tl + kStTmemO, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int n = 0; n < kSharedCols; ++n) o[n] *= alpha[n];
+          tmem_st16_f(tl + kStTmemO, o);
+          tmem_wait_st();
+        }
+      }
+      // ---- P^T row: K-major, 128-byte swizzle (token r = k index) ----
+      uint8_t* prow = pop + (r >> 6) * kStOpHalf + 2 * (r & 7);
+      const int pc = (r & 63) >> 3;
+#pragma unroll
+      for (int n = 0; n < kSharedCols; ++n) {
+        const float pn = x[n] > -INFINITY ? ex2_approx_ftz(x[n] - mref[n]) : 0.f;
+        lacc[n] += pn;
+        *reinterpret_cast<__half*>(prow + n * 128 + ((pc ^ (n & 7)) << 4)) = __float2half_rn(pn);
+      }
+      fence_proxy_async_smem();
+      tcgen05_fence_before();
+      arrive(pready);
+    }
+    // ---- epilogue: column sums over the CTA, O^T row of this dim, outputs ----
+    if (nstages > 0) wait(odone, (nstages - 1) & 1);
+    tcgen05_fence_after();
+#pragma unroll
+    for (int n = 0; n < kSharedCols; ++n) {
+      float v = lacc[n];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(kFullMask, v, o);
+      if (lane == 0) lsum[warp * kSharedCols + n] = v;
+    }
+    named_bar_sync(1, kStWorkers * 32);
+    float o[kSharedCols];
+    if (nstages > 0) {
+      tmem_ld16(tl + kStTmemO, o);
+      tmem_wait_ld();
+    }
+    for (int n = 0; n < ncols; ++n) {
+      const float L = lsum[n] + lsum[kSharedCols + n] + lsum[2 * kSharedCols + n] +
+                      lsum[3 * kSharedCols + n];
+      const float v = L > 0.f ? o[n] * (p.v_mult / L) : 0.f;  // an empty context gives zeros
+      const int j = n / G, hh = n - j * G;
+      store_out(p.out, (int64_t(s0 + j) * p.num_heads + kvh * G + hh) * D + r, v, p.out_dtype);
+    }
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  if (warp == kStMmaWarp) {
+    tcgen05_fence_after();
+    tmem_dealloc(tmem, kStTmemCols);
+  }
+}
+
+template <typename CT, typename QT>
+int launch_shared_typed(const SharedParams& base, int grid_x, cudaStream_t stream) {
+  constexpr bool fp8 = CacheTraits<CT>::bytes == 1;
+  constexpr int stages = fp8 ? kSharedStagesFp8 : kSharedStages16;
+  constexpr size_t smem = shared_smem_bytes<CT, stages>();
+  auto kern = decode_shared_prefix_kernel<CT, QT, stages>;
+  static std::atomic<unsigned long long> smem_set{0};
+  if (set_smem_once(kern, smem, smem_set) != PA_OK) return PA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid_x) * unsigned(base.cluster), unsigned(base.p.num_kv_heads));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(base.cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, base);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts,
+                                const int32_t* prefix_lens, int num_groups, int max_group_size,
+                                cudaStream_t stream) {
+  const int group = a.num_heads / a.num_kv_heads;
+  const int64_t rows = a.num_blocks * a.num_kv_heads * a.block_size;
+  if (a.head_dim != 128 || group > kSharedCols || rows >= (int64_t(1) << 31) ||
+      encode_fn() == nullptr)
+    return PA_ERR_UNSUPPORTED;
+  SharedParams sp;
+  memset(&sp, 0, sizeof sp);
+  Params& p = sp.p;
+  p.out = a.out;
+  p.query = static_cast<const uint8_t*>(a.query);
+  p.block_tables = a.block_tables;
+  p.seq_lens = a.seq_lens;
+  p.max_blocks_per_seq = a.max_blocks_per_seq;
+  p.block_size = a.block_size;
+  p.tiles_per_block = a.block_size / kBlockSize;
+  p.max_seq_len = a.max_seq_len;
+  p.cap = context_cap(a.max_seq_len, a.max_blocks_per_seq, a.block_size);
+  p.num_heads = a.num_heads;
+  p.num_kv_heads = a.num_kv_heads;
+  p.group = group;
+  p.head_groups = 1;
+  p.partition = a.max_seq_len > 0 ? a.max_seq_len : 1;
+  p.max_parts = 1;
+  p.out_dtype = a.out_dtype;
+  p.num_blocks = a.num_blocks;
+  p.num_seqs = a.num_seqs;
+  const bool fp8 = a.cache_dtype == PA_FP8_E4M3;
+  p.q_mult = a.scale * kLog2e * (fp8 ? a.k_scale : 1.f);
+  p.v_mult = fp8 ? a.v_scale : 1.f;
+  sp.group_starts = group_starts;
+  sp.prefix_lens = prefix_lens;
+  sp.seqs_per_cta = kSharedCols / group;
+  sp.ctas_per_group = (max_group_size + sp.seqs_per_cta - 1) / sp.seqs_per_cta;
+  const int64_t grid_x = int64_t(num_groups) * sp.ctas_per_group;
+  // Split each unit's block stream over a cluster of up to 8 CTAs when there are
+  // too few units to keep the GPU streaming, keeping chunks of at least
+  // PA_SHARED_MIN_CHUNK blocks.
+  {
+    const int64_t units = grid_x * a.num_kv_heads;
+    int c = int((kAutoTargetCtas + units - 1) / (units > 0 ? units : 1));
+    const int est_blocks = (a.max_seq_len + kBlockSize - 1) / kBlockSize;
+    c = min(c, max(1, est_blocks / PA_SHARED_MIN_CHUNK));
+    sp.cluster = max(1, min(c, 8));
+  }
+  if (grid_x * sp.cluster > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (!encode_pool_map(&sp.tmk, a.key_cache, rows, fp8) ||
+      !encode_pool_map(&sp.tmv, a.value_cache, rows, fp8))
+    return PA_ERR_CUDA;
+  if (fp8) {  // the tensor-core kernel: no cluster split
+    sp.cluster = 1;
+    constexpr size_t smem = shared_tc_smem_bytes();
+    const dim3 grid(unsigned(grid_x), unsigned(a.num_kv_heads));
+    if (a.q_dtype == PA_F16) {
+      static std::atomic<unsigned long long> done_h{0};
+      if (set_smem_once(decode_shared_tc_kernel<__half>, smem, done_h) != PA_OK) return PA_ERR_CUDA;
+      decode_shared_tc_kernel<__half><<<grid, kStThreads, smem, stream>>>(sp);
+    } else if (a.q_dtype == PA_BF16) {
+      static std::atomic<unsigned long long> done_b{0};
+      if (set_smem_once(decode_shared_tc_kernel<__nv_bfloat16>, smem, done_b) != PA_OK)
+        return PA_ERR_CUDA;
+      decode_shared_tc_kernel<__nv_bfloat16><<<grid, kStThreads, smem, stream>>>(sp);
+    } else {
+      return PA_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  }
+  if (a.cache_dtype == PA_F16 && a.q_dtype == PA_F16)
+    return launch_shared_typed<__half, __half>(sp, int(grid_x), stream);
+  if (a.cache_dtype == PA_BF16 && a.q_dtype == PA_BF16)
+    return launch_shared_typed<__nv_bfloat16, __nv_bfloat16>(sp, int(grid_x), stream);
+  if (fp8 && a.q_dtype == PA_F16) return launch_shared_typed<fp8_e4m3, __half>(sp, int(grid_x), stream);
+  if (fp8 && a.q_dtype == PA_BF16)
+    return launch_shared_typed<fp8_e4m3, __nv_bfloat16>(sp, int(grid_x), stream);
+  return PA_ERR_UNSUPPORTED;
+}
+
+cudaError_t read_and_clear_shared_errors(unsigned* bits, cudaStream_t stream) {
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_shared_err, sizeof v, 0,
+                                            cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_shared_err, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,
+                              stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  *bits |= v;
+  return e;
+}
+
+}  // namespace pa

@@ -113,5 +113,6 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
 cudaError_t read_and_clear_cache_errors(unsigned* bits, cudaStream_t stream);
 cudaError_t read_and_clear_decode_errors(unsigned* bits, cudaStream_t stream);
 cudaError_t read_and_clear_prefill_errors(unsigned* bits, cudaStream_t stream);
+cudaError_t read_and_clear_shared_errors(unsigned* bits, cudaStream_t stream);
 
 }  // namespace pa

@@ -7,6 +7,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
 #include <type_traits>
 
 #include "pa_common.cuh"
@@ -34,6 +35,8 @@ struct Params {
   int block_size;       // tokens per physical block (a multiple of 16)
   int tiles_per_block;  // block_size / 16
   int max_seq_len;
+  int cap;              // longest context the launch serves: min(max_seq_len, table width
+                        // * block_size), computed on the host in 64 bits
   int num_heads;
   int num_kv_heads;
   int group;        // query heads per kv head
@@ -97,6 +100,45 @@ bool encode_pool_map(CUtensorMap* m, const void* base, int64_t rows, bool fp8) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+// Combine region layout: per warp and head the max (log2 units) and the sum, then
+// the unnormalised accumulators with rows padded to D + 4 floats, which keeps the
+// fragment-order writes of the four column groups on distinct banks.
+template <int D>
+constexpr int combine_row() {
+  return D + 4;
+}
+template <int D, int GT>
+constexpr size_t combine_bytes() {
+  return (size_t(kConsumerWarps) * GT * 2 + size_t(kConsumerWarps) * GT * combine_row<D>() +
+          size_t(GT) * (kConsumerWarps + 1)) *
+         sizeof(float);
+}
+
+// Longest context a launch can serve: the host bound, or what the block tables
+// can hold if that is less.  The product is taken in 64 bits, so wide tables of
+// large blocks cannot overflow it; the result fits an int because max_seq_len does.
+inline int context_cap(int max_seq_len, int max_blocks_per_seq, int block_size) {
+  const int64_t table = int64_t(max_blocks_per_seq) * block_size;
+  return table < max_seq_len ? int(table) : max_seq_len;
+}
+
+// Opt a kernel into `smem` bytes of dynamic shared memory on the current device,
+// once per device and instantiation.  `done` records the devices set so far;
+// fetch_or keeps concurrent host threads race-free (two of them may both make the
+// idempotent call).  Devices past 63 are not recorded and get the call every time.
+template <typename Kernel>
+int set_smem_once(Kernel kern, size_t smem, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return PA_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  done.fetch_or(bit, std::memory_order_release);
+  return PA_OK;
+}
 
 __device__ __forceinline__ void store_out(void* out, int64_t idx, float v, int dtype) {
   if (dtype == PA_F32)

@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
   const int G = p.group;
   const int32_t* table_row = p.block_tables + int64_t(seq) * p.max_blocks_per_seq;
 
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+  const int cap = p.cap;
   int L = p.seq_lens[seq];
   const int q0 = pp.query_start[seq];
   int nq = pp.query_start[seq + 1] - q0;
@@ -401,7 +401,7 @@ __device__ __forceinline__ bool tc_tile(const TcPrefillParams& pp, int tile, TcT
   const int rem = tile - t.seq * per_seq;
   t.kvh = rem / pp.row_blocks;
   const int rblk = rem - t.kvh * pp.row_blocks;
-  const int cap = min(p.max_seq_len, p.max_blocks_per_seq * p.block_size);
+  const int cap = p.cap;
   int L = p.seq_lens[t.seq];
   t.q0 = pp.query_start[t.seq];
   int nq = pp.query_start[t.seq + 1] - t.q0;
@@ -885,6 +885,7 @@ int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_quer
   p.block_size = a.block_size;
   p.tiles_per_block = a.block_size / kBlockSize;
   p.max_seq_len = a.max_seq_len;
+  p.cap = context_cap(a.max_seq_len, a.max_blocks_per_seq, a.block_size);
   p.num_heads = a.num_heads;
   p.num_kv_heads = a.num_kv_heads;
   p.group = group;
@@ -901,20 +902,12 @@ int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_quer
       !encode_pool_map(&pp.tmv, a.value_cache, rows, false))
     return PA_ERR_CUDA;
   constexpr int stages = 4;
-  auto run = [&](auto kern, size_t smem, unsigned long long& mask) -> int {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (!(mask & bit)) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-          cudaSuccess)
-        return PA_ERR_CUDA;
-      mask |= bit;
-    }
+  auto run = [&](auto kern, size_t smem, std::atomic<unsigned long long>& mask) -> int {
+    if (set_smem_once(kern, smem, mask) != PA_OK) return PA_ERR_CUDA;
     kern<<<dim3(unsigned(grid_x), unsigned(a.num_kv_heads)), kThreads, smem, stream>>>(pp);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   };
-  static unsigned long long mask_h = 0, mask_b = 0;
+  static std::atomic<unsigned long long> mask_h{0}, mask_b{0};
   if (int64_t(max_query_len) * group >= kTcRows) {
     // 128-row tiles for the 5th-generation tensor cores
     TcPrefillParams tp;
@@ -934,20 +927,12 @@ int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_quer
       return PA_ERR_CUDA;
     const unsigned grid_tc = unsigned(tiles < sms ? tiles : sms);
     constexpr size_t smem = tc_prefill_smem_bytes();
-    auto launch = [&](auto kern, unsigned long long& mask) -> int {
-      int dev = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-      const unsigned long long bit = 1ull << (dev & 63);
-      if (!(mask & bit)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-            cudaSuccess)
-          return PA_ERR_CUDA;
-        mask |= bit;
-      }
+    auto launch = [&](auto kern, std::atomic<unsigned long long>& mask) -> int {
+      if (set_smem_once(kern, smem, mask) != PA_OK) return PA_ERR_CUDA;
       kern<<<grid_tc, kTcThreads, smem, stream>>>(tp);
       return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
     };
-    static unsigned long long tmask_h = 0, tmask_b = 0, tmask_bs = 0;
+    static std::atomic<unsigned long long> tmask_h{0}, tmask_b{0}, tmask_bs{0};
     if (a.cache_dtype == PA_F16) return launch(prefill_tc_kernel<__half, false>, tmask_h);
     if (a.out_dtype == PA_F32) return launch(prefill_tc_kernel<__nv_bfloat16, true>, tmask_bs);
     return launch(prefill_tc_kernel<__nv_bfloat16, false>, tmask_b);

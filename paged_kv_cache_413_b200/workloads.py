@@ -353,14 +353,21 @@ def _shared_prefixes(tables, group_sizes, lens, bs):
 def make_group_workload(num_groups: int, group_size: tuple, prefix_blocks: tuple,
                         own_len: tuple, *, num_heads: int, num_kv_heads: int,
                         head_dim: int = 128, dtype: str = "bf16", seed: int = 0,
-                        pool_factor: float = 1.3, block_size: int = BLOCK_SIZE) -> Workload:
-    """Groups of sequences forked from a shared prompt prefix (16-bit caches).
+                        pool_factor: float = 1.3, block_size: int = BLOCK_SIZE,
+                        cache_dtype: str | None = None) -> Workload:
+    """Groups of sequences forked from a shared prompt prefix.
 
     Each group draws a size in ``group_size`` and a number of shared full blocks
     in ``prefix_blocks`` (inclusive ranges); every member then owns
     ``own_len`` tokens (at least 1: its last token is the new one) in blocks of
     its own.  Draw order: group sizes, prefix blocks, own lengths, block
     permutation, Q, K pool, V pool, new-token K, new-token V.
+
+    The cache is ``dtype`` (16-bit, a bit copy of the draws rounded to it) unless
+    ``cache_dtype`` is "e4m3": the pool then holds the draws divided by one fp32
+    scale per pool (amax / 448 over the pool's and the new tokens' draws) and
+    rounded to E4M3, and the new tokens (``dtype``) are quantised by the step's
+    cache write with the same scales.
     """
     bs = block_size
     rng = np.random.default_rng(seed)
@@ -397,20 +404,29 @@ def make_group_workload(num_groups: int, group_size: tuple, prefix_blocks: tuple
     for i, L in enumerate(lens):  # the new tokens' slots stay poisoned until written
         s = int(slots[i])
         owned[s // bs, s % bs] = False
+    cdt = cache_dtype or dtype
+    k_scale = v_scale = 1.0
+    if cdt == "e4m3":
+        amax = lambda a, b: np.float32(max(np.nanmax(np.abs(a)), np.abs(b).max()))
+        k_scale = float(amax(kpool, nk) / np.float32(448.0))
+        v_scale = float(amax(vpool, nv) / np.float32(448.0))
+        kpool = kpool / np.float32(k_scale)
+        vpool = vpool / np.float32(v_scale)
     for b in np.nonzero(~owned.all(axis=1))[0]:
         kpool[b][:, ~owned[b], :] = np.nan
         vpool[b][:, ~owned[b], :] = np.nan
     cfg = DecodeConfig("groups", num_seqs=B, num_heads=num_heads, num_kv_heads=Hkv, head_dim=D,
                        seq_lens=tuple(int(x) for x in lens), num_blocks=nb, q_dtype=dtype,
-                       cache_dtype=dtype, out_dtype=dtype, seed=seed, block_size=bs)
+                       cache_dtype=cdt, out_dtype=dtype, seed=seed, block_size=bs)
     starts, prefixes = _shared_prefixes(tables, [int(x) for x in sizes], lens, bs)
     width = max(len(t) for t in tables)
-    return Workload(cfg=cfg, query=q, key_cache=_to_storage(kpool, dtype),
-                    value_cache=_to_storage(vpool, dtype), block_tables=_table_tensor(tables, width),
+    return Workload(cfg=cfg, query=q, key_cache=_to_storage(kpool, cdt),
+                    value_cache=_to_storage(vpool, cdt), block_tables=_table_tensor(tables, width),
                     seq_lens=torch.from_numpy(lens.astype(np.int32)),
                     new_key=_to_storage(nk, dtype), new_value=_to_storage(nv, dtype),
-                    slot_mapping=torch.from_numpy(slots), scale=_scale(D), src_dtype=dtype,
-                    refs=dict(pool.refs), group_starts=starts, prefix_lens=prefixes)
+                    slot_mapping=torch.from_numpy(slots), scale=_scale(D), k_scale=k_scale,
+                    v_scale=v_scale, src_dtype=dtype, refs=dict(pool.refs), group_starts=starts,
+                    prefix_lens=prefixes)
 
 
 def make_prefill_workload(num_seqs: int, context: tuple, chunk: tuple, *, num_heads: int,

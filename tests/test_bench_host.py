@@ -57,48 +57,41 @@ def test_prefill_flops_enumerated():
     assert bench.prefill_flops(wl) == pairs * cfg.num_heads * cfg.head_dim * 4
 
 
-def _profile_record(path, key):
-    import re
-    text = open(path).read()
-    sha = re.search(key + r":\s*([0-9a-f]{16})", text)
-    dram = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    return sha.group(1), int(dram.group(1))
+def test_recorded_traffic_only_while_the_profiled_sources_hash_the_same(monkeypatch, tmp_path):
+    """A recorded ncu figure is reported only for the sources it was taken on."""
+    import json
 
-
-def test_recorded_traffic_only_while_the_profiled_sources_hash_the_same(monkeypatch):
-    """A committed ncu figure is reported only for the sources it was taken on."""
-    import glob
-    import os
-    decode = sorted(glob.glob(os.path.join(bench.ROOT, "profiles",
-                                           "paged_attention_decode_*.md")))
-    prefill = sorted(glob.glob(os.path.join(bench.ROOT, "profiles", "prefill_tc_*.md")))
-    assert decode and prefill
-    now_d = bench.source_sha(bench.DECODE_SOURCES)
-    now_p = bench.source_sha(bench.PREFILL_SOURCES)
-    for path in decode:
-        cfg = os.path.basename(path)[len("paged_attention_decode_"):-3]
-        sha, dram = _profile_record(path, "decode_source_sha256_16")
-        assert bench.recorded_traffic(cfg) == (dram if sha == now_d else None)
-    for path in prefill:
-        cfg = os.path.basename(path)[len("prefill_tc_"):-3]
-        sha, dram = _profile_record(path, "prefill_source_sha256_16")
-        assert bench.recorded_prefill_traffic(cfg) == (dram if sha == now_p else None)
-    # both branches, whatever the committed sources hash to: the figure while the
-    # hash matches, none after any change
-    for path in decode:
-        cfg = os.path.basename(path)[len("paged_attention_decode_"):-3]
-        sha, dram = _profile_record(path, "decode_source_sha256_16")
-        monkeypatch.setattr(bench, "source_sha", lambda names=None, s=sha: s)
-        assert bench.recorded_traffic(cfg) == dram
-        monkeypatch.setattr(bench, "source_sha", lambda names=None: "0" * 16)
-        assert bench.recorded_traffic(cfg) is None
-    for path in prefill:
-        cfg = os.path.basename(path)[len("prefill_tc_"):-3]
-        sha, dram = _profile_record(path, "prefill_source_sha256_16")
-        monkeypatch.setattr(bench, "source_sha", lambda names=None, s=sha: s)
-        assert bench.recorded_prefill_traffic(cfg) == dram
-        monkeypatch.setattr(bench, "source_sha", lambda names=None: "0" * 16)
-        assert bench.recorded_prefill_traffic(cfg) is None
-    # and a workload without a profile has none
-    monkeypatch.undo()
+    sha = bench.source_sha(bench.DECODE_SOURCES)
+    rec = {"workloads": {
+        "fresh": {"sources": list(bench.DECODE_SOURCES), "sources_sha256_16": sha,
+                  "dram_bytes_per_launch": 1234},
+        "stale": {"sources": list(bench.DECODE_SOURCES), "sources_sha256_16": "0" * 16,
+                  "dram_bytes_per_launch": 99}}}
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_JSON", str(path))
+    assert bench.recorded_traffic("fresh") == 1234
+    assert bench.recorded_traffic("stale") is None
     assert bench.recorded_traffic("no_such_workload") is None
+    # any change to a listed source retires the figure
+    monkeypatch.setattr(bench, "source_sha", lambda names=None: "f" * 16)
+    assert bench.recorded_traffic("fresh") is None
+    monkeypatch.setattr(bench, "TRAFFIC_JSON", str(tmp_path / "missing.json"))
+    assert bench.recorded_traffic("fresh") is None
+
+
+def test_committed_traffic_records_are_complete():
+    """Every committed record names existing sources, a summary under profiles/
+    and the capture command, and carries a positive byte count."""
+    import json
+    import os
+
+    with open(bench.TRAFFIC_JSON) as f:
+        rec = json.load(f)["workloads"]
+    for name, r in rec.items():
+        for src in r["sources"]:
+            assert os.path.exists(os.path.join(bench.ROOT, "paged_kv_cache_413_b200", "csrc", src))
+        assert len(r["sources_sha256_16"]) == 16
+        assert int(r["dram_bytes_per_launch"]) > 0
+        assert os.path.exists(os.path.join(bench.ROOT, "profiles", r["summary"])), name
+        assert "ncu" in r["command"] and "--clock-control none" in r["command"]

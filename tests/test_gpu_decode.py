@@ -202,8 +202,9 @@ def test_full_llama2_70b_gqa():
 
 
 def test_full_long_splitk():
+    # every output of all 8 sequences (64 partitions each, merged by the reduce)
     wl = W.make_workload("long_splitk")
-    _check(wl, "bf16", wl.cfg.partition_size, seqs=[0, 5])
+    _check(wl, "bf16", wl.cfg.partition_size)
 
 
 def test_full_beam_cow_fp8():

@@ -4,8 +4,9 @@ The oracle is the ordinary per-sequence decode: sharing blocks changes where the
 bytes come from, never the result.  Cases: beam-search workloads with an FP8
 cache (the copy-on-write recipe), random groups of sequences forked from a common
 prefix with GQA group sizes 1..16 (groups larger than one CTA's share included),
-broken promises (they set PA_DEVERR_PREFIX and fault nothing), and the full-size
-beam workload on sampled prompts.
+broken promises (they set PA_DEVERR_PREFIX and fault nothing), E4M3 caches of
+every group shape (the tensor-core kernel), and the full-size beam workload, every
+output.
 """
 
 import numpy as np
@@ -105,10 +106,42 @@ def test_broken_promises_set_error_bits_without_fault():
 
 
 def test_full_beam_cow_fp8_shared():
+    # every output of the full-size workload, in the benchmark's launch configuration
     wl = W.make_workload("beam_cow_fp8")
-    prompts = [0, 21, 63]
-    seqs = [p * 4 + w for p in prompts for w in range(4)]
-    _check(wl, "bf16", seqs=seqs, prompts=prompts)
+    _check(wl, "bf16")
+
+
+@pytest.mark.parametrize("h,hkv,qdt", [(32, 8, "bf16"), (16, 16, "f16"), (32, 16, "bf16"),
+                                       (64, 8, "f16"), (64, 4, "bf16"), (24, 8, "bf16")])
+def test_groups_fp8(h, hkv, qdt):
+    """E4M3 caches: GQA groups of 1 to 16 heads, members whose own tiles span several
+    128-token stages, prefixes of 0 to 5 blocks, groups of 1 to 7 members."""
+    wl = W.make_group_workload(5, (1, 7), (0, 5), (1, 300), num_heads=h, num_kv_heads=hkv,
+                               dtype=qdt, seed=h * 3 + hkv, cache_dtype="e4m3")
+    d, out = _check(wl, "f32")
+    ref = torch.empty_like(out)
+    pa.pa_paged_attention_decode(ref, d.query, d.key_cache, d.value_cache, d.block_tables,
+                                 d.seq_lens, max_seq_len=flow.max_seq_len(wl), scale=wl.scale,
+                                 k_scale=wl.k_scale, v_scale=wl.v_scale, partition_size=1024)
+    assert (out - ref).abs().max().item() <= 2e-3
+
+
+@pytest.mark.parametrize("bs", [32, 64, 128])
+def test_groups_fp8_block_sizes(bs):
+    wl = W.make_group_workload(4, (2, 6), (0, 4), (1, 200), num_heads=32, num_kv_heads=8,
+                               dtype="bf16", seed=bs + 1, block_size=bs, cache_dtype="e4m3")
+    _check(wl, "bf16")
+
+
+def test_fp8_long_prefix_and_one_token_members():
+    """A 4000-token prefix (32 stages) shared by 6 members, next to groups whose
+    members own every token (prefix 0) and one-token members."""
+    wl = W.make_group_workload(3, (6, 6), (250, 250), (1, 40), num_heads=32, num_kv_heads=8,
+                               dtype="bf16", seed=11, cache_dtype="e4m3")
+    _check(wl, "f32")
+    wl = W.make_group_workload(6, (1, 4), (0, 0), (1, 1), num_heads=16, num_kv_heads=4,
+                               dtype="f16", seed=12, cache_dtype="e4m3")
+    _check(wl, "f16")
 
 
 @pytest.mark.parametrize("bs", [32, 64])
