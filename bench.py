@@ -442,6 +442,46 @@ def timed_loop(step, launches, steps, warmup, dev, stream, world, rank):
     return elapsed_ms, launch_ms, (sampler.summary() if sampler else None)
 
 
+def timing_note(args) -> str:
+    if args.no_graphs:
+        return "each timed step calls the library from Python (host launch overhead included)"
+    return ("each timed step replays two CUDA graphs of the library's calls (cache writes, then "
+            "the hot kernels); CUDA events on the stream bracket the hot graph")
+
+
+def graph_step(writes, hot, run_step, inputs, out, ev, dev, stream, args):
+    """The step the timed loop runs.  By default each step replays two CUDA graphs
+    captured from the same library calls -- the cache writes (and copies), then the
+    hot kernel(s) -- with the hot launch's events recorded between them on the
+    stream, so host-side call overhead never idles the GPU inside the timed region.
+    With --no-graphs the step calls the library directly (run_step)."""
+    if args.no_graphs:
+        return lambda timed: run_step(inputs, out, timed)
+    run_step(inputs, out, False)          # warm: every kernel attribute set, maps encoded
+    torch.cuda.synchronize(dev)
+    gw, gh = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.graph(gw, stream=side):
+        writes()
+    with torch.cuda.graph(gh, stream=side):
+        hot()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+
+    def step(timed):
+        gw.replay()
+        if timed:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        gh.replay()
+        if timed:
+            e1.record(stream)
+            ev.append((e0, e1))
+
+    return step
+
+
 def decode_case(cfg, dev, args, world, rank, decode_mode="auto", partition=None,
                 with_e2e=True, with_cpu=False):
     """One decode workload, resident in HBM: W + K steps of (copy-on-write copies,
@@ -484,14 +524,13 @@ def decode_case(cfg, dev, args, world, rank, decode_mode="auto", partition=None,
     if shared:
         inputs.update(gs=gs, pl=pl)
 
-    def run_step(t, out_t, timed: bool = False):
+    def writes(t):
         if "bm" in t:
             pa.pa_copy_blocks([kc], [vc], t["bm"])
         pa.pa_reshape_and_cache(t["nk"], t["nv"], kc, vc, t["sm"], k_scale=wl.k_scale,
                                 v_scale=wl.v_scale)
-        if timed:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+
+    def decode(t, out_t):
         if shared:
             pa.pa_paged_attention_decode_shared_prefix(
                 out_t, t["q"], kc, vc, t["bt"], t["sl"], t["gs"], t["pl"], max_seq_len=max_len,
@@ -502,12 +541,21 @@ def decode_case(cfg, dev, args, world, rank, decode_mode="auto", partition=None,
                                          max_seq_len=max_len, scale=wl.scale,
                                          k_scale=wl.k_scale, v_scale=wl.v_scale,
                                          partition_size=part, workspace=ws)
+
+    def run_step(t, out_t, timed: bool = False):
+        writes(t)
+        if timed:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        decode(t, out_t)
         if timed:
             e1.record(stream)
             ev.append((e0, e1))
 
-    elapsed_ms, decode_ms, clocks = timed_loop(lambda timed: run_step(inputs, out, timed), ev,
-                                               args.steps, args.warmup, dev, stream, world, rank)
+    step = graph_step(lambda: writes(inputs), lambda: decode(inputs, out), run_step, inputs,
+                      out, ev, dev, stream, args)
+    elapsed_ms, decode_ms, clocks = timed_loop(step, ev, args.steps, args.warmup, dev, stream,
+                                               world, rank)
     dec_b = shared_decode_bytes(wl, out_dtype) if shared else decode_bytes(wl, out_dtype)
     step_bytes = dec_b + cache_write_bytes(wl) + copy_bytes(wl)
     res = {"wl": wl, "shared": shared, "part_eff": part_eff, "dec_b": dec_b,
@@ -572,7 +620,8 @@ def run_ours(args, rank, world, local_rank):
                    "partition_tokens": r["part_eff"], "out_dtype": out_dtype,
                    "l2": "no flush: inputs larger than L2 (%.2f GB read per step vs 126 MB L2)"
                          % (r["dec_b"] / 1e9),
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"replicas x{world}",
+                   "timing": timing_note(args)},
         "pct_of_peak": round(100.0 * value / peak, 2),
         "decode_tokens_per_s_per_layer": round(n_seqs * world / (ms_per_step * 1e-3), 1),
         "context_tokens_per_s_per_layer": round(int(L.sum()) * world / (ms_per_step * 1e-3), 1),
@@ -832,19 +881,27 @@ def prefill_case(name, dev, args, world, rank, with_e2e=True, with_cpu=False):
     ev = []
     inputs = {"q": q, "nk": nk, "nv": nv, "sm": sm, "bt": bt, "sl": sl, "qs": qs}
 
-    def run_step(t, out_t, timed=False):
+    def writes(t):
         pa.pa_reshape_and_cache(t["nk"], t["nv"], kc, vc, t["sm"])
+
+    def attend(t, out_t):
+        pa.pa_paged_attention_prefill(out_t, t["q"], kc, vc, t["bt"], t["sl"], t["qs"],
+                                      max_query_len=max_q, max_seq_len=max_len, scale=wl.scale)
+
+    def run_step(t, out_t, timed=False):
+        writes(t)
         if timed:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        pa.pa_paged_attention_prefill(out_t, t["q"], kc, vc, t["bt"], t["sl"], t["qs"],
-                                      max_query_len=max_q, max_seq_len=max_len, scale=wl.scale)
+        attend(t, out_t)
         if timed:
             e1.record(stream)
             ev.append((e0, e1))
 
-    elapsed_ms, kern_ms, clocks = timed_loop(lambda timed: run_step(inputs, out, timed), ev,
-                                             args.steps, args.warmup, dev, stream, world, rank)
+    step = graph_step(lambda: writes(inputs), lambda: attend(inputs, out), run_step, inputs,
+                      out, ev, dev, stream, args)
+    elapsed_ms, kern_ms, clocks = timed_loop(step, ev, args.steps, args.warmup, dev, stream,
+                                             world, rank)
     cfg = wl.cfg
     L = wl.seq_lens.numpy().astype(np.int64)
     res = {"wl": wl, "elapsed_ms": elapsed_ms, "kern_ms": kern_ms, "clocks": clocks,
@@ -905,7 +962,8 @@ def run_prefill(args, rank, world, local_rank):
             "data": "synthetic",
             "config": {"workload": f"{args.config}: {DESCR[args.config]}",
                        "query_tokens": p["query_tokens"], "flops_per_step": flops,
-                       "l2": f"KV read {p['kv_bytes'] / 1e6:.0f} MB per step, above the 126 MB L2"},
+                       "l2": f"KV read {p['kv_bytes'] / 1e6:.0f} MB per step, above the 126 MB L2",
+                       "timing": timing_note(args)},
             "roofline": prefill_roofline(args.config, p),
             "e2e": {"value": round(flops * world * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2),
                     "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -960,6 +1018,9 @@ def main():
     ap.add_argument("--decode", default="auto", choices=["auto", "shared", "standard"],
                     help="copy-on-write workloads: shared-prefix decode (auto) or per sequence")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="timed steps call the library directly instead of replaying CUDA "
+                         "graphs of the same calls")
     ap.add_argument("--no-configs", action="store_true",
                     help="default workload only: skip the `configs` map of the other workloads")
     args = ap.parse_args()

@@ -106,21 +106,34 @@ def _stream(stream) -> int:
     return int(stream)
 
 
-def _device_of(*tensors) -> torch.cuda.device:
-    """The device every CUDA tensor of a call lives on, as a context that makes it
-    current for the call (so the library launches there, on that device's current
-    stream).  Tensors on two different devices are rejected."""
+class _Current:
+    """No-op context: the call's device is already the current one."""
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+_CURRENT = _Current()
+
+
+def _device_of(*tensors):
+    """A context that makes current the device every CUDA tensor of a call lives on
+    (so the library launches there, on that device's current stream); a no-op when
+    it is current already.  Tensors on two different devices are rejected."""
     idx = None
     for t in tensors:
-        if isinstance(t, torch.Tensor) and t.device.type == "cuda":
-            i = t.device.index if t.device.index is not None else torch.cuda.current_device()
+        if isinstance(t, torch.Tensor) and t.is_cuda:
+            i = t.get_device()
             if idx is None:
                 idx = i
             elif i != idx:
                 raise ValueError("all CUDA tensors of a call must be on the same device")
     if idx is None:
         raise ValueError("the call has no CUDA tensor")
-    return torch.cuda.device(idx)
+    return _CURRENT if idx == torch.cuda.current_device() else torch.cuda.device(idx)
 
 
 def _dev(t: torch.Tensor, name: str) -> int:

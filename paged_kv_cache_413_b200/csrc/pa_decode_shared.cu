@@ -590,26 +590,33 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
 //                                                               B = Q^T from smem
 //   O^T[128 dims x 16 columns]   += V^T[128 dims x 128] . P^T   A = V^T from smem
 //                                                               (MN-major), B = P^T
-// One thread issues the 16 MMAs of a stage.  Four worker warps own one TMEM lane
-// quadrant each: thread t widens token t's K row (E4M3 -> f16, exact) into TMEM
-// and its V row into the f16 operand in shared memory, reads its row of S^T,
-// applies the masks (context length, and for a member's own tiles the other
-// members' columns), and writes its P row.  The softmax needs no reduction across
-// threads per stage: every column keeps one reference maximum shared by all
-// threads, moved (with a rescale of l and of O^T's column in TMEM) only when some
-// score passes it by more than 2^8, which a vote and a named barrier detect; each
-// thread sums its own l and the sums meet once, at the end.  P <= 2^8 is exact
-// enough in f16 (relative 2^-11); softmax and accumulation are fp32.  A producer
-// warp streams the raw E4M3 tiles (tiled TMA, 128-byte swizzle, no multicast)
-// into a ring of kStRing stages.  All waits are bounded; after a failure the
-// waits are skipped but every named barrier is still reached.
+// Warp roles (one TMEM lane quadrant each for the first two groups):
+//   * converter warps 4-7: thread t widens token t's E4M3 K row into a TMEM slot
+//     (f16 pairs, exact) and its V row into the f16 operand in shared memory;
+//   * softmax warps 0-3: thread t reads token t's row of S^T, applies the masks
+//     (context length; on a member's own tiles, the other members' columns) and
+//     writes its row of P^T;
+//   * warp 8 streams the raw tiles (tiled TMA, 128-byte swizzle, no multicast)
+//     into a ring of kStRing stages; warp 9 issues the 16 MMAs of each stage
+//     (S of stage st + 1 before P.V of stage st) and owns the TMEM allocation.
+// The converters work on stage st + 1 while the softmax warps work on stage st;
+// K slots, S buffers and P buffers are double-buffered.  The softmax needs no
+// reduction across threads per stage: every column keeps one reference maximum
+// shared by all threads, moved (with a rescale of l and of O^T's column) only
+// when some score passes it by more than 2^8, which a vote and a named barrier
+// detect; each thread sums its own l and the sums meet once, at the end.  P <= 2^8
+// is exact enough in f16 (relative 2^-11); softmax and accumulation are fp32.
+// Every mbarrier a waiter could otherwise see two phases ahead is split per
+// buffer, so no parity wait can alias.  All waits are bounded; after a failure
+// the waits are skipped but every named barrier is still reached.
 // ---------------------------------------------------------------------------
 constexpr int kStTokens = 128;                          // tokens per stage (M of S^T)
 constexpr int kStTiles = kStTokens / kBlockSize;        // pool tiles per stage
-constexpr int kStWorkers = 4;                           // worker warps, one per lane quadrant
-constexpr int kStProducerWarp = kStWorkers;
-constexpr int kStMmaWarp = kStWorkers + 1;
-constexpr int kStThreads = (kStWorkers + 2) * 32;
+constexpr int kStQuads = 4;                             // TMEM lane quadrants
+constexpr int kStConvWarp0 = kStQuads;                  // converters: warps 4..7
+constexpr int kStProducerWarp = 2 * kStQuads;
+constexpr int kStMmaWarp = 2 * kStQuads + 1;
+constexpr int kStThreads = (2 * kStQuads + 2) * 32;
 #ifndef PA_SHARED_TC_RING
 #define PA_SHARED_TC_RING 2
 #endif
@@ -619,18 +626,18 @@ constexpr int kStRawStage = 2 * kStTiles * kStRawTile;  // K tiles, then V tiles
 constexpr int kStVBytes = kStTokens * 128 * 2;          // V of a stage in f16: 32 KB
 constexpr int kStOpBytes = kSharedCols * 128 * 2;       // Q^T or P^T operand: 4 KB
 constexpr int kStOpHalf = kSharedCols * 128;            // one 64-element K half of it
-constexpr uint32_t kStTmemCols = 128;
-constexpr uint32_t kStTmemK = 0;   // K of the stage: 64 columns of f16 pairs (A operand)
-constexpr uint32_t kStTmemS = 64;  // S^T: 16 fp32 columns
-constexpr uint32_t kStTmemO = 80;  // O^T: 16 fp32 columns
+constexpr uint32_t kStTmemCols = 256;
+constexpr uint32_t kStTmemK = 0;     // K slots b = 0, 1: 64 columns of f16 pairs each
+constexpr uint32_t kStTmemS = 128;   // S^T buffers b = 0, 1: 16 fp32 columns each
+constexpr uint32_t kStTmemO = 160;   // O^T: 16 fp32 columns
 constexpr uint32_t kStIdescS = umma_idesc_f16(0, 0, kStTokens, kSharedCols);
 constexpr uint32_t kStIdescPV = umma_idesc_f16_ab(0, 1, 0, 128, kSharedCols);
 static_assert(kStTmemO + kSharedCols <= kStTmemCols, "TMEM budget");
 
 constexpr size_t shared_tc_smem_bytes() {
-  return 1024 + size_t(kStRing) * kStRawStage + kStVBytes + 2 * kStOpBytes +
-         (2 * kStRing + 5) * sizeof(uint64_t) +
-         (8 + 2 * kStWorkers * kSharedCols + kStWorkers * kSharedCols + kStWorkers) * 4 +
+  return 1024 + size_t(kStRing) * kStRawStage + kStVBytes + 3 * kStOpBytes +
+         (2 * kStRing + 11) * sizeof(uint64_t) +
+         (8 + 2 * kStQuads * kSharedCols + kStQuads * kSharedCols + kStQuads) * 4 +
          (2 * (kSharedCols + 1) + 2) * 4;
 }
 static_assert(2 * (shared_tc_smem_bytes() + 1024) <= 228 * 1024, "two CTAs per SM");
@@ -653,6 +660,24 @@ __device__ __forceinline__ void tmem_st16_f(uint32_t taddr, const float (&v)[16]
   tmem_st16(taddr, u);
 }
 
+// The token of row r (0..127) of stage st: its member (-1 = shared prefix; the
+// masked columns follow from it) and whether it lies inside that member's context.
+struct StRow {
+  int owner;
+  bool valid;
+};
+__device__ __forceinline__ StRow st_row(int st, int r, int pblk, int ntotal, int nseq,
+                                        const int* own_start, const int* own_len) {
+  const int T = st * kStTiles + (r >> 4);
+  StRow x{-1, T < ntotal};
+  if (x.valid && T >= pblk) {
+    x.owner = 0;
+    while (x.owner + 1 < nseq && own_start[x.owner + 1] <= T) ++x.owner;
+    x.valid = (pblk + (T - own_start[x.owner])) * kBlockSize + (r & 15) < own_len[x.owner];
+  }
+  return x;
+}
+
 template <typename QT>
 __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     const __grid_constant__ SharedParams sp) {
@@ -663,19 +688,21 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   uint8_t* raw = smem;                                  // [kStRing][K tiles, V tiles]
   uint8_t* vf = raw + kStRing * kStRawStage;            // V f16: [2 halves][128 rows][128 B]
   uint8_t* qop = vf + kStVBytes;                        // Q^T: [2 halves][16 rows][128 B]
-  uint8_t* pop = qop + kStOpBytes;                      // P^T: [2 halves][16 rows][128 B]
-  uint64_t* full = reinterpret_cast<uint64_t*>(pop + kStOpBytes);
+  uint8_t* pop = qop + kStOpBytes;                      // P^T buffers b = 0, 1, same layout
+  uint64_t* full = reinterpret_cast<uint64_t*>(pop + 2 * kStOpBytes);
   uint64_t* empty = full + kStRing;
-  uint64_t* kready = empty + kStRing;                   // K of stage st in TMEM (4 warps)
-  uint64_t* pready = kready + 1;                        // V and P of stage st in smem (4 warps)
-  uint64_t* sdone = pready + 1;                         // S^T of stage st written
-  uint64_t* odone = sdone + 1;                          // P.V of stage st done
-  uint64_t* done = odone + 1;                           // every MMA done
-  int* flags = reinterpret_cast<int*>(done + 1);        // [2][4] rescale votes
+  uint64_t* kready = empty + kStRing;                   // [2] K slot b of stage st written
+  uint64_t* sfull = kready + 2;                         // [2] S buffer b of stage st written
+  uint64_t* pready = sfull + 2;                         // [2] P buffer b written, O rescaled
+  uint64_t* odone = pready + 2;                         // [2] P.V of stage st (b = st & 1) done
+  uint64_t* vready = odone + 2;                         // V of stage st written
+  uint64_t* done = vready + 1;                          // every MMA done
+  uint64_t* qready = done + 1;                          // Q^T written (4 softmax warps)
+  int* flags = reinterpret_cast<int*>(qready + 1);      // [2][4] rescale votes
   float* wmax = reinterpret_cast<float*>(flags + 8);    // [2][4][16] warp column maxima
-  float* lsum = wmax + 2 * kStWorkers * kSharedCols;    // [4][16] warp column sums
-  float* qmax_w = lsum + kStWorkers * kSharedCols;      // [4]
-  int* own_start = reinterpret_cast<int*>(qmax_w + kStWorkers);  // [17] stream position
+  float* lsum = wmax + 2 * kStQuads * kSharedCols;      // [4][16] warp column sums
+  float* qmax_w = lsum + kStQuads * kSharedCols;        // [4]
+  int* own_start = reinterpret_cast<int*>(qmax_w + kStQuads);  // [17] stream positions
   int* own_len = own_start + kSharedCols + 1;           // [16] member lengths
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(own_len + kSharedCols + 1);
 
@@ -698,9 +725,9 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   const int ncols = nseq * G;
 
   // lengths and the shared prefix (device data: checked), as the mma.sync kernel
-  const int cap = p.cap;
-  int Lmin = cap, ntotal = 0;
   if (tid == 0) {
+    const int cap = p.cap;
+    int Lmin = cap;
     for (int j = 0; j < kSharedCols; ++j) {
       int L = j < nseq ? p.seq_lens[s0 + j] : 0;
       if (j < nseq && (L < 0 || L > cap)) {
@@ -715,22 +742,26 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       if (sub == 0 && kvh == 0) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
       P = P < 0 ? 0 : (min(P, Lmin) / p.block_size) * p.block_size;
     }
-    const int pblk = P / kBlockSize;
-    int pos = pblk;
+    const int pb = P / kBlockSize;
+    int pos = pb;
     for (int j = 0; j < kSharedCols; ++j) {
       own_start[j] = pos;
-      if (j < nseq) pos += (own_len[j] + kBlockSize - 1) / kBlockSize - pblk;
+      if (j < nseq) pos += (own_len[j] + kBlockSize - 1) / kBlockSize - pb;
     }
     own_start[kSharedCols] = pos;
-    for (int st = 0; st < kStRing; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&empty[st], kStWorkers);
+    for (int i = 0; i < kStRing; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kStQuads);
     }
-    mbar_init(kready, kStWorkers);
-    mbar_init(pready, kStWorkers);
-    mbar_init(sdone, 1);
-    mbar_init(odone, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&kready[b], kStQuads);
+      mbar_init(&sfull[b], 1);
+      mbar_init(&pready[b], kStQuads);
+      mbar_init(&odone[b], 1);
+    }
+    mbar_init(vready, kStQuads);
     mbar_init(done, 1);
+    mbar_init(qready, kStQuads);
     fence_barrier_init();
   }
   if (warp == kStMmaWarp) {  // the MMA warp owns the TMEM allocation
@@ -742,7 +773,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   tcgen05_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int pblk = own_start[0];
-  ntotal = own_start[kSharedCols];
+  const int ntotal = own_start[kSharedCols];
   const int nstages = (ntotal + kStTiles - 1) / kStTiles;
 
   if (warp == kStProducerWarp) {
@@ -789,10 +820,13 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
           const int n = min(kStTiles, ntotal - st * kStTiles);
           uint8_t* dst = raw + slot * kStRawStage;
           mbar_arrive_expect_tx(&full[slot], uint32_t(n) * 2 * kStRawTile);
-          for (int i = 0; i < n; ++i) {
-            tma_load_2d(dst + i * kStRawTile, &sp.tmk, 0, rows[i], &full[slot], policy);
-            tma_load_2d(dst + (kStTiles + i) * kStRawTile, &sp.tmv, 0, rows[i], &full[slot],
-                        policy);
+#pragma unroll
+          for (int i = 0; i < kStTiles; ++i) {
+            if (i < n) {
+              tma_load_2d(dst + i * kStRawTile, &sp.tmk, 0, rows[i], &full[slot], policy);
+              tma_load_2d(dst + (kStTiles + i) * kStRawTile, &sp.tmv, 0, rows[i], &full[slot],
+                          policy);
+            }
           }
           ++issued;
         }
@@ -806,120 +840,69 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     }
     __syncwarp();
   } else if (warp == kStMmaWarp) {
-    // ---------------- MMA issuer (one thread) ----------------
+    // ---------------- MMA issuer (one thread): S(st + 1), then P.V(st) ----------------
     if (lane == 0) {
       const uint64_t qdesc = umma_smem_desc(smem_u32(qop), 16, 1024, kUmmaSwizzle128B);
       const uint64_t pdesc = umma_smem_desc(smem_u32(pop), 16, 1024, kUmmaSwizzle128B);
       const uint64_t vdesc = umma_smem_desc(smem_u32(vf), kStVBytes / 2, 1024, kUmmaSwizzle128B);
       bool ok = true;
-      for (int st = 0; st < nstages && ok; ++st) {
-        if (!(ok = mbar_wait_bounded(kready, st & 1))) break;
+      auto issue_s = [&](int st) {  // S of stage st into S buffer st & 1, K from slot st & 1
+        const uint32_t b = uint32_t(st & 1);
+        if (!(ok = mbar_wait_bounded(&kready[b], (st >> 1) & 1))) return;
         tcgen05_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)  // 16 dims per step: K columns 8 ks.., Q^T k-step ks
-          umma_f16_ts(tmem + kStTmemS, tmem + kStTmemK + uint32_t(8 * ks),
+          umma_f16_ts(tmem + kStTmemS + 16 * b, tmem + kStTmemK + 64 * b + uint32_t(8 * ks),
                       qdesc + uint64_t(((ks >> 2) * kStOpHalf + (ks & 3) * 32) >> 4), kStIdescS,
                       ks > 0 ? 1u : 0u);
-        umma_commit(sdone);
-        if (!(ok = mbar_wait_bounded(pready, st & 1))) break;
+        umma_commit(&sfull[b]);
+      };
+      if (nstages > 0) {
+        ok = mbar_wait_bounded(qready, 0);
+        if (ok) issue_s(0);
+      }
+      for (int st = 0; st < nstages && ok; ++st) {
+        if (st + 1 < nstages) {
+          issue_s(st + 1);
+          if (!ok) break;
+        }
+        const uint32_t b = uint32_t(st & 1);
+        if (!(ok = mbar_wait_bounded(vready, st & 1))) break;
+        if (!(ok = mbar_wait_bounded(&pready[b], (st >> 1) & 1))) break;
         tcgen05_fence_after();
+        const uint64_t pd = pdesc + uint64_t((b * kStOpBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)  // 16 tokens per step
           umma_f16_ss(tmem + kStTmemO, vdesc + uint64_t((ks * 2048) >> 4),
-                      pdesc + uint64_t(((ks >> 2) * kStOpHalf + (ks & 3) * 32) >> 4), kStIdescPV,
+                      pd + uint64_t(((ks >> 2) * kStOpHalf + (ks & 3) * 32) >> 4), kStIdescPV,
                       (st > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(odone);
+        umma_commit(&odone[b]);
       }
       if (!ok) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
       umma_commit(done);  // fires once every MMA issued above has completed
       if (!mbar_wait_bounded(done, 0)) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
     }
     __syncwarp();
-  } else {
-    // ---------------- workers: thread = token row of S^T / dim row of O^T ----------------
-    const int r = tid;                                       // 0..127
-    const uint32_t tl = tmem + (uint32_t(32 * warp) << 16);  // this warp's lane quadrant
-    bool ok = true;  // warp-uniform; after a failure waits are skipped, barriers still met
+  } else if (warp >= kStConvWarp0) {
+    // ---------------- converters: token row r of each stage ----------------
+    const int q = warp - kStConvWarp0;
+    const int r = 32 * q + lane;
+    const uint32_t tl = tmem + (uint32_t(32 * q) << 16);  // this warp's lane quadrant
+    const int rr = r & 15, sw = rr & 7;                     // row in its tile, TMA swizzle
+    bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
     };
-    auto arrive = [&](uint64_t* bar) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar);
-    };
-    // ---- Q^T: thread t writes column n = t / 8, dims 16 (t % 8) .. + 15 (f16) ----
-    float mult = p.q_mult;
-    {
-      const int n = r >> 3, dc = r & 7;
-      const int j = n / G, hi = n - j * G;
-      const bool has = n < ncols;
-      uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
-      if (has) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            p.query + (int64_t(s0 + j) * p.num_heads + kvh * G + hi) * D * 2 + dc * 32);
-        w0 = src[0];
-        w1 = src[1];
-      }
-      uint32_t q[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      if constexpr (!std::is_same<QT, __half>::value) {
-        // bf16 -> f16 with one power of two for the CTA: its largest |q| lands in
-        // [2^14, 2^15); the score multiplier takes the inverse
-        float qm = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 a = unpack2(q[i], QT{});
-          qm = fmaxf(qm, fmaxf(fabsf(a.x), fabsf(a.y)));
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(kFullMask, qm, o));
-        if (lane == 0) qmax_w[warp] = qm;
-        named_bar_sync(1, kStWorkers * 32);
-        qm = fmaxf(fmaxf(qmax_w[0], qmax_w[1]), fmaxf(qmax_w[2], qmax_w[3]));
-        int e = 0;
-        if (qm > 0.f && isfinite(qm)) frexpf(qm, &e);
-        const int sq = min(max(15 - e, -100), 100);
-        mult = ldexpf(mult, -sq);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 a = unpack2(q[i], QT{});
-          q[i] = pack2(ldexpf(a.x, sq), ldexpf(a.y, sq), __half{});
-        }
-      }
-      // K-major, 128-byte swizzle: dim d of row n in half d / 64, 16-byte chunk
-      // (d % 64) / 8 stored at chunk ^ (n % 8)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int d0 = 16 * dc + 8 * c, h = d0 >> 6, ch = (d0 & 63) >> 3;
-        *reinterpret_cast<uint4*>(qop + h * kStOpHalf + n * 128 + ((ch ^ (n & 7)) << 4)) =
-            make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
-      }
-      fence_proxy_async_smem();  // the MMA reads it through the async proxy
-    }
-
-    float mref[kSharedCols], lacc[kSharedCols];
-#pragma unroll
-    for (int n = 0; n < kSharedCols; ++n) {
-      mref[n] = -INFINITY;
-      lacc[n] = 0.f;
-    }
-    const int rr = r & 15;             // row within its pool tile
-    const int sw = (rr & 7);           // the TMA's 128-byte swizzle of that row
     for (int st = 0; st < nstages; ++st) {
       const int slot = st % kStRing;
-      // this row's token: stream tile T, its member (-1: prefix) and validity
-      const int T = st * kStTiles + (r >> 4);
-      int owner = -1;
-      bool valid = T < ntotal;
-      if (valid && T >= pblk) {
-        owner = 0;
-        while (owner + 1 < nseq && own_start[owner + 1] <= T) ++owner;
-        valid = (pblk + (T - own_start[owner])) * kBlockSize + rr < own_len[owner];
-      }
-      const int lo = owner < 0 ? 0 : owner * G, hi = owner < 0 ? ncols : lo + G;
+      const StRow x = st_row(st, r, pblk, ntotal, nseq, own_start, own_len);
       wait(&full[slot], (st / kStRing) & 1);
       const uint8_t* rk = raw + slot * kStRawStage + (r >> 4) * kStRawTile + rr * 128;
       const uint8_t* rv = rk + kStTiles * kStRawTile;
-      // ---- K row -> TMEM (A operand), f16 pairs: column c holds dims 2c, 2c + 1 ----
+      // K row -> TMEM slot st & 1 (f16 pairs: column c holds dims 2c, 2c + 1), once
+      // S(st - 2) has read that slot
+      if (st >= 2) wait(&sfull[st & 1], ((st - 2) >> 1) & 1);
+      tcgen05_fence_after();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float kw[32];
@@ -935,17 +918,18 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
             kw[8 * c + 2 * i + 1] = __uint_as_float(b);
           }
         }
-        tmem_st32(tl + kStTmemK + 32 * h, kw);
+        tmem_st32(tl + kStTmemK + 64 * uint32_t(st & 1) + 32 * h, kw);
       }
       tmem_wait_st();
       tcgen05_fence_before();
-      arrive(kready);
-      // ---- V row -> f16 operand (MN-major, 128-byte swizzle), once P.V(st - 1) is done ----
-      if (st > 0) wait(odone, (st - 1) & 1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&kready[st & 1]);
+      // V row -> the f16 operand (MN-major, 128-byte swizzle), once P.V(st - 1) is done
+      if (st >= 1) wait(&odone[(st - 1) & 1], ((st - 1) >> 1) & 1);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (valid) w = *reinterpret_cast<const uint4*>(rv + ((c ^ sw) << 4));
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);  // rows past the context: zero, never NaN
+        if (x.valid) w = *reinterpret_cast<const uint4*>(rv + ((c ^ sw) << 4));
         uint32_t f[8];
         e4m3x4_to_f16x4(w.x, f[0], f[1]);
         e4m3x4_to_f16x4(w.y, f[2], f[3]);
@@ -958,33 +942,108 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
         *reinterpret_cast<uint4*>(vrow + (((c0 + 1) ^ (r & 7)) << 4)) =
             make_uint4(f[4], f[5], f[6], f[7]);
       }
-      arrive(&empty[slot]);  // the raw stage is read (K and V)
+      fence_proxy_async_smem();  // the MMA reads it through the async proxy
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(vready);
+        mbar_arrive(&empty[slot]);  // the raw stage is read (K and V)
+      }
+    }
+    if (!ok && lane == 0) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+  } else {
+    // ---------------- softmax warps: token row r of S^T, dim row r of O^T ----------------
+    const int r = tid;                                       // 0..127
+    const uint32_t tl = tmem + (uint32_t(32 * warp) << 16);  // this warp's lane quadrant
+    bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
+    };
+    // ---- Q^T: thread t writes column n = t / 8, dims 16 (t % 8) .. + 15 (f16) ----
+    float mult = p.q_mult;
+    {
+      const int n = r >> 3, dc = r & 7;
+      const int j = n / G, hi = n - j * G;
+      uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+      if (n < ncols) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.query + (int64_t(s0 + j) * p.num_heads + kvh * G + hi) * D * 2 + dc * 32);
+        w0 = src[0];
+        w1 = src[1];
+      }
+      uint32_t qw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      if constexpr (!std::is_same<QT, __half>::value) {
+        // bf16 -> f16 with one power of two for the CTA: its largest |q| lands in
+        // [2^14, 2^15); the score multiplier takes the inverse
+        float qm = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 a = unpack2(qw[i], QT{});
+          qm = fmaxf(qm, fmaxf(fabsf(a.x), fabsf(a.y)));
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(kFullMask, qm, o));
+        if (lane == 0) qmax_w[warp] = qm;
+        named_bar_sync(1, kStQuads * 32);
+        qm = fmaxf(fmaxf(qmax_w[0], qmax_w[1]), fmaxf(qmax_w[2], qmax_w[3]));
+        int e = 0;
+        if (qm > 0.f && isfinite(qm)) frexpf(qm, &e);
+        const int sq = min(max(15 - e, -100), 100);
+        mult = ldexpf(mult, -sq);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 a = unpack2(qw[i], QT{});
+          qw[i] = pack2(ldexpf(a.x, sq), ldexpf(a.y, sq), __half{});
+        }
+      }
+      // K-major, 128-byte swizzle: dim d of row n in half d / 64, 16-byte chunk
+      // (d % 64) / 8 stored at chunk ^ (n % 8)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int d0 = 16 * dc + 8 * c, h = d0 >> 6, ch = (d0 & 63) >> 3;
+        *reinterpret_cast<uint4*>(qop + h * kStOpHalf + n * 128 + ((ch ^ (n & 7)) << 4)) =
+            make_uint4(qw[4 * c], qw[4 * c + 1], qw[4 * c + 2], qw[4 * c + 3]);
+      }
+      fence_proxy_async_smem();  // the MMA reads it through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qready);
+    }
+
+    float mref[kSharedCols], lacc[kSharedCols];
+#pragma unroll
+    for (int n = 0; n < kSharedCols; ++n) {
+      mref[n] = -INFINITY;
+      lacc[n] = 0.f;
+    }
+    for (int st = 0; st < nstages; ++st) {
+      const uint32_t b = uint32_t(st & 1);
+      const StRow x = st_row(st, r, pblk, ntotal, nseq, own_start, own_len);
+      const int lo = x.owner < 0 ? 0 : x.owner * G, hi = x.owner < 0 ? ncols : lo + G;
       // ---- scores of this row, masked, in log2 units ----
-      wait(sdone, st & 1);
+      wait(&sfull[b], (st >> 1) & 1);
       tcgen05_fence_after();
-      float x[kSharedCols];
-      tmem_ld16(tl + kStTmemS, x);
+      float s[kSharedCols];
+      tmem_ld16(tl + kStTmemS + 16 * b, s);
       tmem_wait_ld();
       bool up = false;
 #pragma unroll
       for (int n = 0; n < kSharedCols; ++n) {
-        x[n] = (valid && n >= lo && n < hi) ? x[n] * mult : -INFINITY;
-        up |= x[n] > mref[n] + kSharedRescaleLog2;
+        s[n] = (x.valid && n >= lo && n < hi) ? s[n] * mult : -INFINITY;
+        up |= s[n] > mref[n] + kSharedRescaleLog2;
       }
       // ---- does any column's reference maximum move?  (vote, 128 threads) ----
-      const int fb = (st & 1) * kStWorkers;
+      const int fb = (st & 1) * kStQuads;
       const unsigned vote = __ballot_sync(kFullMask, up);
       if (lane == 0) flags[fb + warp] = vote != 0u;
-      named_bar_sync(1, kStWorkers * 32);
+      named_bar_sync(1, kStQuads * 32);
       if (flags[fb] | flags[fb + 1] | flags[fb + 2] | flags[fb + 3]) {  // uniform
 #pragma unroll
         for (int n = 0; n < kSharedCols; ++n) {
-          float m = x[n];
+          float m = s[n];
 #pragma unroll
           for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
           if (lane == 0) wmax[(fb + warp) * kSharedCols + n] = m;
         }
-        named_bar_sync(1, kStWorkers * 32);
+        named_bar_sync(1, kStQuads * 32);
         float alpha[kSharedCols];
         bool moved = false;
 #pragma unroll
@@ -998,7 +1057,9 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
           mref[n] = mn;
           lacc[n] *= alpha[n];
         }
-        if (st > 0 && moved) {  // O^T columns (this thread's dim row) follow
+        if (st > 0 && moved) {  // O^T columns (this thread's dim row), once P.V(st - 1) is done
+          wait(&odone[(st - 1) & 1], ((st - 1) >> 1) & 1);
+          tcgen05_fence_after();
           float o[kSharedCols];
           tmem_ld16(tl + kStTmemO, o);
           tmem_wait_ld();
@@ -1008,21 +1069,24 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
           tmem_wait_st();
         }
       }
-      // ---- P^T row: K-major, 128-byte swizzle (token r = k index) ----
-      uint8_t* prow = pop + (r >> 6) * kStOpHalf + 2 * (r & 7);
+      // ---- P^T row into buffer b (K-major, 128-byte swizzle; token r = k index),
+      // once P.V(st - 2) has read that buffer ----
+      if (st >= 2) wait(&odone[b], ((st - 2) >> 1) & 1);
+      uint8_t* prow = pop + b * kStOpBytes + (r >> 6) * kStOpHalf + 2 * (r & 7);
       const int pc = (r & 63) >> 3;
 #pragma unroll
       for (int n = 0; n < kSharedCols; ++n) {
-        const float pn = x[n] > -INFINITY ? ex2_approx_ftz(x[n] - mref[n]) : 0.f;
+        const float pn = s[n] > -INFINITY ? ex2_approx_ftz(s[n] - mref[n]) : 0.f;
         lacc[n] += pn;
         *reinterpret_cast<__half*>(prow + n * 128 + ((pc ^ (n & 7)) << 4)) = __float2half_rn(pn);
       }
       fence_proxy_async_smem();
       tcgen05_fence_before();
-      arrive(pready);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pready[b]);
     }
     // ---- epilogue: column sums over the CTA, O^T row of this dim, outputs ----
-    if (nstages > 0) wait(odone, (nstages - 1) & 1);
+    if (nstages > 0) wait(&odone[(nstages - 1) & 1], ((nstages - 1) >> 1) & 1);
     tcgen05_fence_after();
 #pragma unroll
     for (int n = 0; n < kSharedCols; ++n) {
@@ -1031,8 +1095,10 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(kFullMask, v, o);
       if (lane == 0) lsum[warp * kSharedCols + n] = v;
     }
-    named_bar_sync(1, kStWorkers * 32);
+    named_bar_sync(1, kStQuads * 32);
     float o[kSharedCols];
+#pragma unroll
+    for (int n = 0; n < kSharedCols; ++n) o[n] = 0.f;
     if (nstages > 0) {
       tmem_ld16(tl + kStTmemO, o);
       tmem_wait_ld();
@@ -1044,6 +1110,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       const int j = n / G, hh = n - j * G;
       store_out(p.out, (int64_t(s0 + j) * p.num_heads + kvh * G + hh) * D + r, v, p.out_dtype);
     }
+    if (!ok && lane == 0) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
   }
   tcgen05_fence_before();
   __syncthreads();
