@@ -585,71 +585,72 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
 // The same work unit as above (one CTA per group part and kv head, up to 16
 // columns = the kv head's query heads of up to 16 / G members), but the stream
 // of 16-token tiles -- the shared prefix first, then each member's own tiles --
-// is cut into stages of 128 tokens with the tokens on the M axis:
-//   S^T[128 tokens x 16 columns]  = K[128 x 128 dims] . Q^T     A = K from TMEM,
-//                                                               B = Q^T from smem
-//   O^T[128 dims x 16 columns]   += V^T[128 dims x 128] . P^T   A = V^T from smem
-//                                                               (MN-major), B = P^T
-// Warp roles (one TMEM lane quadrant each for the first two groups):
-//   * converter warps 4-7: thread t widens token t's E4M3 K row into a TMEM slot
-//     (f16 pairs, exact) and its V row into the f16 operand in shared memory;
-//   * softmax warps 0-3: thread t reads token t's row of S^T, applies the masks
-//     (context length; on a member's own tiles, the other members' columns) and
-//     writes its row of P^T;
-//   * warp 8 streams the raw tiles (tiled TMA, 128-byte swizzle, no multicast)
-//     into a ring of kStRing stages; warp 9 issues the 16 MMAs of each stage
-//     (S of stage st + 1 before P.V of stage st) and owns the TMEM allocation.
-// The converters work on stage st + 1 while the softmax warps work on stage st;
-// K slots, S buffers and P buffers are double-buffered.  The softmax needs no
-// reduction across threads per stage: every column keeps one reference maximum
-// shared by all threads, moved (with a rescale of l and of O^T's column) only
-// when some score passes it by more than 2^8, which a vote and a named barrier
-// detect; each thread sums its own l and the sums meet once, at the end.  P <= 2^8
-// is exact enough in f16 (relative 2^-11); softmax and accumulation are fp32.
+// is cut into stages of 128 tokens with the tokens on the M axis, and both
+// contractions run on E4M3 operands straight from the TMA-staged tiles:
+//   S^T[128 tokens x 16 columns]  = K[128 x 128 dims] . Q^T     kind::f8f6f4
+//   O^T[128 dims x 16 columns]   += V^T[128 dims x 128] . P^T   kind::f8f6f4
+// Nothing is widened.  Q is split per column into E4M3 terms instead: scaled by
+// a power of two so that its largest |q| lies in [128, 256), then
+// q' = t_0 + 2^-4 t_1 (+ 2^-8 t_2), each t the E4M3 rounding of what is left.
+// A bf16 value (8 significant bits) is exactly two such terms, an f16 value
+// (11) exactly three, so S^T = sum 2^-4k K.T_k^T is the product with the exact
+// query (each term's products are exact, accumulation is fp32).  P <= 2^8 (the
+// lazy reference maximum below) is split the same way into three terms, about
+// 12 significant bits, one more than the f16 P of the other kernels; O^T keeps
+// one fp32 accumulator per term.  Rows past the context are zeroed in the staged
+// V tile before P.V reads it.
+//   * softmax warps 0-3: thread t owns token t of a stage (its row of S^T) and
+//     dim t of O^T; every column keeps one reference maximum shared by all
+//     threads, moved (with a rescale of l and of O^T's columns) only when some
+//     score passes it by more than 2^8, which a vote and a named barrier detect;
+//     each thread sums its own l and the sums meet once, at the end;
+//   * warp 4 streams the raw tiles (tiled TMA, 128-byte swizzle, no multicast)
+//     into a ring of kStRing stages; warp 5 issues each stage's MMAs (S of stage
+//     st + 1 before P.V of stage st) and owns the TMEM allocation.
 // Every mbarrier a waiter could otherwise see two phases ahead is split per
-// buffer, so no parity wait can alias.  All waits are bounded; after a failure
-// the waits are skipped but every named barrier is still reached.
+// buffer.  All waits are bounded; after a failure the waits are skipped but every
+// named barrier is still reached.
 // ---------------------------------------------------------------------------
 constexpr int kStTokens = 128;                          // tokens per stage (M of S^T)
 constexpr int kStTiles = kStTokens / kBlockSize;        // pool tiles per stage
-constexpr int kStQuads = 4;                             // TMEM lane quadrants
-constexpr int kStConvWarp0 = kStQuads;                  // converters: warps 4..7
-constexpr int kStProducerWarp = 2 * kStQuads;
-constexpr int kStMmaWarp = 2 * kStQuads + 1;
-constexpr int kStThreads = (2 * kStQuads + 2) * 32;
+constexpr int kStQuads = 4;                             // softmax warps (TMEM lane quadrants)
+constexpr int kStProducerWarp = kStQuads;
+constexpr int kStMmaWarp = kStQuads + 1;
+constexpr int kStThreads = (kStQuads + 2) * 32;
 #ifndef PA_SHARED_TC_RING
-#define PA_SHARED_TC_RING 2
+#define PA_SHARED_TC_RING 3
 #endif
 constexpr int kStRing = PA_SHARED_TC_RING;              // raw stages in flight
 constexpr int kStRawTile = kBlockSize * 128;            // one E4M3 tile of K or V: 2 KB
 constexpr int kStRawStage = 2 * kStTiles * kStRawTile;  // K tiles, then V tiles: 32 KB
-constexpr int kStVBytes = kStTokens * 128 * 2;          // V of a stage in f16: 32 KB
-constexpr int kStOpBytes = kSharedCols * 128 * 2;       // Q^T or P^T operand: 4 KB
-constexpr int kStOpHalf = kSharedCols * 128;            // one 64-element K half of it
+constexpr int kStTerm = kSharedCols * 128;              // one E4M3 term of Q^T or P^T: 2 KB
+constexpr int kStPTerms = 3;                            // terms of P
 constexpr uint32_t kStTmemCols = 256;
-constexpr uint32_t kStTmemK = 0;     // K slots b = 0, 1: 64 columns of f16 pairs each
-constexpr uint32_t kStTmemS = 128;   // S^T buffers b = 0, 1: 16 fp32 columns each
-constexpr uint32_t kStTmemO = 160;   // O^T: 16 fp32 columns
+constexpr uint32_t kStTmemS = 0;    // S^T buffers b = 0, 1: [terms of Q][16] fp32 columns
+constexpr uint32_t kStTmemO = 128;  // O^T: [terms of P][16] fp32 columns
+// kind::f8f6f4, E4M3 x E4M3 (format code 0), fp32 accumulate; S: both K-major;
+// P.V: A = V^T and B = P^T both MN-major
 constexpr uint32_t kStIdescS = umma_idesc_f16(0, 0, kStTokens, kSharedCols);
-constexpr uint32_t kStIdescPV = umma_idesc_f16_ab(0, 1, 0, 128, kSharedCols);
-static_assert(kStTmemO + kSharedCols <= kStTmemCols, "TMEM budget");
+constexpr uint32_t kStIdescPV = umma_idesc_f16_ab(0, 1, 1, 128, kSharedCols);
 
+template <int NQ>
 constexpr size_t shared_tc_smem_bytes() {
-  return 1024 + size_t(kStRing) * kStRawStage + kStVBytes + 3 * kStOpBytes +
-         (2 * kStRing + 11) * sizeof(uint64_t) +
-         (8 + 2 * kStQuads * kSharedCols + kStQuads * kSharedCols + kStQuads) * 4 +
+  return 1024 + size_t(kStRing) * kStRawStage + size_t(NQ + kStPTerms) * kStTerm +
+         (kStRing * 2 + 8) * sizeof(uint64_t) +
+         (8 + 2 * kStQuads * kSharedCols + kStQuads * kSharedCols + kSharedCols) * 4 +
          (2 * (kSharedCols + 1) + 2) * 4;
 }
-static_assert(2 * (shared_tc_smem_bytes() + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(2 * (shared_tc_smem_bytes<3>() + 1024) <= 228 * 1024, "two CTAs per SM");
 
-// Four E4M3 bytes (byte 0 = element 0) to four f16: lo = elements 0, 1, hi = 2, 3.
-__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b16 a, b;\n\t"
-      "mov.b32 {a, b}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(w));
+// D[tmem] (+)= A[smem desc] * B[smem desc] with 8-bit (E4M3) operands.
+__device__ __forceinline__ void umma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // 16 32-bit words into this warp's 32 TMEM lanes, columns taddr .. taddr + 15.
@@ -658,6 +659,21 @@ __device__ __forceinline__ void tmem_st16_f(uint32_t taddr, const float (&v)[16]
 #pragma unroll
   for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
   tmem_st16(taddr, u);
+}
+
+// Split x0, x1 (|x| < 448) into `terms` E4M3 pairs: code k holds the E4M3 rounding
+// of what the codes before it leave, times 16^k.
+template <int terms>
+__device__ __forceinline__ void split_e4m3x2(float x0, float x1, uint16_t (&code)[terms]) {
+#pragma unroll
+  for (int k = 0; k < terms; ++k) {
+    code[k] = pack2_e4m3(x0, x1);
+    if (k + 1 < terms) {
+      const float2 back = unpack2_e4m3(code[k]);
+      x0 = (x0 - back.x) * 16.f;  // exact: the difference has at most the bits left
+      x1 = (x1 - back.y) * 16.f;
+    }
+  }
 }
 
 // The token of row r (0..127) of stage st: its member (-1 = shared prefix; the
@@ -682,27 +698,25 @@ template <typename QT>
 __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     const __grid_constant__ SharedParams sp) {
   constexpr int D = 128;
+  constexpr int NQ = std::is_same<QT, __half>::value ? 3 : 2;  // terms of Q
   const Params& p = sp.p;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* raw = smem;                                  // [kStRing][K tiles, V tiles]
-  uint8_t* vf = raw + kStRing * kStRawStage;            // V f16: [2 halves][128 rows][128 B]
-  uint8_t* qop = vf + kStVBytes;                        // Q^T: [2 halves][16 rows][128 B]
-  uint8_t* pop = qop + kStOpBytes;                      // P^T buffers b = 0, 1, same layout
-  uint64_t* full = reinterpret_cast<uint64_t*>(pop + 2 * kStOpBytes);
+  uint8_t* qop = raw + kStRing * kStRawStage;           // Q^T terms: [NQ][16 rows][128 B] SW128
+  uint8_t* pop = qop + NQ * kStTerm;                    // P^T terms: [3][128 tokens][16 B]
+  uint64_t* full = reinterpret_cast<uint64_t*>(pop + kStPTerms * kStTerm);
   uint64_t* empty = full + kStRing;
-  uint64_t* kready = empty + kStRing;                   // [2] K slot b of stage st written
-  uint64_t* sfull = kready + 2;                         // [2] S buffer b of stage st written
-  uint64_t* pready = sfull + 2;                         // [2] P buffer b written, O rescaled
-  uint64_t* odone = pready + 2;                         // [2] P.V of stage st (b = st & 1) done
-  uint64_t* vready = odone + 2;                         // V of stage st written
-  uint64_t* done = vready + 1;                          // every MMA done
-  uint64_t* qready = done + 1;                          // Q^T written (4 softmax warps)
-  int* flags = reinterpret_cast<int*>(qready + 1);      // [2][4] rescale votes
+  uint64_t* sfull = empty + kStRing;                    // [2] S buffer b of stage st written
+  uint64_t* pready = sfull + 2;                         // P of stage st written, O rescaled
+  uint64_t* odone = pready + 1;                         // P.V of stage st done
+  uint64_t* qready = odone + 1;                         // Q^T terms written
+  uint64_t* done = qready + 1;                          // every MMA done
+  int* flags = reinterpret_cast<int*>(done + 2);        // [2][4] rescale votes
   float* wmax = reinterpret_cast<float*>(flags + 8);    // [2][4][16] warp column maxima
   float* lsum = wmax + 2 * kStQuads * kSharedCols;      // [4][16] warp column sums
-  float* qmax_w = lsum + kStQuads * kSharedCols;        // [4]
-  int* own_start = reinterpret_cast<int*>(qmax_w + kStQuads);  // [17] stream positions
+  float* colmult = lsum + kStQuads * kSharedCols;       // [16] score multiplier per column
+  int* own_start = reinterpret_cast<int*>(colmult + kSharedCols);  // [17] stream positions
   int* own_len = own_start + kSharedCols + 1;           // [16] member lengths
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(own_len + kSharedCols + 1);
 
@@ -751,17 +765,14 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     own_start[kSharedCols] = pos;
     for (int i = 0; i < kStRing; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kStQuads);
+      mbar_init(&empty[i], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&kready[b], kStQuads);
-      mbar_init(&sfull[b], 1);
-      mbar_init(&pready[b], kStQuads);
-      mbar_init(&odone[b], 1);
-    }
-    mbar_init(vready, kStQuads);
-    mbar_init(done, 1);
+    mbar_init(&sfull[0], 1);
+    mbar_init(&sfull[1], 1);
+    mbar_init(pready, kStQuads);
+    mbar_init(odone, 1);
     mbar_init(qready, kStQuads);
+    mbar_init(done, 1);
     fence_barrier_init();
   }
   if (warp == kStMmaWarp) {  // the MMA warp owns the TMEM allocation
@@ -842,114 +853,69 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   } else if (warp == kStMmaWarp) {
     // ---------------- MMA issuer (one thread): S(st + 1), then P.V(st) ----------------
     if (lane == 0) {
+      // K tiles of a stage: [128 token rows][128 B], 128-byte swizzle (K-major A);
+      // V tiles: the same rows read as MN-major A (V^T); Q^T terms: [16][128 B]
+      // K-major B; P^T terms: [128 tokens][16 B], 8-token core matrices (MN-major B)
+      const uint64_t kdesc = umma_smem_desc(smem_u32(raw), 16, 1024, kUmmaSwizzle128B);
       const uint64_t qdesc = umma_smem_desc(smem_u32(qop), 16, 1024, kUmmaSwizzle128B);
-      const uint64_t pdesc = umma_smem_desc(smem_u32(pop), 16, 1024, kUmmaSwizzle128B);
-      const uint64_t vdesc = umma_smem_desc(smem_u32(vf), kStVBytes / 2, 1024, kUmmaSwizzle128B);
-      bool ok = true;
-      auto issue_s = [&](int st) {  // S of stage st into S buffer st & 1, K from slot st & 1
-        const uint32_t b = uint32_t(st & 1);
-        if (!(ok = mbar_wait_bounded(&kready[b], (st >> 1) & 1))) return;
-        tcgen05_fence_after();
+      const uint64_t pdesc = umma_smem_desc(smem_u32(pop), 128, 128, 0);
+      bool ok = mbar_wait_bounded(qready, 0);
+      // Polls the barriers and issues S(ns) as soon as its stage has landed and its
+      // S buffer is free (the P.V of stage ns - 2 is issued, so its softmax has read
+      // S(ns - 2)), and P.V(npv) as soon as P(npv) is written; sleeps otherwise.
+      int ns = 0, npv = 0, idle = 0;
+      unsigned long long t_idle = 0;
+      while (ok && npv < nstages) {
+        bool prog = false;
+        if (ns < nstages && ns <= npv + 1 &&
+            mbar_test(&full[ns % kStRing], (ns / kStRing) & 1)) {
+          tcgen05_fence_after();
+          const uint64_t kd = kdesc + uint64_t(((ns % kStRing) * kStRawStage) >> 4);
+          const uint32_t sb = tmem + kStTmemS + uint32_t(ns & 1) * (16 * 3);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)  // 16 dims per step: K columns 8 ks.., Q^T k-step ks
-          umma_f16_ts(tmem + kStTmemS + 16 * b, tmem + kStTmemK + 64 * b + uint32_t(8 * ks),
-                      qdesc + uint64_t(((ks >> 2) * kStOpHalf + (ks & 3) * 32) >> 4), kStIdescS,
-                      ks > 0 ? 1u : 0u);
-        umma_commit(&sfull[b]);
-      };
-      if (nstages > 0) {
-        ok = mbar_wait_bounded(qready, 0);
-        if (ok) issue_s(0);
-      }
-      for (int st = 0; st < nstages && ok; ++st) {
-        if (st + 1 < nstages) {
-          issue_s(st + 1);
-          if (!ok) break;
+          for (int t = 0; t < NQ; ++t)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // 32 dims per step
+              umma_f8_ss(sb + 16 * t, kd + uint64_t((ks * 32) >> 4),
+                         qdesc + uint64_t((t * kStTerm + ks * 32) >> 4), kStIdescS,
+                         ks > 0 ? 1u : 0u);
+          umma_commit(&sfull[ns & 1]);
+          ++ns;
+          prog = true;
         }
-        const uint32_t b = uint32_t(st & 1);
-        if (!(ok = mbar_wait_bounded(vready, st & 1))) break;
-        if (!(ok = mbar_wait_bounded(&pready[b], (st >> 1) & 1))) break;
-        tcgen05_fence_after();
-        const uint64_t pd = pdesc + uint64_t((b * kStOpBytes) >> 4);
+        if (npv < ns && mbar_test(pready, npv & 1)) {
+          tcgen05_fence_after();
+          const uint64_t vd = kdesc + uint64_t(((npv % kStRing) * kStRawStage +
+                                                kStTiles * kStRawTile) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)  // 16 tokens per step
-          umma_f16_ss(tmem + kStTmemO, vdesc + uint64_t((ks * 2048) >> 4),
-                      pd + uint64_t(((ks >> 2) * kStOpHalf + (ks & 3) * 32) >> 4), kStIdescPV,
-                      (st > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(&odone[b]);
+          for (int t = 0; t < kStPTerms; ++t)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // 32 tokens per step
+              umma_f8_ss(tmem + kStTmemO + 16 * t, vd + uint64_t((ks * 4096) >> 4),
+                         pdesc + uint64_t((t * kStTerm + ks * 512) >> 4), kStIdescPV,
+                         (npv > 0 || ks > 0) ? 1u : 0u);
+          umma_commit(odone);
+          umma_commit(&empty[npv % kStRing]);  // the raw stage is read (S and P.V)
+          ++npv;
+          prog = true;
+        }
+        if (prog) {
+          idle = 0;
+          continue;
+        }
+        // sleep on the barrier the next step most likely waits for
+        if (npv < ns)
+          mbar_try_wait(pready, npv & 1, 500);
+        else
+          mbar_try_wait(&full[ns % kStRing], (ns / kStRing) & 1, 500);
+        if (idle == 0) t_idle = global_timer_ns();
+        if ((++idle & 63) == 0 && global_timer_ns() - t_idle > kWaitLimitNs) ok = false;
       }
       if (!ok) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
       umma_commit(done);  // fires once every MMA issued above has completed
       if (!mbar_wait_bounded(done, 0)) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp >= kStConvWarp0) {
-    // ---------------- converters: token row r of each stage ----------------
-    const int q = warp - kStConvWarp0;
-    const int r = 32 * q + lane;
-    const uint32_t tl = tmem + (uint32_t(32 * q) << 16);  // this warp's lane quadrant
-    const int rr = r & 15, sw = rr & 7;                     // row in its tile, TMA swizzle
-    bool ok = true;
-    auto wait = [&](uint64_t* bar, uint32_t parity) {
-      if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
-    };
-    for (int st = 0; st < nstages; ++st) {
-      const int slot = st % kStRing;
-      const StRow x = st_row(st, r, pblk, ntotal, nseq, own_start, own_len);
-      wait(&full[slot], (st / kStRing) & 1);
-      const uint8_t* rk = raw + slot * kStRawStage + (r >> 4) * kStRawTile + rr * 128;
-      const uint8_t* rv = rk + kStTiles * kStRawTile;
-      // K row -> TMEM slot st & 1 (f16 pairs: column c holds dims 2c, 2c + 1), once
-      // S(st - 2) has read that slot
-      if (st >= 2) wait(&sfull[st & 1], ((st - 2) >> 1) & 1);
-      tcgen05_fence_after();
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float kw[32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(rk + (((4 * h + c) ^ sw) << 4));
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t a, b;
-            e4m3x4_to_f16x4(ww[i], a, b);
-            kw[8 * c + 2 * i] = __uint_as_float(a);
-            kw[8 * c + 2 * i + 1] = __uint_as_float(b);
-          }
-        }
-        tmem_st32(tl + kStTmemK + 64 * uint32_t(st & 1) + 32 * h, kw);
-      }
-      tmem_wait_st();
-      tcgen05_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&kready[st & 1]);
-      // V row -> the f16 operand (MN-major, 128-byte swizzle), once P.V(st - 1) is done
-      if (st >= 1) wait(&odone[(st - 1) & 1], ((st - 1) >> 1) & 1);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);  // rows past the context: zero, never NaN
-        if (x.valid) w = *reinterpret_cast<const uint4*>(rv + ((c ^ sw) << 4));
-        uint32_t f[8];
-        e4m3x4_to_f16x4(w.x, f[0], f[1]);
-        e4m3x4_to_f16x4(w.y, f[2], f[3]);
-        e4m3x4_to_f16x4(w.z, f[4], f[5]);
-        e4m3x4_to_f16x4(w.w, f[6], f[7]);
-        // dims 16c .. 16c + 15: chunks 2c and 2c + 1 of the row, half c / 4
-        uint8_t* vrow = vf + (c >> 2) * (kStVBytes / 2) + r * 128;
-        const int c0 = (2 * c) & 7;
-        *reinterpret_cast<uint4*>(vrow + ((c0 ^ (r & 7)) << 4)) = make_uint4(f[0], f[1], f[2], f[3]);
-        *reinterpret_cast<uint4*>(vrow + (((c0 + 1) ^ (r & 7)) << 4)) =
-            make_uint4(f[4], f[5], f[6], f[7]);
-      }
-      fence_proxy_async_smem();  // the MMA reads it through the async proxy
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(vready);
-        mbar_arrive(&empty[slot]);  // the raw stage is read (K and V)
-      }
-    }
-    if (!ok && lane == 0) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
   } else {
     // ---------------- softmax warps: token row r of S^T, dim row r of O^T ----------------
     const int r = tid;                                       // 0..127
@@ -958,8 +924,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
     };
-    // ---- Q^T: thread t writes column n = t / 8, dims 16 (t % 8) .. + 15 (f16) ----
-    float mult = p.q_mult;
+    // ---- Q^T terms: thread t takes column n = t / 8, dims 16 (t % 8) .. + 15 ----
     {
       const int n = r >> 3, dc = r & 7;
       const int j = n / G, hi = n - j * G;
@@ -970,43 +935,49 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
         w0 = src[0];
         w1 = src[1];
       }
-      uint32_t qw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      if constexpr (!std::is_same<QT, __half>::value) {
-        // bf16 -> f16 with one power of two for the CTA: its largest |q| lands in
-        // [2^14, 2^15); the score multiplier takes the inverse
-        float qm = 0.f;
+      const uint32_t qw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      float qf[16];
+      float qm = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 a = unpack2(qw[i], QT{});
-          qm = fmaxf(qm, fmaxf(fabsf(a.x), fabsf(a.y)));
-        }
+      for (int i = 0; i < 8; ++i) {
+        const float2 a = unpack2(qw[i], QT{});
+        qf[2 * i] = a.x;
+        qf[2 * i + 1] = a.y;
+        qm = fmaxf(qm, fmaxf(fabsf(a.x), fabsf(a.y)));
+      }
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(kFullMask, qm, o));
-        if (lane == 0) qmax_w[warp] = qm;
-        named_bar_sync(1, kStQuads * 32);
-        qm = fmaxf(fmaxf(qmax_w[0], qmax_w[1]), fmaxf(qmax_w[2], qmax_w[3]));
-        int e = 0;
-        if (qm > 0.f && isfinite(qm)) frexpf(qm, &e);
-        const int sq = min(max(15 - e, -100), 100);
-        mult = ldexpf(mult, -sq);
+      for (int o = 4; o >= 1; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(kFullMask, qm, o));
+      // the column's largest |q| goes to [128, 256): a power of two, exact
+      int e = 0;
+      if (qm > 0.f && isfinite(qm)) frexpf(qm, &e);
+      const int sa = min(max(8 - e, -120), 120);
+      if (dc == 0) colmult[n] = ldexpf(p.q_mult, -sa);
+      uint32_t tw[NQ][4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 a = unpack2(qw[i], QT{});
-          qw[i] = pack2(ldexpf(a.x, sq), ldexpf(a.y, sq), __half{});
+      for (int i = 0; i < 8; ++i) {
+        uint16_t code[NQ];
+        split_e4m3x2<NQ>(ldexpf(qf[2 * i], sa), ldexpf(qf[2 * i + 1], sa), code);
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) {
+          if (i & 1)
+            tw[t][i >> 1] |= uint32_t(code[t]) << 16;
+          else
+            tw[t][i >> 1] = code[t];
         }
       }
-      // K-major, 128-byte swizzle: dim d of row n in half d / 64, 16-byte chunk
-      // (d % 64) / 8 stored at chunk ^ (n % 8)
+      // K-major, 128-byte swizzle: the 16 dims of chunk dc of row n at chunk dc ^ (n % 8)
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int d0 = 16 * dc + 8 * c, h = d0 >> 6, ch = (d0 & 63) >> 3;
-        *reinterpret_cast<uint4*>(qop + h * kStOpHalf + n * 128 + ((ch ^ (n & 7)) << 4)) =
-            make_uint4(qw[4 * c], qw[4 * c + 1], qw[4 * c + 2], qw[4 * c + 3]);
-      }
-      fence_proxy_async_smem();  // the MMA reads it through the async proxy
+      for (int t = 0; t < NQ; ++t)
+        *reinterpret_cast<uint4*>(qop + t * kStTerm + n * 128 + ((dc ^ (n & 7)) << 4)) =
+            make_uint4(tw[t][0], tw[t][1], tw[t][2], tw[t][3]);
+      fence_proxy_async_smem();  // the MMA reads them through the async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(qready);
+      named_bar_sync(1, kStQuads * 32);  // colmult written
     }
+    float cmul[kSharedCols];
+#pragma unroll
+    for (int n = 0; n < kSharedCols; ++n) cmul[n] = colmult[n];
 
     float mref[kSharedCols], lacc[kSharedCols];
 #pragma unroll
@@ -1018,27 +989,40 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       const uint32_t b = uint32_t(st & 1);
       const StRow x = st_row(st, r, pblk, ntotal, nseq, own_start, own_len);
       const int lo = x.owner < 0 ? 0 : x.owner * G, hi = x.owner < 0 ? ncols : lo + G;
-      // ---- scores of this row, masked, in log2 units ----
+      // ---- scores of this row: the Q terms' products combined, masked, log2 units ----
       wait(&sfull[b], (st >> 1) & 1);
       tcgen05_fence_after();
-      float s[kSharedCols];
-      tmem_ld16(tl + kStTmemS + 16 * b, s);
-      tmem_wait_ld();
+      float sc[kSharedCols];
+      {
+        float st_[NQ][kSharedCols];
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) tmem_ld16(tl + kStTmemS + b * (16 * 3) + 16 * t, st_[t]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int n = 0; n < kSharedCols; ++n) {
+          float v = st_[NQ - 1][n];
+#pragma unroll
+          for (int t = NQ - 2; t >= 0; --t) v = fmaf(v, 0.0625f, st_[t][n]);
+          sc[n] = v;
+        }
+      }
       bool up = false;
 #pragma unroll
       for (int n = 0; n < kSharedCols; ++n) {
-        s[n] = (x.valid && n >= lo && n < hi) ? s[n] * mult : -INFINITY;
-        up |= s[n] > mref[n] + kSharedRescaleLog2;
+        sc[n] = (x.valid && n >= lo && n < hi) ? sc[n] * cmul[n] : -INFINITY;
+        up |= sc[n] > mref[n] + kSharedRescaleLog2;
       }
       // ---- does any column's reference maximum move?  (vote, 128 threads) ----
       const int fb = (st & 1) * kStQuads;
       const unsigned vote = __ballot_sync(kFullMask, up);
       if (lane == 0) flags[fb + warp] = vote != 0u;
       named_bar_sync(1, kStQuads * 32);
+      // P.V(st - 1) must be done before O^T is rescaled or the P^T buffer rewritten
+      if (st >= 1) wait(odone, (st - 1) & 1);
       if (flags[fb] | flags[fb + 1] | flags[fb + 2] | flags[fb + 3]) {  // uniform
 #pragma unroll
         for (int n = 0; n < kSharedCols; ++n) {
-          float m = s[n];
+          float m = sc[n];
 #pragma unroll
           for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
           if (lane == 0) wmax[(fb + warp) * kSharedCols + n] = m;
@@ -1057,36 +1041,56 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
           mref[n] = mn;
           lacc[n] *= alpha[n];
         }
-        if (st > 0 && moved) {  // O^T columns (this thread's dim row), once P.V(st - 1) is done
-          wait(&odone[(st - 1) & 1], ((st - 1) >> 1) & 1);
+        if (st > 0 && moved) {  // O^T columns of this thread's dim row, every P term
           tcgen05_fence_after();
-          float o[kSharedCols];
-          tmem_ld16(tl + kStTmemO, o);
-          tmem_wait_ld();
 #pragma unroll
-          for (int n = 0; n < kSharedCols; ++n) o[n] *= alpha[n];
-          tmem_st16_f(tl + kStTmemO, o);
+          for (int t = 0; t < kStPTerms; ++t) {
+            float o[kSharedCols];
+            tmem_ld16(tl + kStTmemO + 16 * t, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int n = 0; n < kSharedCols; ++n) o[n] *= alpha[n];
+            tmem_st16_f(tl + kStTmemO + 16 * t, o);
+          }
           tmem_wait_st();
         }
       }
-      // ---- P^T row into buffer b (K-major, 128-byte swizzle; token r = k index),
-      // once P.V(st - 2) has read that buffer ----
-      if (st >= 2) wait(&odone[b], ((st - 2) >> 1) & 1);
-      uint8_t* prow = pop + b * kStOpBytes + (r >> 6) * kStOpHalf + 2 * (r & 7);
-      const int pc = (r & 63) >> 3;
+      // ---- P^T row: three E4M3 terms of 16 bytes, token r of each ----
+      uint32_t pw[kStPTerms][4];
 #pragma unroll
-      for (int n = 0; n < kSharedCols; ++n) {
-        const float pn = s[n] > -INFINITY ? ex2_approx_ftz(s[n] - mref[n]) : 0.f;
-        lacc[n] += pn;
-        *reinterpret_cast<__half*>(prow + n * 128 + ((pc ^ (n & 7)) << 4)) = __float2half_rn(pn);
+      for (int i = 0; i < 8; ++i) {
+        const int n0 = 2 * i, n1 = 2 * i + 1;
+        const float p0 = sc[n0] > -INFINITY ? ex2_approx_ftz(sc[n0] - mref[n0]) : 0.f;
+        const float p1 = sc[n1] > -INFINITY ? ex2_approx_ftz(sc[n1] - mref[n1]) : 0.f;
+        lacc[n0] += p0;
+        lacc[n1] += p1;
+        uint16_t code[kStPTerms];
+        split_e4m3x2<kStPTerms>(p0, p1, code);
+#pragma unroll
+        for (int t = 0; t < kStPTerms; ++t) {
+          if (i & 1)
+            pw[t][i >> 1] |= uint32_t(code[t]) << 16;
+          else
+            pw[t][i >> 1] = code[t];
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kStPTerms; ++t)
+        *reinterpret_cast<uint4*>(pop + t * kStTerm + r * 16) =
+            make_uint4(pw[t][0], pw[t][1], pw[t][2], pw[t][3]);
+      if (!x.valid) {  // V rows past the context may hold anything, even NaN: zero them
+        uint8_t* vrow = raw + (st % kStRing) * kStRawStage + (kStTiles + (r >> 4)) * kStRawTile +
+                        (r & 15) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();
       tcgen05_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&pready[b]);
+      if (lane == 0) mbar_arrive(pready);
     }
     // ---- epilogue: column sums over the CTA, O^T row of this dim, outputs ----
-    if (nstages > 0) wait(&odone[(nstages - 1) & 1], ((nstages - 1) >> 1) & 1);
+    if (nstages > 0) wait(odone, (nstages - 1) & 1);
     tcgen05_fence_after();
 #pragma unroll
     for (int n = 0; n < kSharedCols; ++n) {
@@ -1100,8 +1104,13 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
 #pragma unroll
     for (int n = 0; n < kSharedCols; ++n) o[n] = 0.f;
     if (nstages > 0) {
-      tmem_ld16(tl + kStTmemO, o);
+      float ot[kStPTerms][kSharedCols];
+#pragma unroll
+      for (int t = 0; t < kStPTerms; ++t) tmem_ld16(tl + kStTmemO + 16 * t, ot[t]);
       tmem_wait_ld();
+#pragma unroll
+      for (int n = 0; n < kSharedCols; ++n)
+        o[n] = fmaf(fmaf(ot[2][n], 0.0625f, ot[1][n]), 0.0625f, ot[0][n]);
     }
     for (int n = 0; n < ncols; ++n) {
       const float L = lsum[n] + lsum[kSharedCols + n] + lsum[2 * kSharedCols + n] +
@@ -1199,13 +1208,14 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
     return PA_ERR_CUDA;
   if (fp8) {  // the tensor-core kernel: no cluster split
     sp.cluster = 1;
-    constexpr size_t smem = shared_tc_smem_bytes();
     const dim3 grid(unsigned(grid_x), unsigned(a.num_kv_heads));
     if (a.q_dtype == PA_F16) {
+      constexpr size_t smem = shared_tc_smem_bytes<3>();
       static std::atomic<unsigned long long> done_h{0};
       if (set_smem_once(decode_shared_tc_kernel<__half>, smem, done_h) != PA_OK) return PA_ERR_CUDA;
       decode_shared_tc_kernel<__half><<<grid, kStThreads, smem, stream>>>(sp);
     } else if (a.q_dtype == PA_BF16) {
+      constexpr size_t smem = shared_tc_smem_bytes<2>();
       static std::atomic<unsigned long long> done_b{0};
       if (set_smem_once(decode_shared_tc_kernel<__nv_bfloat16>, smem, done_b) != PA_OK)
         return PA_ERR_CUDA;
