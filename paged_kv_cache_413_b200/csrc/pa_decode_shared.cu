@@ -805,10 +805,13 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
           }
           const int e = lt / p.tiles_per_block;
           int32_t phys = p.block_tables[int64_t(s0 + j) * p.max_blocks_per_seq + e];
-          if (T < pblk) {  // the promise: every member has these blocks
-            for (int jj = 1; jj < nseq; ++jj)
-              if (p.block_tables[int64_t(s0 + jj) * p.max_blocks_per_seq + e] != phys)
-                atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+          if (T < pblk) {  // the promise: every member has these blocks (loads issued together)
+            bool same = true;
+#pragma unroll
+            for (int jj = 1; jj < kSharedCols; ++jj)
+              if (jj < nseq)
+                same &= p.block_tables[int64_t(s0 + jj) * p.max_blocks_per_seq + e] == phys;
+            if (!same) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
           }
           if (phys < 0 || phys >= p.num_blocks) {
             atomicOr(&g_shared_err, PA_DEVERR_BLOCK_RANGE);
@@ -1018,7 +1021,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       if (lane == 0) flags[fb + warp] = vote != 0u;
       named_bar_sync(1, kStQuads * 32);
       // P.V(st - 1) must be done before O^T is rescaled or the P^T buffer rewritten
-      if (st >= 1) wait(odone, (st - 1) & 1);
+      bool pv_done = st == 0;
       if (flags[fb] | flags[fb + 1] | flags[fb + 2] | flags[fb + 3]) {  // uniform
 #pragma unroll
         for (int n = 0; n < kSharedCols; ++n) {
@@ -1042,6 +1045,8 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
           lacc[n] *= alpha[n];
         }
         if (st > 0 && moved) {  // O^T columns of this thread's dim row, every P term
+          wait(odone, (st - 1) & 1);
+          pv_done = true;
           tcgen05_fence_after();
 #pragma unroll
           for (int t = 0; t < kStPTerms; ++t) {
@@ -1074,6 +1079,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
             pw[t][i >> 1] = code[t];
         }
       }
+      if (!pv_done) wait(odone, (st - 1) & 1);
 #pragma unroll
       for (int t = 0; t < kStPTerms; ++t)
         *reinterpret_cast<uint4*>(pop + t * kStTerm + r * 16) =
@@ -1100,6 +1106,19 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       if (lane == 0) lsum[warp * kSharedCols + n] = v;
     }
     named_bar_sync(1, kStQuads * 32);
+    // per column, once: 1 / l (v_scale folded in) and the output row; the vote
+    // arrays are free now
+    float* einv = wmax;
+    int64_t* ebase = reinterpret_cast<int64_t*>(wmax + 2 * kSharedCols);
+    if (tid < kSharedCols) {
+      const int n = tid;
+      const float L = lsum[n] + lsum[kSharedCols + n] + lsum[2 * kSharedCols + n] +
+                      lsum[3 * kSharedCols + n];
+      einv[n] = L > 0.f ? p.v_mult / L : 0.f;  // an empty context gives zeros
+      const int j = n / G, hh = n - j * G;
+      ebase[n] = n < ncols ? (int64_t(s0 + j) * p.num_heads + kvh * G + hh) * D : -1;
+    }
+    named_bar_sync(1, kStQuads * 32);
     float o[kSharedCols];
 #pragma unroll
     for (int n = 0; n < kSharedCols; ++n) o[n] = 0.f;
@@ -1112,12 +1131,10 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       for (int n = 0; n < kSharedCols; ++n)
         o[n] = fmaf(fmaf(ot[2][n], 0.0625f, ot[1][n]), 0.0625f, ot[0][n]);
     }
-    for (int n = 0; n < ncols; ++n) {
-      const float L = lsum[n] + lsum[kSharedCols + n] + lsum[2 * kSharedCols + n] +
-                      lsum[3 * kSharedCols + n];
-      const float v = L > 0.f ? o[n] * (p.v_mult / L) : 0.f;  // an empty context gives zeros
-      const int j = n / G, hh = n - j * G;
-      store_out(p.out, (int64_t(s0 + j) * p.num_heads + kvh * G + hh) * D + r, v, p.out_dtype);
+#pragma unroll
+    for (int n = 0; n < kSharedCols; ++n) {
+      const int64_t base = ebase[n];
+      if (base >= 0) store_out(p.out, base + r, o[n] * einv[n], p.out_dtype);
     }
     if (!ok && lane == 0) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
   }
