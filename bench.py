@@ -437,7 +437,8 @@ def timed_loop(step, launches, steps, warmup, dev, stream, world, rank):
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error bits set during the timed steps")
     elapsed_ms = t0.elapsed_time(t1)
-    launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in launches)
+    pairs = {id(e0): (e0, e1) for e0, e1 in launches}  # a pair replayed twice: its last
+    launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in pairs.values())
     elapsed_ms, launch_ms = max_over_ranks([elapsed_ms, launch_ms], world, dev)
     return elapsed_ms, launch_ms, (sampler.summary() if sampler else None)
 
@@ -446,37 +447,52 @@ def timing_note(args) -> str:
     if args.no_graphs:
         return "each timed step calls the library from Python (host launch overhead included)"
     return ("each timed step replays two CUDA graphs of the library's calls (cache writes, then "
-            "the hot kernels); CUDA events on the stream bracket the hot graph")
+            "the hot kernels); the step time brackets both with CUDA events on the stream, the "
+            "launch time brackets the hot kernels with event record nodes inside the graph "
+            "(graph launch latency excluded)")
+
+
+MAX_HOT_GRAPHS = 200
 
 
 def graph_step(writes, hot, run_step, inputs, out, ev, dev, stream, args):
     """The step the timed loop runs.  By default each step replays two CUDA graphs
     captured from the same library calls -- the cache writes (and copies), then the
-    hot kernel(s) -- with the hot launch's events recorded between them on the
-    stream, so host-side call overhead never idles the GPU inside the timed region.
-    With --no-graphs the step calls the library directly (run_step)."""
+    hot kernel(s) -- so host-side call overhead never idles the GPU inside the timed
+    region.  Each hot graph holds its own pair of timing events, recorded as event
+    nodes around the hot kernels, so a launch's time is the kernels' and not the
+    graph launch's; one hot graph per timed step (up to MAX_HOT_GRAPHS, replayed in
+    turn) keeps every timed step's pair apart.  With --no-graphs the step calls the
+    library directly (run_step)."""
     if args.no_graphs:
         return lambda timed: run_step(inputs, out, timed)
     run_step(inputs, out, False)          # warm: every kernel attribute set, maps encoded
     torch.cuda.synchronize(dev)
-    gw, gh = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
+    gw = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gw, stream=side):
         writes()
-    with torch.cuda.graph(gh, stream=side):
-        hot()
+    hots = []
+    for _ in range(max(1, min(args.steps, MAX_HOT_GRAPHS))):
+        g = torch.cuda.CUDAGraph()
+        e0 = torch.cuda.Event(enable_timing=True, external=True)
+        e1 = torch.cuda.Event(enable_timing=True, external=True)
+        with torch.cuda.graph(g, stream=side):
+            e0.record(side)
+            hot()
+            e1.record(side)
+        hots.append((g, e0, e1))
     stream.wait_stream(side)
     torch.cuda.synchronize(dev)
+    count = [0]
 
     def step(timed):
+        g, e0, e1 = hots[count[0] % len(hots)]
+        count[0] += 1
         gw.replay()
+        g.replay()
         if timed:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        gh.replay()
-        if timed:
-            e1.record(stream)
             ev.append((e0, e1))
 
     return step

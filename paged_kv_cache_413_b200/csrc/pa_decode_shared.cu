@@ -630,8 +630,7 @@ constexpr uint32_t kStTmemS = 0;    // S^T buffers b = 0, 1: [terms of Q][16] fp
 constexpr uint32_t kStTmemO = 128;  // O^T: [terms of P][16] fp32 columns
 // kind::f8f6f4, E4M3 x E4M3 (format code 0), fp32 accumulate; S: both K-major;
 // P.V: A = V^T and B = P^T both MN-major
-constexpr uint32_t kStIdescS = umma_idesc_f16(0, 0, kStTokens, kSharedCols);
-constexpr uint32_t kStIdescPV = umma_idesc_f16_ab(0, 1, 1, 128, kSharedCols);
+constexpr uint32_t kStIdescPV = umma_idesc_f16_ab(0, 1, 1, 128, kSharedCols * kStPTerms);
 
 template <int NQ>
 constexpr size_t shared_tc_smem_bytes() {
@@ -792,34 +791,52 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     const uint64_t policy = l2_policy_evict_first();
     int issued = 0, ent = -1;
     bool ok = true;
-    for (int st = 0; st < nstages && ok; ++st) {
-      // one table read per lane covers 4 stages: lane l takes stream tile 8 st + l
-      if ((st & 3) == 0) {
-        const int T = st * kStTiles + lane;
-        ent = -1;
-        if (T < ntotal) {
-          int j = 0, lt = T;  // member whose table holds the tile, logical tile there
-          if (T >= pblk) {
-            while (j + 1 < nseq && own_start[j + 1] <= T) ++j;
-            lt = pblk + (T - own_start[j]);
-          }
-          const int e = lt / p.tiles_per_block;
-          int32_t phys = p.block_tables[int64_t(s0 + j) * p.max_blocks_per_seq + e];
-          if (T < pblk) {  // the promise: every member has these blocks (loads issued together)
-            bool same = true;
+    // Lane l takes stream tile 32 g + l of each group g of 4 stages.  The block-table
+    // entries of group g + 1 are read while group g streams and are checked (the
+    // prefix promise, the block range) when their group starts, so no table read
+    // sits between a freed ring slot and its next load.
+    int32_t nx[kSharedCols];  // the fetched tile's entry in each member's table (prefix)
+    int nx_T = 0, nx_lt = 0;  // or in its owner's (nx[0]); its logical tile there
+    auto fetch = [&](int T) {
+      nx_T = T;
+      if (T >= ntotal) return;
+      int j = 0, lt = T;  // member whose table holds the tile, logical tile there
+      if (T >= pblk) {
+        while (j + 1 < nseq && own_start[j + 1] <= T) ++j;
+        lt = pblk + (T - own_start[j]);
+      }
+      nx_lt = lt;
+      const int e = lt / p.tiles_per_block;
+      nx[0] = p.block_tables[int64_t(s0 + j) * p.max_blocks_per_seq + e];
+      if (T < pblk) {
 #pragma unroll
-            for (int jj = 1; jj < kSharedCols; ++jj)
-              if (jj < nseq)
-                same &= p.block_tables[int64_t(s0 + jj) * p.max_blocks_per_seq + e] == phys;
-            if (!same) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
-          }
-          if (phys < 0 || phys >= p.num_blocks) {
-            atomicOr(&g_shared_err, PA_DEVERR_BLOCK_RANGE);
-            phys = 0;
-          }
-          ent = ((phys * p.num_kv_heads + kvh) * p.tiles_per_block + (lt - e * p.tiles_per_block)) *
-                kBlockSize;
-        }
+        for (int jj = 1; jj < kSharedCols; ++jj)
+          if (jj < nseq) nx[jj] = p.block_tables[int64_t(s0 + jj) * p.max_blocks_per_seq + e];
+      }
+    };
+    auto resolve = [&]() -> int {  // pool row of the fetched tile, -1 past the stream
+      if (nx_T >= ntotal) return -1;
+      int32_t phys = nx[0];
+      if (nx_T < pblk) {  // the promise: every member has these blocks
+        bool same = true;
+#pragma unroll
+        for (int jj = 1; jj < kSharedCols; ++jj)
+          if (jj < nseq) same &= nx[jj] == phys;
+        if (!same) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+      }
+      if (phys < 0 || phys >= p.num_blocks) {
+        atomicOr(&g_shared_err, PA_DEVERR_BLOCK_RANGE);
+        phys = 0;
+      }
+      const int e = nx_lt / p.tiles_per_block;
+      return ((phys * p.num_kv_heads + kvh) * p.tiles_per_block + (nx_lt - e * p.tiles_per_block)) *
+             kBlockSize;
+    };
+    fetch(lane);
+    for (int st = 0; st < nstages && ok; ++st) {
+      if ((st & 3) == 0) {
+        ent = resolve();
+        fetch((st + 4) * kStTiles + lane);
       }
       int rows[kStTiles];
 #pragma unroll
@@ -857,11 +874,16 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     // ---------------- MMA issuer (one thread): S(st + 1), then P.V(st) ----------------
     if (lane == 0) {
       // K tiles of a stage: [128 token rows][128 B], 128-byte swizzle (K-major A);
-      // V tiles: the same rows read as MN-major A (V^T); Q^T terms: [16][128 B]
-      // K-major B; P^T terms: [128 tokens][16 B], 8-token core matrices (MN-major B)
+      // V tiles: the same rows read as MN-major A (V^T).  The terms of Q^T and of P^T
+      // sit side by side along N, so one MMA of N = 16 x terms covers them all and
+      // reads each K or V tile once: Q^T terms [16 rows][128 B] K-major B, their
+      // 8-row groups 1024 B apart, term after term; P^T terms [128 tokens][16 B]
+      // MN-major B, 8-token core matrices 128 B apart along K, terms 2 KB apart
+      // along N.
       const uint64_t kdesc = umma_smem_desc(smem_u32(raw), 16, 1024, kUmmaSwizzle128B);
       const uint64_t qdesc = umma_smem_desc(smem_u32(qop), 16, 1024, kUmmaSwizzle128B);
-      const uint64_t pdesc = umma_smem_desc(smem_u32(pop), 128, 128, 0);
+      const uint64_t pdesc = umma_smem_desc(smem_u32(pop), 128, kStTerm, 0);
+      constexpr uint32_t kIdescS = umma_idesc_f16(0, 0, kStTokens, kSharedCols * NQ);
       bool ok = mbar_wait_bounded(qready, 0);
       // Polls the barriers and issues S(ns) as soon as its stage has landed and its
       // S buffer is free (the P.V of stage ns - 2 is issued, so its softmax has read
@@ -876,12 +898,9 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
           const uint64_t kd = kdesc + uint64_t(((ns % kStRing) * kStRawStage) >> 4);
           const uint32_t sb = tmem + kStTmemS + uint32_t(ns & 1) * (16 * 3);
 #pragma unroll
-          for (int t = 0; t < NQ; ++t)
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // 32 dims per step
-              umma_f8_ss(sb + 16 * t, kd + uint64_t((ks * 32) >> 4),
-                         qdesc + uint64_t((t * kStTerm + ks * 32) >> 4), kStIdescS,
-                         ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < 4; ++ks)  // 32 dims per step, every Q term at once
+            umma_f8_ss(sb, kd + uint64_t((ks * 32) >> 4), qdesc + uint64_t((ks * 32) >> 4),
+                       kIdescS, ks > 0 ? 1u : 0u);
           umma_commit(&sfull[ns & 1]);
           ++ns;
           prog = true;
@@ -891,12 +910,10 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
           const uint64_t vd = kdesc + uint64_t(((npv % kStRing) * kStRawStage +
                                                 kStTiles * kStRawTile) >> 4);
 #pragma unroll
-          for (int t = 0; t < kStPTerms; ++t)
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // 32 tokens per step
-              umma_f8_ss(tmem + kStTmemO + 16 * t, vd + uint64_t((ks * 4096) >> 4),
-                         pdesc + uint64_t((t * kStTerm + ks * 512) >> 4), kStIdescPV,
-                         (npv > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < 4; ++ks)  // 32 tokens per step, every P term at once
+            umma_f8_ss(tmem + kStTmemO, vd + uint64_t((ks * 4096) >> 4),
+                       pdesc + uint64_t((ks * 512) >> 4), kStIdescPV,
+                       (npv > 0 || ks > 0) ? 1u : 0u);
           umma_commit(odone);
           umma_commit(&empty[npv % kStRing]);  // the raw stage is read (S and P.V)
           ++npv;

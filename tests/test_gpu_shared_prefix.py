@@ -149,3 +149,33 @@ def test_groups_block_sizes(bs):
     wl = W.make_group_workload(5, (1, 6), (0, 3), (1, 90), num_heads=32, num_kv_heads=8,
                                dtype="bf16", seed=bs, block_size=bs)
     _check(wl, "f32")
+
+
+@pytest.mark.parametrize("qdt", ["bf16", "f16"])
+def test_fp8_persistent_walk_many_units_and_empty_contexts(qdt):
+    """E4M3 caches, far more units than resident CTAs (1440 here: each CTA walks
+    several, their stages through one ring), units past a small group's members
+    (no sequence: nothing written), and whole groups whose contexts are empty
+    (prefix 0, length 0: zero outputs) among them."""
+    wl = W.make_group_workload(90, (1, 7), (0, 3), (1, 60), num_heads=32, num_kv_heads=8,
+                               dtype=qdt, seed=31, cache_dtype="e4m3")
+    d = flow.to_device(wl)
+    pa.pa_reshape_and_cache(d.new_key, d.new_value, d.key_cache, d.value_cache, d.slot_mapping,
+                            k_scale=wl.k_scale, v_scale=wl.v_scale)
+    gs = wl.group_starts.tolist()
+    sl, pl = wl.seq_lens.clone(), wl.prefix_lens.clone()
+    empty = []
+    for g in (3, 40, 89):
+        empty += list(range(gs[g], gs[g + 1]))
+        pl[g] = 0
+    sl[empty] = 0
+    d2 = flow.Dev(**{**d.__dict__, "seq_lens": sl.cuda()})
+    out = _run_shared(wl, d2, "f32", prefix_lens=pl)
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error() == 0
+    assert torch.equal(out[empty], torch.zeros_like(out[empty]))
+    rest = [i for i in range(len(sl)) if i not in set(empty)]
+    kc, vc = flow.oracle_caches(wl)
+    ref = flow.oracle_decode(wl, kc, vc, rest)
+    err = flow.max_abs_err(out[torch.as_tensor(rest, device="cuda")], ref)
+    assert err <= flow.TOL["f32"], f"max abs error {err:.3e}"
