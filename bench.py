@@ -446,51 +446,47 @@ def timed_loop(step, launches, steps, warmup, dev, stream, world, rank):
 def timing_note(args) -> str:
     if args.no_graphs:
         return "each timed step calls the library from Python (host launch overhead included)"
-    return ("each timed step replays two CUDA graphs of the library's calls (cache writes, then "
-            "the hot kernels); the step time brackets both with CUDA events on the stream, the "
-            "launch time brackets the hot kernels with event record nodes inside the graph "
-            "(graph launch latency excluded)")
+    return ("each timed step replays one CUDA graph of the library's calls (cache writes, then "
+            "the hot kernels); the step time brackets the steps with CUDA events on the stream, "
+            "the launch time brackets the hot kernels with event record nodes inside the graph")
 
 
 MAX_HOT_GRAPHS = 200
 
 
 def graph_step(writes, hot, run_step, inputs, out, ev, dev, stream, args):
-    """The step the timed loop runs.  By default each step replays two CUDA graphs
-    captured from the same library calls -- the cache writes (and copies), then the
-    hot kernel(s) -- so host-side call overhead never idles the GPU inside the timed
-    region.  Each hot graph holds its own pair of timing events, recorded as event
-    nodes around the hot kernels, so a launch's time is the kernels' and not the
-    graph launch's; one hot graph per timed step (up to MAX_HOT_GRAPHS, replayed in
-    turn) keeps every timed step's pair apart.  With --no-graphs the step calls the
-    library directly (run_step)."""
+    """The step the timed loop runs.  By default each step replays one CUDA graph
+    captured from the same library calls: the cache writes (and copies), then the
+    hot kernel(s) between a pair of timing events recorded as event nodes of the
+    graph, so host-side call overhead never idles the GPU inside the timed region and
+    a launch's time is the hot kernels' (their launch prepared while the writes run).
+    One graph per timed step (up to MAX_HOT_GRAPHS, replayed in turn) keeps every
+    timed step's pair apart.  With --no-graphs the step calls the library directly
+    (run_step)."""
     if args.no_graphs:
         return lambda timed: run_step(inputs, out, timed)
     run_step(inputs, out, False)          # warm: every kernel attribute set, maps encoded
     torch.cuda.synchronize(dev)
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
-    gw = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gw, stream=side):
-        writes()
-    hots = []
+    graphs = []
     for _ in range(max(1, min(args.steps, MAX_HOT_GRAPHS))):
         g = torch.cuda.CUDAGraph()
         e0 = torch.cuda.Event(enable_timing=True, external=True)
         e1 = torch.cuda.Event(enable_timing=True, external=True)
         with torch.cuda.graph(g, stream=side):
+            writes()
             e0.record(side)
             hot()
             e1.record(side)
-        hots.append((g, e0, e1))
+        graphs.append((g, e0, e1))
     stream.wait_stream(side)
     torch.cuda.synchronize(dev)
     count = [0]
 
     def step(timed):
-        g, e0, e1 = hots[count[0] % len(hots)]
+        g, e0, e1 = graphs[count[0] % len(graphs)]
         count[0] += 1
-        gw.replay()
         g.replay()
         if timed:
             ev.append((e0, e1))

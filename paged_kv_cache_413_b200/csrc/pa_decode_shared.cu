@@ -119,13 +119,18 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
   const int nseq = min(sp.seqs_per_cta, gs1 - s0);
   if (nseq <= 0) return;
 
-  // lengths of the CTA's sequences and the shared prefix (device data: checked)
+  // lengths of the CTA's sequences and the shared prefix (device data: checked);
+  // every read is issued before the first check, whose error report would order
+  // the reads after it one by one
   const int cap = p.cap;
   int Lmin = cap;
   int Ls[kSharedCols];
 #pragma unroll
+  for (int j = 0; j < kSharedCols; ++j) Ls[j] = j < nseq ? p.seq_lens[s0 + j] : 0;
+  int P = sp.prefix_lens[grp];
+#pragma unroll
   for (int j = 0; j < kSharedCols; ++j) {
-    int L = j < nseq ? p.seq_lens[s0 + j] : 0;
+    int L = Ls[j];
     if (j < nseq && (L < 0 || L > cap)) {
       if (tid == 0) atomicOr(&g_shared_err, PA_DEVERR_SEQ_LEN);
       L = L < 0 ? 0 : cap;
@@ -133,7 +138,6 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
     Ls[j] = L;
     if (j < nseq) Lmin = min(Lmin, L);
   }
-  int P = sp.prefix_lens[grp];
   if (P < 0 || P % p.block_size != 0 || P > Lmin) {
     if (tid == 0 && sub == 0 && kvh == 0) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
     P = P < 0 ? 0 : (min(P, Lmin) / p.block_size) * p.block_size;
@@ -721,9 +725,9 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.x;
+  const int kvh = blockIdx.y;
   const int grp = unit / sp.ctas_per_group;
   const int sub = unit - grp * sp.ctas_per_group;
-  const int kvh = blockIdx.y;
   const int G = p.group;
   int gs0 = sp.group_starts[grp], gs1 = sp.group_starts[grp + 1];
   if (gs0 < 0 || gs1 > p.num_seqs || gs1 < gs0) {  // outside the batch: skip the group
@@ -737,12 +741,33 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   if (nseq <= 0) return;  // uniform over the CTA, before any barrier or TMEM
   const int ncols = nseq * G;
 
-  // lengths and the shared prefix (device data: checked), as the mma.sync kernel
+  // The producer's block-table entries of the first group of 4 stages: lane l takes
+  // stream tile l.  They are read now, before the lengths are known, on the guess
+  // that the tile lies in the shared prefix (member 0's table, logical tile l, and
+  // every member's entry for the promise check); a lane whose guess fails reads
+  // its entry again once the stream layout is known.  The reads stay inside the
+  // members' table rows.
+  int32_t nx[kSharedCols];  // the fetched tile's entry in each member's table (prefix)
+  const bool spec = warp == kStProducerWarp && lane / p.tiles_per_block < p.max_blocks_per_seq;
+  if (spec) {
+    const int e = lane / p.tiles_per_block;
+#pragma unroll
+    for (int jj = 0; jj < kSharedCols; ++jj)
+      if (jj < nseq) nx[jj] = p.block_tables[int64_t(s0 + jj) * p.max_blocks_per_seq + e];
+  }
+  // lengths and the shared prefix (device data: checked), as the mma.sync kernel;
+  // every read is issued before the first check, whose error report would order
+  // the reads after it one by one
   if (tid == 0) {
     const int cap = p.cap;
+    int Lr[kSharedCols];
+#pragma unroll
+    for (int j = 0; j < kSharedCols; ++j) Lr[j] = j < nseq ? p.seq_lens[s0 + j] : 0;
+    int P = sp.prefix_lens[grp];
     int Lmin = cap;
+#pragma unroll
     for (int j = 0; j < kSharedCols; ++j) {
-      int L = j < nseq ? p.seq_lens[s0 + j] : 0;
+      int L = Lr[j];
       if (j < nseq && (L < 0 || L > cap)) {
         atomicOr(&g_shared_err, PA_DEVERR_SEQ_LEN);
         L = L < 0 ? 0 : cap;
@@ -750,7 +775,6 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       own_len[j] = L;
       if (j < nseq) Lmin = min(Lmin, L);
     }
-    int P = sp.prefix_lens[grp];
     if (P < 0 || P % p.block_size != 0 || P > Lmin) {
       if (sub == 0 && kvh == 0) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
       P = P < 0 ? 0 : (min(P, Lmin) / p.block_size) * p.block_size;
@@ -795,8 +819,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     // entries of group g + 1 are read while group g streams and are checked (the
     // prefix promise, the block range) when their group starts, so no table read
     // sits between a freed ring slot and its next load.
-    int32_t nx[kSharedCols];  // the fetched tile's entry in each member's table (prefix)
-    int nx_T = 0, nx_lt = 0;  // or in its owner's (nx[0]); its logical tile there
+    int nx_T = 0, nx_lt = 0;  // the fetched tile (entries in nx); its logical tile
     auto fetch = [&](int T) {
       nx_T = T;
       if (T >= ntotal) return;
@@ -832,7 +855,12 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       return ((phys * p.num_kv_heads + kvh) * p.tiles_per_block + (nx_lt - e * p.tiles_per_block)) *
              kBlockSize;
     };
-    fetch(lane);
+    if (spec && lane < pblk && lane < ntotal) {  // the guess held: entries in nx already
+      nx_T = lane;
+      nx_lt = lane;
+    } else {
+      fetch(lane);
+    }
     for (int st = 0; st < nstages && ok; ++st) {
       if ((st & 3) == 0) {
         ent = resolve();
@@ -1115,12 +1143,36 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     // ---- epilogue: column sums over the CTA, O^T row of this dim, outputs ----
     if (nstages > 0) wait(odone, (nstages - 1) & 1);
     tcgen05_fence_after();
+    // column sums of the warp: halve the columns a lane holds at each step (16
+    // shuffles); lanes 2c' and 2c' + 1 end with one column's sum
 #pragma unroll
-    for (int n = 0; n < kSharedCols; ++n) {
-      float v = lacc[n];
+    for (int i = 0; i < 8; ++i) {
+      const bool h = lane & 16;
+      const float keep = h ? lacc[i + 8] : lacc[i], send = h ? lacc[i] : lacc[i + 8];
+      lacc[i] = keep + __shfl_xor_sync(kFullMask, send, 16);
+    }
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(kFullMask, v, o);
-      if (lane == 0) lsum[warp * kSharedCols + n] = v;
+    for (int i = 0; i < 4; ++i) {
+      const bool h = lane & 8;
+      const float keep = h ? lacc[i + 4] : lacc[i], send = h ? lacc[i] : lacc[i + 4];
+      lacc[i] = keep + __shfl_xor_sync(kFullMask, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const bool h = lane & 4;
+      const float keep = h ? lacc[i + 2] : lacc[i], send = h ? lacc[i] : lacc[i + 2];
+      lacc[i] = keep + __shfl_xor_sync(kFullMask, send, 4);
+    }
+    {
+      const bool h = lane & 2;
+      const float keep = h ? lacc[1] : lacc[0], send = h ? lacc[0] : lacc[1];
+      lacc[0] = keep + __shfl_xor_sync(kFullMask, send, 2);
+    }
+    lacc[0] += __shfl_xor_sync(kFullMask, lacc[0], 1);
+    {
+      const int c = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                    ((lane >> 1) & 1);
+      if ((lane & 1) == 0) lsum[warp * kSharedCols + c] = lacc[0];
     }
     named_bar_sync(1, kStQuads * 32);
     // per column, once: 1 / l (v_scale folded in) and the output row; the vote
