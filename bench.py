@@ -935,10 +935,13 @@ def prefill_case(name, dev, args, world, rank, with_e2e=True, with_cpu=False):
 def prefill_roofline(name, p):
     cfg = p["wl"].cfg
     peak, kind = tensor_peak()
-    # the launcher's rule: 128-row tcgen05 tiles once a chunk fills one
-    kernel = ("prefill_tc_kernel (tcgen05.mma, TMEM accumulators)"
-              if p["max_q"] * (cfg.num_heads // cfg.num_kv_heads) >= 128
-              else "prefill_kernel (mma.sync m16n8k16)")
+    # the launcher's rule: 128-row tcgen05 tiles once a chunk fills one, two of them
+    # in ping-pong once a (sequence, kv head) has two
+    rows = p["max_q"] * (cfg.num_heads // cfg.num_kv_heads)
+    kernel = ("prefill_pp_kernel (tcgen05.mma, two tiles in ping-pong, TMEM accumulators)"
+              if rows > 128 else
+              "prefill_tc_kernel (tcgen05.mma, TMEM accumulators)" if rows == 128 else
+              "prefill_kernel (mma.sync m16n8k16)")
     achieved = p["flops"] / (p["kern_ms"] * 1e-3) / 1e12
     return {"bound": "tensor", "kernel": kernel, "achieved": round(achieved, 2), "peak": peak,
             "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),

@@ -865,6 +865,488 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Ping-pong form of the tcgen05 prefill: a CTA works on two 128-row tiles of one
+// (sequence, kv head) at once -- row blocks 2k and 2k + 1, which share every KV
+// stage -- with one softmax warpgroup per tile (warps 0-3 tile A, 4-7 tile B;
+// thread = row, all 128 columns of S, read from TMEM once per stage into
+// registers: setmaxnreg gives the softmax warpgroups 216 registers a thread and
+// the load/MMA warpgroup 72).  TMEM holds S and O of both tiles (4 x 128
+// columns); Q moves to shared memory (K-major, 128-byte swizzle) and S becomes an
+// SS MMA.  The MMA thread issues, per stage j,
+//     P.V_A(j), S_A(j + 1), P.V_B(j), S_B(j + 1)
+// so each tile's softmax runs while the tensor core works on the other tile.  P is
+// written over its own S as 16-bit pairs (two bf16 terms for kSplitP) and O stays
+// in TMEM for the whole pair, rescaled per row only when the row's reference
+// maximum moves by more than 2^8.  No barrier is shared between the two
+// warpgroups, and a row never needs another thread.  K and V keep their rings and
+// producer warps; a K stage is released after the last S that reads it, a V stage
+// after the last P.V.
+// ---------------------------------------------------------------------------
+// Warpgroups: 0 and 1 softmax (tiles A and B), 2 the K loader, the MMA issuer, the
+// V loader and one idle warp (setmaxnreg acts on whole warpgroups).  The split
+// moves registers from warpgroup 2 to the softmax warpgroups, so that a thread
+// holds its row's 128 scores; 72 / 216 spilled least of the splits that add up to
+// the launch's registers (40 / 232: the loaders spill, 88 / 208: the softmax).
+constexpr int kPpThreads = 12 * 32;
+constexpr int kPpKWarp = 8;
+constexpr int kPpMmaWarp = 9;
+constexpr int kPpVWarp = 10;
+constexpr int kPpLaunchRegs = 168;   // 65536 / 384, rounded down to 8
+constexpr int kPpLoadRegs = 72;      // warpgroup 2 after setmaxnreg.dec
+constexpr int kPpSoftmaxRegs = 216;  // warpgroups 0, 1 after setmaxnreg.inc
+static_assert(128 * kPpLoadRegs + 256 * kPpSoftmaxRegs <= kPpThreads * kPpLaunchRegs,
+              "the split draws only on the registers the CTA was launched with");
+constexpr int kPpQBytes = kTcRows * 128 * 2;  // Q of a tile: [2 halves][128 rows][128 B]
+constexpr uint32_t kPpTmemCols = 512;
+__host__ __device__ constexpr uint32_t pp_tmem_s(int x) { return uint32_t(x) * 128; }
+__host__ __device__ constexpr uint32_t pp_tmem_o(int x) { return 256 + uint32_t(x) * 128; }
+
+constexpr size_t pp_prefill_smem_bytes() {
+  return 1024 + 2 * size_t(kTcStages) * kTcTileBytes + 2 * size_t(kPpQBytes) +
+         (4 * kTcStages + 9) * sizeof(uint64_t) + 16;
+}
+static_assert(kTcKv == 128, "one S buffer of 128 columns per tile");
+static_assert(pp_prefill_smem_bytes() <= 227 * 1024, "rings and Q fit 227 KB");
+
+// The pair of row blocks (2 pr, 2 pr + 1) of (sequence, kv head): both tiles' info.
+struct PpPair {
+  TcTile t[2];
+  bool has[2];
+  int nkb, ntiles, pos_last;  // stages, 16-token pool tiles, last visible position
+};
+
+__device__ __forceinline__ bool pp_pair(const TcPrefillParams& pp, int pair, PpPair& x,
+                                        bool report) {
+  const int pairs_per = (pp.row_blocks + 1) / 2;
+  const int skv = pair / pairs_per, pr = pair - skv * pairs_per;  // skv = seq * Hkv + kvh
+  const int base = skv * pp.row_blocks;
+  x.has[0] = tc_tile(pp, base + 2 * pr, x.t[0], report);
+  if (!x.has[0]) return false;
+  x.has[1] = 2 * pr + 1 < pp.row_blocks && tc_tile(pp, base + 2 * pr + 1, x.t[1], false);
+  const TcTile& last = x.has[1] ? x.t[1] : x.t[0];
+  x.nkb = last.nkb;
+  x.ntiles = last.ntiles;
+  x.pos_last = last.pos_last;
+  return true;
+}
+
+__device__ __forceinline__ bool pp_next(const TcPrefillParams& pp, int num_pairs, int& pair,
+                                        PpPair& x, bool report) {
+  for (pair = pair < 0 ? int(blockIdx.x) : pair + int(gridDim.x); pair < num_pairs;
+       pair += gridDim.x)
+    if (pp_pair(pp, pair, x, report)) return true;
+  return false;
+}
+
+template <typename CT, bool kSplitP>
+__global__ void __launch_bounds__(kPpThreads, 1)
+    prefill_pp_kernel(const __grid_constant__ TcPrefillParams pp, int num_pairs) {
+  constexpr int D = 128;
+  static_assert(CacheTraits<CT>::bytes == 2, "16-bit caches");
+  constexpr uint32_t kFmt = std::is_same<CT, __nv_bfloat16>::value ? 1u : 0u;
+  constexpr uint32_t kIdescS = umma_idesc_f16(kFmt, 0, kTcRows, kTcKv);
+  constexpr uint32_t kIdescPV = umma_idesc_f16(kFmt, 1, kTcRows, D);
+  const Params& p = pp.p;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* ksm = smem;                                  // K ring
+  uint8_t* vsm = ksm + kTcStages * kTcTileBytes;        // V ring
+  uint8_t* qsm = vsm + kTcStages * kTcTileBytes;        // Q of tiles A, B
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(qsm + 2 * kPpQBytes);
+  uint64_t* kempty = kfull + kTcStages;
+  uint64_t* vfull = kempty + kTcStages;
+  uint64_t* vempty = vfull + kTcStages;
+  uint64_t* s_full = vempty + kTcStages;  // [2 tiles]: S of the tile's stage written
+  uint64_t* o_full = s_full + 2;          // [2]: P.V of the tile's stage done
+  uint64_t* p_ready = o_full + 2;         // [2]: P in TMEM, O rescaled (4 warps)
+  uint64_t* q_ready = p_ready + 2;        // [2]: Q of the tile's pair in smem (4 warps)
+  uint64_t* done = q_ready + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int st = 0; st < kTcStages; ++st) {
+      mbar_init(&kfull[st], 1);
+      mbar_init(&kempty[st], 1);
+      mbar_init(&vfull[st], 1);
+      mbar_init(&vempty[st], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&o_full[x], 1);
+      mbar_init(&p_ready[x], 4);
+      mbar_init(&q_ready[x], 4);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == kPpMmaWarp) {  // the MMA warp owns the TMEM allocation
+    tmem_alloc(tmem_slot, kPpTmemCols);
+    tmem_relinquish();
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  tcgen05_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kPpLoadRegs));
+  if (warp == kPpKWarp || warp == kPpVWarp) {
+    // ---------------- TMA producers: stage j = pool tiles 8 j .. 8 j + 7 of the pair ----------------
+    const bool is_k = warp == kPpKWarp;
+    const CUtensorMap* map = is_k ? &pp.tmk : &pp.tmv;
+    uint8_t* ring = is_k ? ksm : vsm;
+    uint64_t* full = is_k ? kfull : vfull;
+    uint64_t* empty = is_k ? kempty : vempty;
+    const uint64_t policy = l2_policy_evict_last();  // the pair's other row blocks read it again
+    constexpr int kPre = 32 / kTcTiles;
+    int g = 0;
+    bool ok = true;
+    int pair = -1;
+    PpPair x;
+    while (ok && pp_next(pp, num_pairs, pair, x, is_k && lane == 0)) {
+      const TcTile& t = x.t[0];
+      const int32_t* table_row = p.block_tables + int64_t(t.seq) * p.max_blocks_per_seq;
+      int ent = 0;
+      for (int jb = 0; jb < x.nkb && ok; ++jb, ++g) {
+        const int stage = g % kTcStages;
+        const int ntl = min(kTcTiles, x.ntiles - kTcTiles * jb);
+        if (jb % kPre == 0) {
+          const int tt = kTcTiles * jb + lane;
+          ent = 0;
+          if (tt < x.ntiles) {
+            const int e = tt / p.tiles_per_block;
+            int32_t phys = table_row[e];
+            if (phys < 0 || phys >= p.num_blocks) {
+              if (is_k) atomicOr(&g_prefill_err, PA_DEVERR_BLOCK_RANGE);
+              phys = 0;
+            }
+            ent = (phys * p.num_kv_heads + t.kvh) * p.tiles_per_block +
+                  (tt - e * p.tiles_per_block);
+          }
+        }
+        int tls[kTcTiles];
+#pragma unroll
+        for (int i = 0; i < kTcTiles; ++i)
+          tls[i] = __shfl_sync(kFullMask, ent, kTcTiles * (jb % kPre) + i);
+        if (lane == 0) {
+          if (g >= kTcStages && !mbar_wait_bounded(&empty[stage], ((g / kTcStages) - 1) & 1)) {
+            atomicOr(&g_prefill_err, PA_DEVERR_PIPE_TIMEOUT);
+            ok = false;
+          }
+          if (ok) {
+            uint8_t* dst = ring + stage * kTcTileBytes;
+            mbar_arrive_expect_tx(&full[stage], uint32_t(ntl) * 2 * 2048);
+            for (int i = 0; i < ntl; ++i) {
+              const int row = tls[i] * kBlockSize;
+              tma_load_2d(dst + i * 2048, map, 0, row, &full[stage], policy);
+              tma_load_2d(dst + kTcTileBytes / 2 + i * 2048, map, 64, row, &full[stage], policy);
+            }
+          }
+        }
+        ok = __shfl_sync(kFullMask, ok, 0);
+        if (!ok) break;
+      }
+    }
+    if (lane == 0) {  // no copy may still be landing when the CTA exits (one ring)
+      for (int i = max(0, g - kTcStages); i < g; ++i)
+        if (!mbar_wait_bounded(&full[i % kTcStages], (i / kTcStages) & 1))
+          atomicOr(&g_prefill_err, PA_DEVERR_PIPE_TIMEOUT);
+    }
+  } else if (warp == kPpMmaWarp) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      const uint64_t kdesc0 = umma_smem_desc(smem_u32(ksm), 16, 1024, kUmmaSwizzle128B);
+      const uint64_t vdesc0 = umma_smem_desc(smem_u32(vsm), kTcTileBytes / 2, 1024,
+                                             kUmmaSwizzle128B);
+      const uint64_t qdesc0 = umma_smem_desc(smem_u32(qsm), 16, 1024, kUmmaSwizzle128B);
+      int g = 0;
+      int cnt[2] = {0, 0};   // stages each tile has taken part in (phase counters)
+      int nq[2] = {0, 0};    // pairs in which each tile was present (Q phases)
+      bool ok = true;
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        if (ok && !mbar_wait_bounded(bar, parity)) ok = false;
+        return ok;
+      };
+      auto issue_s = [&](int xt, int gs) {  // S of tile xt from K stage gs
+        tcgen05_fence_after();
+        const uint64_t kd = kdesc0 + uint64_t(((gs % kTcStages) * kTcTileBytes) >> 4);
+        const uint64_t qd = qdesc0 + uint64_t((xt * kPpQBytes) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t off = uint64_t(((ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32) >> 4);
+          umma_f16_ss(tmem + pp_tmem_s(xt), qd + off, kd + off, kIdescS, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[xt]);
+      };
+      auto issue_pv = [&](int xt, int gs, int jb) {  // O_xt += P_xt . V(stage gs)
+        tcgen05_fence_after();
+        const uint64_t vd = vdesc0 + uint64_t(((gs % kTcStages) * kTcTileBytes) >> 4);
+        const uint32_t pt = tmem + pp_tmem_s(xt);
+#pragma unroll
+        for (int t = 0; t < (kSplitP ? 2 : 1); ++t) {
+#pragma unroll
+          for (int ks = 0; ks < kTcKv / 16; ++ks)
+            umma_f16_ts(tmem + pp_tmem_o(xt), pt + uint32_t(t * (kTcKv / 2) + ks * 8),
+                        vd + uint64_t((ks * 2048) >> 4), kIdescPV,
+                        (jb > 0 || t > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(&o_full[xt]);
+      };
+      int pair = -1;
+      PpPair x;
+      while (ok && pp_next(pp, num_pairs, pair, x, false)) {
+        const int nkb = x.nkb;
+        auto in = [&](int xt, int jb) { return x.has[xt] && jb < x.t[xt].nkb; };
+        // Q of the pair's tiles
+        for (int xt = 0; xt < 2; ++xt)
+          if (x.has[xt]) wait(&q_ready[xt], (nq[xt]++) & 1);
+        // stage 0: S of both tiles
+        if (!wait(&kfull[g % kTcStages], (g / kTcStages) & 1)) break;
+        for (int xt = 0; xt < 2; ++xt)
+          if (in(xt, 0)) issue_s(xt, g);
+        umma_commit(&kempty[g % kTcStages]);
+        for (int jb = 0; jb < nkb && ok; ++jb, ++g) {
+          bool vwaited = false, kwaited = false;
+          // P.V_A(jb), then S_A(jb + 1)
+          if (in(0, jb)) {
+            if (!wait(&p_ready[0], cnt[0] & 1)) break;
+            if (!wait(&vfull[g % kTcStages], (g / kTcStages) & 1)) break;
+            vwaited = true;
+            issue_pv(0, g, jb);
+            ++cnt[0];
+          }
+          if (jb + 1 < nkb && in(0, jb + 1)) {
+            if (!wait(&kfull[(g + 1) % kTcStages], ((g + 1) / kTcStages) & 1)) break;
+            kwaited = true;
+            issue_s(0, g + 1);
+          }
+          // P.V_B(jb), then S_B(jb + 1)
+          if (in(1, jb)) {
+            if (!wait(&p_ready[1], cnt[1] & 1)) break;
+            if (!vwaited && !wait(&vfull[g % kTcStages], (g / kTcStages) & 1)) break;
+            issue_pv(1, g, jb);
+            ++cnt[1];
+          }
+          umma_commit(&vempty[g % kTcStages]);  // the V stage's last P.V is issued
+          if (jb + 1 < nkb) {
+            if (in(1, jb + 1)) {
+              if (!kwaited && !wait(&kfull[(g + 1) % kTcStages], ((g + 1) / kTcStages) & 1))
+                break;
+              issue_s(1, g + 1);
+            }
+            umma_commit(&kempty[(g + 1) % kTcStages]);  // its last S is issued
+          }
+        }
+      }
+      if (!ok) atomicOr(&g_prefill_err, PA_DEVERR_PIPE_TIMEOUT);
+      umma_commit(done);  // fires once every MMA issued above has completed
+    }
+    __syncwarp();
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kPpSoftmaxRegs));
+    // ---------------- softmax warpgroups: thread = row of tile xt ----------------
+    const int xt = warp >> 2, qd = warp & 3;
+    const int r = 32 * qd + lane;                           // TMEM lane and row of the tile
+    const uint32_t tl = tmem + (uint32_t(32 * qd) << 16);  // this warp's lane quadrant
+    const float mult = fabsf(p.q_mult);                     // Q carries the sign
+    const uint32_t flip = p.q_mult < 0.f ? 0x80008000u : 0u;
+    uint8_t* qx = qsm + xt * kPpQBytes;
+    bool ok = true;  // warp-uniform; after a failure waits are skipped
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
+    };
+    auto arrive = [&](uint64_t* bar) {
+      tcgen05_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+    int g = 0, cnt = 0;  // stages of the CTA, stages of this tile
+    int pair = -1;
+    PpPair x;
+    while (pp_next(pp, num_pairs, pair, x, false)) {
+      const int gp = g;
+      g += x.nkb;
+      if (!x.has[xt]) continue;  // tile B of a pair with a single row block
+      const TcTile& t = x.t[xt];
+      const int gr = t.row0 + r;
+      const bool valid = gr < t.rows;
+      const int pos = valid ? t.L - t.nq + gr / p.group : -1;
+      // ---- Q row into shared memory (K-major, 128-byte swizzle), sign carried ----
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.query + (int64_t(t.q0 + (valid ? gr / p.group : 0)) * p.num_heads +
+                       t.kvh * p.group + (valid ? gr % p.group : 0)) * D * 2);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+          v.x ^= flip;
+          v.y ^= flip;
+          v.z ^= flip;
+          v.w ^= flip;
+          *reinterpret_cast<uint4*>(qx + (c >> 3) * (kPpQBytes / 2) + r * 128 +
+                                    (((c & 7) ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        arrive(&q_ready[xt]);
+      }
+      float m = -INFINITY, l = 0.f;  // reference max (exp2 domain), row sum
+      const uint32_t sb = tl + pp_tmem_s(xt);
+      for (int jb = 0; jb < t.nkb; ++jb, ++cnt) {
+        wait(&s_full[xt], cnt & 1);
+        tcgen05_fence_after();
+        // causal, context and padding mask: only stages that cross this row's last
+        // visible position pay for it
+        const int nvis = pos - jb * kTcKv + 1;
+        const bool edge = nvis < kTcKv;
+        // the row's 128 scores, one TMEM read
+        float v[128];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32(sb + 32 * q, *reinterpret_cast<float(*)[32]>(v + 32 * q));
+        tmem_wait_ld();
+        // (an edge stage scales before masking, so that a zero scale never meets -inf)
+        if (edge) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) v[i] = i < nvis ? v[i] * mult : -INFINITY;
+        }
+        float r8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) r8[k] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; i += 2) r8[(i >> 1) & 7] = max3(r8[(i >> 1) & 7], v[i], v[i + 1]);
+        const float mx = fmaxf(fmaxf(fmaxf(r8[0], r8[1]), fmaxf(r8[2], r8[3])),
+                               fmaxf(fmaxf(r8[4], r8[5]), fmaxf(r8[6], r8[7]))) *
+                         (edge ? 1.f : mult);
+        if (jb == 0) {
+          m = mx;  // O is written, not accumulated, by the tile's first P.V
+        } else {
+          const bool move = mx > m + kTcRescaleLog2;
+          if (__any_sync(kFullMask, move)) {
+            // rescale this warp's rows of O once P.V(jb - 1) of this tile has landed
+            wait(&o_full[xt], (cnt - 1) & 1);
+            tcgen05_fence_after();
+            const float f = move ? ex2_approx(m - mx) : 1.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float o[32];
+              tmem_ld32(tl + pp_tmem_o(xt) + 32 * q, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] *= f;
+              tmem_st32(tl + pp_tmem_o(xt) + 32 * q, o);
+            }
+            l *= f;
+            if (move) m = mx;
+          }
+        }
+        const float mu = m == -INFINITY ? 0.f : m;
+        const float me = edge ? 1.f : mult;  // multiplier still to apply
+        const float2 me2 = make_float2(me, me), nmu2 = make_float2(-mu, -mu);
+        float2 a4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        // exponentials, then P over S as 16-bit pairs: chunk q's hi term into columns
+        // [16 q, 16 q + 16), its lo term into [64 + 16 q, ...) (S is all in registers)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pw[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int i = 32 * q + 2 * c;
+            const float2 e = fma2(make_float2(v[i], v[i + 1]), me2, nmu2);
+            v[i] = ex2_approx(e.x);
+            v[i + 1] = ex2_approx(e.y);
+            a4[c & 3] = add2(a4[c & 3], make_float2(v[i], v[i + 1]));
+            pw[c] = pack2(v[i], v[i + 1], CT{});
+          }
+          tmem_st16(sb + 16 * q, pw);
+          if constexpr (kSplitP) {
+            uint32_t lw[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int i = 32 * q + 2 * c;
+              const float2 hi = unpack2(pw[c], CT{});
+              lw[c] = pack2(v[i] - hi.x, v[i + 1] - hi.y, CT{});
+            }
+            tmem_st16(sb + kTcKv / 2 + 16 * q, lw);
+          }
+        }
+        const float2 a2 = add2(add2(a4[0], a4[1]), add2(a4[2], a4[3]));
+        l += a2.x + a2.y;
+        // The pair's last stage: V rows past its last visible token may be stale or
+        // NaN.  The tile whose P.V reads that stage first zeroes them (tile A if it
+        // takes part in the stage), before its P is announced.
+        if (jb == x.nkb - 1 && (xt == 0 || t.nkb != x.t[0].nkb || !x.has[0])) {
+          const int gs = gp + jb;
+          wait(&vfull[gs % kTcStages], (gs / kTcStages) & 1);
+          if (ok && jb * kTcKv + r > x.pos_last) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint8_t* vrow = vsm + (gs % kTcStages) * kTcTileBytes + half * (kTcTileBytes / 2) +
+                              r * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        tmem_wait_st();
+        arrive(&p_ready[xt]);
+      }
+      // epilogue: O / l of this tile's rows
+      wait(&o_full[xt], (cnt - 1) & 1);
+      if (ok) {
+        tcgen05_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const int64_t orow = (int64_t(t.q0 + (valid ? gr / p.group : 0)) * p.num_heads +
+                              t.kvh * p.group + (valid ? gr % p.group : 0)) * D;
+        uint8_t* dst = static_cast<uint8_t*>(p.out);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float v[32];
+          tmem_ld32(tl + pp_tmem_o(xt) + 32 * q, v);
+          tmem_wait_ld();
+          if (!valid) continue;
+          if (p.out_dtype == PA_F32) {
+#pragma unroll
+            for (int d = 0; d < 32; d += 4)
+              *reinterpret_cast<float4*>(dst + (orow + 32 * q + d) * 4) =
+                  make_float4(v[d] * inv, v[d + 1] * inv, v[d + 2] * inv, v[d + 3] * inv);
+          } else if (p.out_dtype == PA_F16) {
+#pragma unroll
+            for (int d = 0; d < 32; d += 8)
+              *reinterpret_cast<uint4*>(dst + (orow + 32 * q + d) * 2) =
+                  make_uint4(pack2(v[d] * inv, v[d + 1] * inv, __half{}),
+                             pack2(v[d + 2] * inv, v[d + 3] * inv, __half{}),
+                             pack2(v[d + 4] * inv, v[d + 5] * inv, __half{}),
+                             pack2(v[d + 6] * inv, v[d + 7] * inv, __half{}));
+          } else {
+#pragma unroll
+            for (int d = 0; d < 32; d += 8)
+              *reinterpret_cast<uint4*>(dst + (orow + 32 * q + d) * 2) =
+                  make_uint4(pack2(v[d] * inv, v[d + 1] * inv, __nv_bfloat16{}),
+                             pack2(v[d + 2] * inv, v[d + 3] * inv, __nv_bfloat16{}),
+                             pack2(v[d + 4] * inv, v[d + 5] * inv, __nv_bfloat16{}),
+                             pack2(v[d + 6] * inv, v[d + 7] * inv, __nv_bfloat16{}));
+          }
+        }
+      }
+      tcgen05_fence_before();  // O is read before the next pair's first P.V overwrites it
+    }
+    if (!ok && lane == 0) atomicOr(&g_prefill_err, PA_DEVERR_PIPE_TIMEOUT);
+  }
+  // Free TMEM only after every MMA has completed and every TMEM access is done.
+  __syncthreads();
+  if (warp == kPpMmaWarp) {
+    if (!__all_sync(kFullMask, mbar_wait_bounded(done, 0)) && lane == 0)
+      atomicOr(&g_prefill_err, PA_DEVERR_PIPE_TIMEOUT);
+    tcgen05_fence_after();
+    tmem_dealloc(tmem, kPpTmemCols);
+  }
+}
+
 }  // namespace
 
 int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_query_len,
@@ -925,6 +1407,40 @@ int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_quer
     if (cudaGetDevice(&dev_sm) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_sm) != cudaSuccess)
       return PA_ERR_CUDA;
+    // two 128-row tiles of one (sequence, kv head) per CTA at a time, when a
+    // (sequence, kv head) has two: the other warpgroup would idle otherwise
+    const int64_t pairs = int64_t(a.num_seqs) * a.num_kv_heads * ((tp.row_blocks + 1) / 2);
+    if (tp.row_blocks >= 2 && pairs <= INT32_MAX) {
+      const unsigned grid_pp = unsigned(pairs < sms ? pairs : sms);
+      constexpr size_t smem_pp = pp_prefill_smem_bytes();
+      // The register split assumes the CTA is launched with kPpLaunchRegs a thread
+      // (a split above the launch's registers would wait forever); a build whose
+      // kernel has another count takes the one-tile kernel.  Checked once.
+      auto launch_pp = [&](auto kern, std::atomic<unsigned long long>& mask,
+                           std::atomic<int>& regs) -> int {
+        int r = regs.load(std::memory_order_relaxed);
+        if (r == 0) {
+          cudaFuncAttributes fa;
+          if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return PA_ERR_CUDA;
+          r = fa.numRegs == kPpLaunchRegs ? 1 : -1;
+          regs.store(r, std::memory_order_relaxed);
+        }
+        if (r < 0) return PA_ERR_UNSUPPORTED;
+        if (set_smem_once(kern, smem_pp, mask) != PA_OK) return PA_ERR_CUDA;
+        kern<<<grid_pp, kPpThreads, smem_pp, stream>>>(tp, int(pairs));
+        return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+      };
+      static std::atomic<unsigned long long> pmask_h{0}, pmask_b{0}, pmask_bs{0};
+      static std::atomic<int> pregs_h{0}, pregs_b{0}, pregs_bs{0};
+      int rc;
+      if (a.cache_dtype == PA_F16)
+        rc = launch_pp(prefill_pp_kernel<__half, false>, pmask_h, pregs_h);
+      else if (a.out_dtype == PA_F32)
+        rc = launch_pp(prefill_pp_kernel<__nv_bfloat16, true>, pmask_bs, pregs_bs);
+      else
+        rc = launch_pp(prefill_pp_kernel<__nv_bfloat16, false>, pmask_b, pregs_b);
+      if (rc != PA_ERR_UNSUPPORTED) return rc;
+    }
     const unsigned grid_tc = unsigned(tiles < sms ? tiles : sms);
     constexpr size_t smem = tc_prefill_smem_bytes();
     auto launch = [&](auto kern, std::atomic<unsigned long long>& mask) -> int {
