@@ -608,9 +608,13 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
 //     threads, moved (with a rescale of l and of O^T's columns) only when some
 //     score passes it by more than 2^8, which a vote and a named barrier detect;
 //     each thread sums its own l and the sums meet once, at the end;
-//   * warp 4 streams the raw tiles (tiled TMA, 128-byte swizzle, no multicast)
-//     into a ring of kStRing stages; warp 5 issues each stage's MMAs (S of stage
-//     st + 1 before P.V of stage st) and owns the TMEM allocation.
+//   * warps 4 and 6 stream the raw K and V tiles (tiled TMA, 128-byte swizzle, no
+//     multicast) into two rings of kStRing stages, K and V each with barriers of
+//     their own: a K slot refills as soon as S has read it, so S and the softmax
+//     of a stage can finish while its V is still landing; warp 5 issues each
+//     stage's MMAs (S of stage st + 1 before P.V of stage st) and owns the TMEM
+//     allocation; warp 7 idles.  setmaxnreg gives warps 4-7 72 registers a thread
+//     and the softmax warps 184, so that two CTAs of 8 warps fit an SM.
 // Every mbarrier a waiter could otherwise see two phases ahead is split per
 // buffer.  All waits are bounded; after a failure the waits are skipped but every
 // named barrier is still reached.
@@ -618,15 +622,23 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
 constexpr int kStTokens = 128;                          // tokens per stage (M of S^T)
 constexpr int kStTiles = kStTokens / kBlockSize;        // pool tiles per stage
 constexpr int kStQuads = 4;                             // softmax warps (TMEM lane quadrants)
-constexpr int kStProducerWarp = kStQuads;
-constexpr int kStMmaWarp = kStQuads + 1;
-constexpr int kStThreads = (kStQuads + 2) * 32;
+constexpr int kStKWarp = kStQuads;        // streams the K tiles
+constexpr int kStMmaWarp = kStQuads + 1;  // issues the MMAs, owns TMEM
+constexpr int kStVWarp = kStQuads + 2;    // streams the V tiles; warp 7 idles
+constexpr int kStThreads = (kStQuads + 4) * 32;
+// Two CTAs per SM launch with 128 registers a thread; setmaxnreg then moves them
+// from the loader/MMA warpgroup (72) to the softmax warpgroup (184).
+constexpr int kStLaunchRegs = 128;
+constexpr int kStLoadRegs = 72;      // the least that spills nothing (40 and 56 spill)
+constexpr int kStSoftmaxRegs = 184;
+static_assert(128 * kStLoadRegs + 128 * kStSoftmaxRegs <= kStThreads * kStLaunchRegs,
+              "the split draws only on the registers the CTA was launched with");
 #ifndef PA_SHARED_TC_RING
 #define PA_SHARED_TC_RING 3
 #endif
-constexpr int kStRing = PA_SHARED_TC_RING;              // raw stages in flight
+constexpr int kStRing = PA_SHARED_TC_RING;              // stages in flight, K and V each
 constexpr int kStRawTile = kBlockSize * 128;            // one E4M3 tile of K or V: 2 KB
-constexpr int kStRawStage = 2 * kStTiles * kStRawTile;  // K tiles, then V tiles: 32 KB
+constexpr int kStRawHalf = kStTiles * kStRawTile;      // a stage's K (or V) tiles: 16 KB
 constexpr int kStTerm = kSharedCols * 128;              // one E4M3 term of Q^T or P^T: 2 KB
 constexpr int kStPTerms = 3;                            // terms of P
 constexpr uint32_t kStTmemCols = 256;
@@ -638,8 +650,8 @@ constexpr uint32_t kStIdescPV = umma_idesc_f16_ab(0, 1, 1, 128, kSharedCols * kS
 
 template <int NQ>
 constexpr size_t shared_tc_smem_bytes() {
-  return 1024 + size_t(kStRing) * kStRawStage + size_t(NQ + kStPTerms) * kStTerm +
-         (kStRing * 2 + 8) * sizeof(uint64_t) +
+  return 1024 + size_t(2 * kStRing) * kStRawHalf + size_t(NQ + kStPTerms) * kStTerm +
+         (kStRing * 4 + 8) * sizeof(uint64_t) +
          (8 + 2 * kStQuads * kSharedCols + kStQuads * kSharedCols + kSharedCols) * 4 +
          (2 * (kSharedCols + 1) + 2) * 4;
 }
@@ -705,12 +717,17 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   const Params& p = sp.p;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* raw = smem;                                  // [kStRing][K tiles, V tiles]
-  uint8_t* qop = raw + kStRing * kStRawStage;           // Q^T terms: [NQ][16 rows][128 B] SW128
+  uint8_t* rawk = smem;                                 // [kStRing][8 K tiles]
+  uint8_t* rawv = rawk + kStRing * kStRawHalf;          // [kStRing][8 V tiles]
+  uint8_t* qop = rawv + kStRing * kStRawHalf;           // Q^T terms: [NQ][16 rows][128 B] SW128
   uint8_t* pop = qop + NQ * kStTerm;                    // P^T terms: [3][128 tokens][16 B]
-  uint64_t* full = reinterpret_cast<uint64_t*>(pop + kStPTerms * kStTerm);
-  uint64_t* empty = full + kStRing;
-  uint64_t* sfull = empty + kStRing;                    // [2] S buffer b of stage st written
+  // K and V of a stage have rings and barriers of their own: a K slot is free once
+  // S has read it, a whole softmax and P.V before the V slot of the same stage
+  uint64_t* fullk = reinterpret_cast<uint64_t*>(pop + kStPTerms * kStTerm);
+  uint64_t* fullv = fullk + kStRing;
+  uint64_t* emptyk = fullv + kStRing;
+  uint64_t* emptyv = emptyk + kStRing;
+  uint64_t* sfull = emptyv + kStRing;                    // [2] S buffer b of stage st written
   uint64_t* pready = sfull + 2;                         // P of stage st written, O rescaled
   uint64_t* odone = pready + 1;                         // P.V of stage st done
   uint64_t* qready = odone + 1;                         // Q^T terms written
@@ -748,7 +765,8 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   // its entry again once the stream layout is known.  The reads stay inside the
   // members' table rows.
   int32_t nx[kSharedCols];  // the fetched tile's entry in each member's table (prefix)
-  const bool spec = warp == kStProducerWarp && lane / p.tiles_per_block < p.max_blocks_per_seq;
+  const bool spec = (warp == kStKWarp || warp == kStVWarp) &&
+                    lane / p.tiles_per_block < p.max_blocks_per_seq;
   if (spec) {
     const int e = lane / p.tiles_per_block;
 #pragma unroll
@@ -787,8 +805,10 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     }
     own_start[kSharedCols] = pos;
     for (int i = 0; i < kStRing; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&fullk[i], 1);
+      mbar_init(&fullv[i], 1);
+      mbar_init(&emptyk[i], 1);
+      mbar_init(&emptyv[i], 1);
     }
     mbar_init(&sfull[0], 1);
     mbar_init(&sfull[1], 1);
@@ -810,8 +830,17 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   const int ntotal = own_start[kSharedCols];
   const int nstages = (ntotal + kStTiles - 1) / kStTiles;
 
-  if (warp == kStProducerWarp) {
-    // ---------------- producer: raw E4M3 tiles of each stage ----------------
+  if (warp >= kStQuads) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kStLoadRegs));
+  if (warp == kStKWarp || warp == kStVWarp) {
+    // ---------------- producers: the raw E4M3 K (or V) tiles of each stage ----------------
+    // Both warps walk the same stream and block-table entries; the K warp reports
+    // bad entries.
+    const bool is_k = warp == kStKWarp;
+    uint64_t* fullx = is_k ? fullk : fullv;
+    uint64_t* emptyx = is_k ? emptyk : emptyv;
+    uint8_t* ring = is_k ? rawk : rawv;
+    const CUtensorMap* map = is_k ? &sp.tmk : &sp.tmv;
     const uint64_t policy = l2_policy_evict_first();
     int issued = 0, ent = -1;
     bool ok = true;
@@ -845,10 +874,10 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
 #pragma unroll
         for (int jj = 1; jj < kSharedCols; ++jj)
           if (jj < nseq) same &= nx[jj] == phys;
-        if (!same) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
+        if (!same && is_k) atomicOr(&g_shared_err, PA_DEVERR_PREFIX);
       }
       if (phys < 0 || phys >= p.num_blocks) {
-        atomicOr(&g_shared_err, PA_DEVERR_BLOCK_RANGE);
+        if (is_k) atomicOr(&g_shared_err, PA_DEVERR_BLOCK_RANGE);
         phys = 0;
       }
       const int e = nx_lt / p.tiles_per_block;
@@ -871,22 +900,17 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       for (int i = 0; i < kStTiles; ++i) rows[i] = __shfl_sync(kFullMask, ent, (st & 3) * kStTiles + i);
       const int slot = st % kStRing;
       if (lane == 0) {
-        if (st >= kStRing && !mbar_wait_bounded(&empty[slot], ((st / kStRing) - 1) & 1)) {
+        if (st >= kStRing && !mbar_wait_bounded(&emptyx[slot], ((st / kStRing) - 1) & 1)) {
           atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
           ok = false;
         }
         if (ok) {
           const int n = min(kStTiles, ntotal - st * kStTiles);
-          uint8_t* dst = raw + slot * kStRawStage;
-          mbar_arrive_expect_tx(&full[slot], uint32_t(n) * 2 * kStRawTile);
+          uint8_t* dst = ring + slot * kStRawHalf;
+          mbar_arrive_expect_tx(&fullx[slot], uint32_t(n) * kStRawTile);
 #pragma unroll
-          for (int i = 0; i < kStTiles; ++i) {
-            if (i < n) {
-              tma_load_2d(dst + i * kStRawTile, &sp.tmk, 0, rows[i], &full[slot], policy);
-              tma_load_2d(dst + (kStTiles + i) * kStRawTile, &sp.tmv, 0, rows[i], &full[slot],
-                          policy);
-            }
-          }
+          for (int i = 0; i < kStTiles; ++i)
+            if (i < n) tma_load_2d(dst + i * kStRawTile, map, 0, rows[i], &fullx[slot], policy);
           ++issued;
         }
       }
@@ -894,7 +918,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     }
     if (lane == 0) {  // no copy may still be landing when the CTA exits
       for (int i = max(0, issued - kStRing); i < issued; ++i)
-        if (!mbar_wait_bounded(&full[i % kStRing], (i / kStRing) & 1))
+        if (!mbar_wait_bounded(&fullx[i % kStRing], (i / kStRing) & 1))
           atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
     }
     __syncwarp();
@@ -908,7 +932,8 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       // 8-row groups 1024 B apart, term after term; P^T terms [128 tokens][16 B]
       // MN-major B, 8-token core matrices 128 B apart along K, terms 2 KB apart
       // along N.
-      const uint64_t kdesc = umma_smem_desc(smem_u32(raw), 16, 1024, kUmmaSwizzle128B);
+      const uint64_t kdesc = umma_smem_desc(smem_u32(rawk), 16, 1024, kUmmaSwizzle128B);
+      const uint64_t vdesc = umma_smem_desc(smem_u32(rawv), 16, 1024, kUmmaSwizzle128B);
       const uint64_t qdesc = umma_smem_desc(smem_u32(qop), 16, 1024, kUmmaSwizzle128B);
       const uint64_t pdesc = umma_smem_desc(smem_u32(pop), 128, kStTerm, 0);
       constexpr uint32_t kIdescS = umma_idesc_f16(0, 0, kStTokens, kSharedCols * NQ);
@@ -921,29 +946,30 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       while (ok && npv < nstages) {
         bool prog = false;
         if (ns < nstages && ns <= npv + 1 &&
-            mbar_test(&full[ns % kStRing], (ns / kStRing) & 1)) {
+            mbar_test(&fullk[ns % kStRing], (ns / kStRing) & 1)) {
           tcgen05_fence_after();
-          const uint64_t kd = kdesc + uint64_t(((ns % kStRing) * kStRawStage) >> 4);
+          const uint64_t kd = kdesc + uint64_t(((ns % kStRing) * kStRawHalf) >> 4);
           const uint32_t sb = tmem + kStTmemS + uint32_t(ns & 1) * (16 * 3);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)  // 32 dims per step, every Q term at once
             umma_f8_ss(sb, kd + uint64_t((ks * 32) >> 4), qdesc + uint64_t((ks * 32) >> 4),
                        kIdescS, ks > 0 ? 1u : 0u);
           umma_commit(&sfull[ns & 1]);
+          umma_commit(&emptyk[ns % kStRing]);  // the K slot is read
           ++ns;
           prog = true;
         }
-        if (npv < ns && mbar_test(pready, npv & 1)) {
+        if (npv < ns && mbar_test(pready, npv & 1) &&
+            mbar_test(&fullv[npv % kStRing], (npv / kStRing) & 1)) {
           tcgen05_fence_after();
-          const uint64_t vd = kdesc + uint64_t(((npv % kStRing) * kStRawStage +
-                                                kStTiles * kStRawTile) >> 4);
+          const uint64_t vd = vdesc + uint64_t(((npv % kStRing) * kStRawHalf) >> 4);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)  // 32 tokens per step, every P term at once
             umma_f8_ss(tmem + kStTmemO, vd + uint64_t((ks * 4096) >> 4),
                        pdesc + uint64_t((ks * 512) >> 4), kStIdescPV,
                        (npv > 0 || ks > 0) ? 1u : 0u);
           umma_commit(odone);
-          umma_commit(&empty[npv % kStRing]);  // the raw stage is read (S and P.V)
+          umma_commit(&emptyv[npv % kStRing]);  // the V slot is read
           ++npv;
           prog = true;
         }
@@ -955,7 +981,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
         if (npv < ns)
           mbar_try_wait(pready, npv & 1, 500);
         else
-          mbar_try_wait(&full[ns % kStRing], (ns / kStRing) & 1, 500);
+          mbar_try_wait(&fullk[ns % kStRing], (ns / kStRing) & 1, 500);
         if (idle == 0) t_idle = global_timer_ns();
         if ((++idle & 63) == 0 && global_timer_ns() - t_idle > kWaitLimitNs) ok = false;
       }
@@ -964,7 +990,9 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       if (!mbar_wait_bounded(done, 0)) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
     }
     __syncwarp();
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kStSoftmaxRegs));
     // ---------------- softmax warps: token row r of S^T, dim row r of O^T ----------------
     const int r = tid;                                       // 0..127
     const uint32_t tl = tmem + (uint32_t(32 * warp) << 16);  // this warp's lane quadrant
@@ -1129,9 +1157,11 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       for (int t = 0; t < kStPTerms; ++t)
         *reinterpret_cast<uint4*>(pop + t * kStTerm + r * 16) =
             make_uint4(pw[t][0], pw[t][1], pw[t][2], pw[t][3]);
-      if (!x.valid) {  // V rows past the context may hold anything, even NaN: zero them
-        uint8_t* vrow = raw + (st % kStRing) * kStRawStage + (kStTiles + (r >> 4)) * kStRawTile +
-                        (r & 15) * 128;
+      // V rows past the context may hold anything, even NaN: zero them once the
+      // stage's V has landed (its slot is not refilled before this P.V)
+      if (__any_sync(kFullMask, !x.valid)) wait(&fullv[st % kStRing], (st / kStRing) & 1);
+      if (!x.valid) {
+        uint8_t* vrow = rawv + (st % kStRing) * kStRawHalf + (r >> 4) * kStRawTile + (r & 15) * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0, 0, 0, 0);
       }
@@ -1292,24 +1322,36 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
   if (!encode_pool_map(&sp.tmk, a.key_cache, rows, fp8) ||
       !encode_pool_map(&sp.tmv, a.value_cache, rows, fp8))
     return PA_ERR_CUDA;
-  if (fp8) {  // the tensor-core kernel: no cluster split
-    sp.cluster = 1;
+  if (fp8 && (a.q_dtype == PA_F16 || a.q_dtype == PA_BF16)) {
+    // the tensor-core kernel: no cluster split.  Its register split assumes the CTA
+    // is launched with kStLaunchRegs a thread (a split above the launch's registers
+    // would wait forever); a build whose kernel has another count takes the
+    // mma.sync kernel below.  Checked once per kernel.
     const dim3 grid(unsigned(grid_x), unsigned(a.num_kv_heads));
-    if (a.q_dtype == PA_F16) {
-      constexpr size_t smem = shared_tc_smem_bytes<3>();
-      static std::atomic<unsigned long long> done_h{0};
-      if (set_smem_once(decode_shared_tc_kernel<__half>, smem, done_h) != PA_OK) return PA_ERR_CUDA;
-      decode_shared_tc_kernel<__half><<<grid, kStThreads, smem, stream>>>(sp);
-    } else if (a.q_dtype == PA_BF16) {
-      constexpr size_t smem = shared_tc_smem_bytes<2>();
-      static std::atomic<unsigned long long> done_b{0};
-      if (set_smem_once(decode_shared_tc_kernel<__nv_bfloat16>, smem, done_b) != PA_OK)
-        return PA_ERR_CUDA;
-      decode_shared_tc_kernel<__nv_bfloat16><<<grid, kStThreads, smem, stream>>>(sp);
-    } else {
-      return PA_ERR_UNSUPPORTED;
-    }
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    auto launch_tc = [&](auto kern, size_t smem, std::atomic<unsigned long long>& mask,
+                         std::atomic<int>& regs) -> int {
+      int r = regs.load(std::memory_order_relaxed);
+      if (r == 0) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return PA_ERR_CUDA;
+        r = fa.numRegs == kStLaunchRegs ? 1 : -1;
+        regs.store(r, std::memory_order_relaxed);
+      }
+      if (r < 0) return PA_ERR_UNSUPPORTED;
+      SharedParams tcp = sp;
+      tcp.cluster = 1;
+      if (set_smem_once(kern, smem, mask) != PA_OK) return PA_ERR_CUDA;
+      kern<<<grid, kStThreads, smem, stream>>>(tcp);
+      return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    };
+    static std::atomic<unsigned long long> done_h{0}, done_b{0};
+    static std::atomic<int> regs_h{0}, regs_b{0};
+    const int rc = a.q_dtype == PA_F16
+                       ? launch_tc(decode_shared_tc_kernel<__half>, shared_tc_smem_bytes<3>(),
+                                   done_h, regs_h)
+                       : launch_tc(decode_shared_tc_kernel<__nv_bfloat16>,
+                                   shared_tc_smem_bytes<2>(), done_b, regs_b);
+    if (rc != PA_ERR_UNSUPPORTED) return rc;
   }
   if (a.cache_dtype == PA_F16 && a.q_dtype == PA_F16)
     return launch_shared_typed<__half, __half>(sp, int(grid_x), stream);
