@@ -21,6 +21,12 @@
  *     range-checked on the device.  A bad value never faults: the access is
  *     clamped or skipped, the result of that item is unspecified, and a bit is set
  *     in a device error word that pa_get_device_error() reads and clears.
+ *   - Two kernels (the E4M3 shared-prefix decode and the chunked prefill over two
+ *     or more 128-row tiles per sequence and kv head) move registers between warp
+ *     groups and check once that their build has the register count this assumes;
+ *     otherwise the call takes a slower kernel of the same result (mma.sync, and
+ *     one tile per CTA).  PA_FALLBACK_KERNELS=1 in the environment, read at each
+ *     call, selects those kernels regardless.
  *
  * Cache layout (one layer): key_cache and value_cache are each
  *   [num_blocks][num_kv_heads][block_size][head_dim]

@@ -6,6 +6,7 @@
 // over such a group reads each shared block once for all of its members; the result
 // is the per-sequence decode's ("vLLM 推理优化技术深度调研报告" sec 3 formulas 3, 4).
 
+#include "pa_fallback.h"
 #include "pa_kernels.cuh"
 #include "pa_tcgen05.cuh"
 
@@ -1322,7 +1323,7 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
   if (!encode_pool_map(&sp.tmk, a.key_cache, rows, fp8) ||
       !encode_pool_map(&sp.tmv, a.value_cache, rows, fp8))
     return PA_ERR_CUDA;
-  if (fp8 && (a.q_dtype == PA_F16 || a.q_dtype == PA_BF16)) {
+  if (fp8 && (a.q_dtype == PA_F16 || a.q_dtype == PA_BF16) && !fallback_kernels_forced()) {
     // the tensor-core kernel: no cluster split.  Its register split assumes the CTA
     // is launched with kStLaunchRegs a thread (a split above the launch's registers
     // would wait forever); a build whose kernel has another count takes the

@@ -2,6 +2,7 @@
 // for sm_100a: a 64-row mma.sync kernel for short chunks and a persistent
 // 128-row tcgen05 kernel (TMEM accumulators) for the rest.
 
+#include "pa_fallback.h"
 #include "pa_kernels.cuh"
 #include "pa_tcgen05.cuh"
 
@@ -1410,7 +1411,7 @@ int launch_prefill(const DecodeArgs& a, const int32_t* query_start, int max_quer
     // two 128-row tiles of one (sequence, kv head) per CTA at a time, when a
     // (sequence, kv head) has two: the other warpgroup would idle otherwise
     const int64_t pairs = int64_t(a.num_seqs) * a.num_kv_heads * ((tp.row_blocks + 1) / 2);
-    if (tp.row_blocks >= 2 && pairs <= INT32_MAX) {
+    if (tp.row_blocks >= 2 && pairs <= INT32_MAX && !fallback_kernels_forced()) {
       const unsigned grid_pp = unsigned(pairs < sms ? pairs : sms);
       constexpr size_t smem_pp = pp_prefill_smem_bytes();
       // The register split assumes the CTA is launched with kPpLaunchRegs a thread
