@@ -896,26 +896,24 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
         ent = resolve();
         fetch((st + 4) * kStTiles + lane);
       }
-      int rows[kStTiles];
-#pragma unroll
-      for (int i = 0; i < kStTiles; ++i) rows[i] = __shfl_sync(kFullMask, ent, (st & 3) * kStTiles + i);
+      // lane i (< 8) loads tile i of the stage: the copies of a stage leave in one
+      // instruction of 8 lanes (a copy costs its issuing thread far more than the
+      // instruction does, so lanes issuing together keep many more in flight)
+      const int row = __shfl_sync(kFullMask, ent, (st & 3) * kStTiles + (lane & (kStTiles - 1)));
       const int slot = st % kStRing;
-      if (lane == 0) {
-        if (st >= kStRing && !mbar_wait_bounded(&emptyx[slot], ((st / kStRing) - 1) & 1)) {
-          atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
-          ok = false;
-        }
-        if (ok) {
-          const int n = min(kStTiles, ntotal - st * kStTiles);
-          uint8_t* dst = ring + slot * kStRawHalf;
-          mbar_arrive_expect_tx(&fullx[slot], uint32_t(n) * kStRawTile);
-#pragma unroll
-          for (int i = 0; i < kStTiles; ++i)
-            if (i < n) tma_load_2d(dst + i * kStRawTile, map, 0, rows[i], &fullx[slot], policy);
-          ++issued;
-        }
+      if (lane == 0 && st >= kStRing &&
+          !mbar_wait_bounded(&emptyx[slot], ((st / kStRing) - 1) & 1)) {
+        atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
+        ok = false;
       }
       ok = __shfl_sync(kFullMask, ok, 0);
+      if (!ok) break;
+      const int n = min(kStTiles, ntotal - st * kStTiles);
+      if (lane == 0) mbar_arrive_expect_tx(&fullx[slot], uint32_t(n) * kStRawTile);
+      __syncwarp();
+      if (lane < n)
+        tma_load_2d(ring + slot * kStRawHalf + lane * kStRawTile, map, 0, row, &fullx[slot], policy);
+      ++issued;
     }
     if (lane == 0) {  // no copy may still be landing when the CTA exits
       for (int i = max(0, issued - kStRing); i < issued; ++i)
