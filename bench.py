@@ -404,94 +404,92 @@ def pipelined_e2e(dev, stream, inputs, host_src, out, run_step, steps, world):
 
 
 # ---------------------------------------------------------------- GPU arm
-def timed_loop(step, launches, steps, warmup, dev, stream, world, rank):
+def timed_loop(step, launches, steps, warmup, dev, stream, world, rank, writes_step=None):
     """`warmup` untimed steps, then exactly `steps` timed ones bracketed by a
     barrier and a device synchronize on both sides, with clocks sampled meanwhile
-    on rank 0.  step(timed) appends its hot launch's (start, end) events to
-    `launches` when timed.  Returns (max-over-ranks elapsed ms, mean launch ms,
-    clock summary or None)."""
-    for _ in range(warmup):
-        step(False)
-    torch.cuda.synchronize(dev)
+    on rank 0.  With writes_step (CUDA-graph steps) a second region of `steps`
+    replays of the step's cache writes alone follows, bracketed the same way, and a
+    hot launch's time is the difference of the two regions' per-step times;
+    otherwise step(timed) appends its hot launch's (start, end) events to
+    `launches` when timed.  Returns (max-over-ranks elapsed ms, launch ms, clock
+    summary or None)."""
     import paged_kv_cache_413_b200 as pa
 
+    def region(fn, sampled):
+        sampler = ClockSampler(dev.index) if (rank == 0 and sampled) else None
+        if sampler:
+            sampler.__enter__()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            fn(True)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        if sampler:
+            sampler.__exit__(None, None, None)
+        if pa.pa_get_device_error() != 0:
+            raise RuntimeError("device error bits set during the timed steps")
+        return t0.elapsed_time(t1), (sampler.summary() if sampler else None)
+
+    for _ in range(warmup):
+        step(False)
+        if writes_step is not None:
+            writes_step(False)
+    torch.cuda.synchronize(dev)
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error bits set during warm-up")
-    sampler = ClockSampler(dev.index) if rank == 0 else None
-    if sampler:
-        sampler.__enter__()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches.clear()
-    t0.record(stream)
-    for _ in range(steps):
-        step(True)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    if sampler:
-        sampler.__exit__(None, None, None)
-    if pa.pa_get_device_error() != 0:
-        raise RuntimeError("device error bits set during the timed steps")
-    elapsed_ms = t0.elapsed_time(t1)
-    pairs = {id(e0): (e0, e1) for e0, e1 in launches}  # a pair replayed twice: its last
-    launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in pairs.values())
+    elapsed_ms, clocks = region(step, True)
+    if writes_step is not None:
+        writes_ms, _ = region(writes_step, False)
+        launch_ms = max(elapsed_ms - writes_ms, 0.0) / steps
+    else:
+        pairs = {id(e0): (e0, e1) for e0, e1 in launches}
+        launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in pairs.values())
     elapsed_ms, launch_ms = max_over_ranks([elapsed_ms, launch_ms], world, dev)
-    return elapsed_ms, launch_ms, (sampler.summary() if sampler else None)
+    return elapsed_ms, launch_ms, clocks
 
 
 def timing_note(args) -> str:
     if args.no_graphs:
-        return "each timed step calls the library from Python (host launch overhead included)"
+        return ("each timed step calls the library from Python (host launch overhead "
+                "included); the launch time brackets the hot kernels with CUDA events")
     return ("each timed step replays one CUDA graph of the library's calls (cache writes, then "
-            "the hot kernels); the step time brackets the steps with CUDA events on the stream, "
-            "the launch time brackets the hot kernels with event record nodes inside the graph")
-
-
-MAX_HOT_GRAPHS = 200
+            "the hot kernels), bracketed as a whole by CUDA events on the stream; the launch "
+            "time is the step time minus that of as many replays of a graph of the writes "
+            "alone (timing events inside a graph would add ~4 us to what they bracket)")
 
 
 def graph_step(writes, hot, run_step, inputs, out, ev, dev, stream, args):
-    """The step the timed loop runs.  By default each step replays one CUDA graph
-    captured from the same library calls: the cache writes (and copies), then the
-    hot kernel(s) between a pair of timing events recorded as event nodes of the
-    graph, so host-side call overhead never idles the GPU inside the timed region and
-    a launch's time is the hot kernels' (their launch prepared while the writes run).
-    One graph per timed step (up to MAX_HOT_GRAPHS, replayed in turn) keeps every
-    timed step's pair apart.  With --no-graphs the step calls the library directly
-    (run_step)."""
+    """The steps the timed loop runs: (step, writes_step).  By default the step
+    replays one CUDA graph captured from the same library calls -- the cache writes
+    (and copies), then the hot kernel(s) -- so host-side call overhead never idles
+    the GPU inside the timed region, and writes_step replays a graph of the writes
+    alone, which the timed loop subtracts to get the hot launches' time (an event
+    record node inside a graph adds ~4 us to the interval it brackets, which is why
+    the graph holds none).  With --no-graphs the step calls the library directly
+    (run_step, events around the hot call) and writes_step is None."""
     if args.no_graphs:
-        return lambda timed: run_step(inputs, out, timed)
+        return (lambda timed: run_step(inputs, out, timed)), None
     run_step(inputs, out, False)          # warm: every kernel attribute set, maps encoded
     torch.cuda.synchronize(dev)
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
-    graphs = []
-    for _ in range(max(1, min(args.steps, MAX_HOT_GRAPHS))):
-        g = torch.cuda.CUDAGraph()
-        e0 = torch.cuda.Event(enable_timing=True, external=True)
-        e1 = torch.cuda.Event(enable_timing=True, external=True)
-        with torch.cuda.graph(g, stream=side):
-            writes()
-            e0.record(side)
-            hot()
-            e1.record(side)
-        graphs.append((g, e0, e1))
+    g_step, g_writes = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=side):
+        writes()
+        hot()
+    with torch.cuda.graph(g_writes, stream=side):
+        writes()
     stream.wait_stream(side)
     torch.cuda.synchronize(dev)
-    count = [0]
-
-    def step(timed):
-        g, e0, e1 = graphs[count[0] % len(graphs)]
-        count[0] += 1
-        g.replay()
-        if timed:
-            ev.append((e0, e1))
-
-    return step
+    graphs = (g_step, g_writes)  # kept alive with the closures
+    return (lambda timed: graphs[0].replay()), (lambda timed: graphs[1].replay())
 
 
 def decode_case(cfg, dev, args, world, rank, decode_mode="auto", partition=None,
@@ -564,10 +562,10 @@ def decode_case(cfg, dev, args, world, rank, decode_mode="auto", partition=None,
             e1.record(stream)
             ev.append((e0, e1))
 
-    step = graph_step(lambda: writes(inputs), lambda: decode(inputs, out), run_step, inputs,
-                      out, ev, dev, stream, args)
+    step, writes_step = graph_step(lambda: writes(inputs), lambda: decode(inputs, out),
+                                   run_step, inputs, out, ev, dev, stream, args)
     elapsed_ms, decode_ms, clocks = timed_loop(step, ev, args.steps, args.warmup, dev, stream,
-                                               world, rank)
+                                               world, rank, writes_step)
     dec_b = shared_decode_bytes(wl, out_dtype) if shared else decode_bytes(wl, out_dtype)
     step_bytes = dec_b + cache_write_bytes(wl) + copy_bytes(wl)
     res = {"wl": wl, "shared": shared, "part_eff": part_eff, "dec_b": dec_b,
@@ -866,12 +864,21 @@ def prefill_flops(wl: W.Workload) -> int:
     return pairs * cfg.num_heads * cfg.head_dim * 4
 
 
-def tensor_peak():
+# A timed region at least this long is a sustained run: its tensor-core kernel is
+# held against the sustained peak (cuBLAS back to back for seconds, under the power
+# cap), a shorter one against the burst peak.
+SUSTAINED_REGION_S = 1.0
+
+
+def tensor_peaks():
+    """(burst, sustained) dense bf16 TFLOP/s and their description."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
-            return float(json.load(fh)["bf16_tflops"]), "measured (bf16_tflops, cuBLAS burst)"
+            m = json.load(fh)
+        return (float(m["bf16_tflops"]), float(m.get("bf16_tflops_sustained", m["bf16_tflops"])),
+                "measured")
     except Exception:
-        return 1590.0, "fallback"
+        return 1590.0, 1400.0, "fallback"
 
 
 def prefill_case(name, dev, args, world, rank, with_e2e=True, with_cpu=False):
@@ -910,10 +917,10 @@ def prefill_case(name, dev, args, world, rank, with_e2e=True, with_cpu=False):
             e1.record(stream)
             ev.append((e0, e1))
 
-    step = graph_step(lambda: writes(inputs), lambda: attend(inputs, out), run_step, inputs,
-                      out, ev, dev, stream, args)
+    step, writes_step = graph_step(lambda: writes(inputs), lambda: attend(inputs, out),
+                                   run_step, inputs, out, ev, dev, stream, args)
     elapsed_ms, kern_ms, clocks = timed_loop(step, ev, args.steps, args.warmup, dev, stream,
-                                             world, rank)
+                                             world, rank, writes_step)
     cfg = wl.cfg
     L = wl.seq_lens.numpy().astype(np.int64)
     res = {"wl": wl, "elapsed_ms": elapsed_ms, "kern_ms": kern_ms, "clocks": clocks,
@@ -934,7 +941,15 @@ def prefill_case(name, dev, args, world, rank, with_e2e=True, with_cpu=False):
 
 def prefill_roofline(name, p):
     cfg = p["wl"].cfg
-    peak, kind = tensor_peak()
+    burst, sustained, src = tensor_peaks()
+    region_s = p["elapsed_ms"] * 1e-3
+    if region_s >= SUSTAINED_REGION_S:
+        peak = sustained
+        kind = (f"{src} (bf16_tflops_sustained, cuBLAS back to back under the power cap: the "
+                f"timed region ran {region_s:.1f} s of back-to-back steps)")
+    else:
+        peak = burst
+        kind = f"{src} (bf16_tflops, cuBLAS burst: the timed region ran {region_s:.2f} s)"
     # the launcher's rule: 128-row tcgen05 tiles once a chunk fills one, two of them
     # in ping-pong once a (sequence, kv head) has two
     rows = p["max_q"] * (cfg.num_heads // cfg.num_kv_heads)
@@ -945,6 +960,7 @@ def prefill_roofline(name, p):
     achieved = p["flops"] / (p["kern_ms"] * 1e-3) / 1e12
     return {"bound": "tensor", "kernel": kernel, "achieved": round(achieved, 2), "peak": peak,
             "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "frac_of_burst": round(achieved / burst, 4),
             "traffic": recorded_traffic(name), "launch_ms": round(p["kern_ms"], 5),
             "flops_per_launch": p["flops"],
             "hbm_gbs": round((p["kv_bytes"] + p["qo_bytes"]) / (p["kern_ms"] * 1e-3) / 1e9, 1)}
@@ -954,8 +970,8 @@ def prefill_entry(name, p, steps, world):
     roof = prefill_roofline(name, p)
     return {"workload": f"{name}: {DESCR[name]}", "launch_ms": roof["launch_ms"],
             "flops_per_launch": p["flops"], "achieved_tflops": roof["achieved"],
-            "frac": roof["frac"], "peak": roof["peak"], "peak_kind": roof["peak_kind"],
-            "traffic": roof["traffic"], "kernel": roof["kernel"],
+            "frac": roof["frac"], "frac_of_burst": roof["frac_of_burst"], "peak": roof["peak"],
+            "peak_kind": roof["peak_kind"], "traffic": roof["traffic"], "kernel": roof["kernel"],
             "step_value": round(p["flops"] * world * steps / (p["elapsed_ms"] * 1e-3) / 1e12, 2),
             "unit": "TFLOP/s", "ms_per_step": round(p["elapsed_ms"] / steps, 5), "steps": steps,
             "gpu_launches": 2 * steps, "clocks": p["clocks"]}
