@@ -774,6 +774,41 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     for (int jj = 0; jj < kSharedCols; ++jj)
       if (jj < nseq) nx[jj] = p.block_tables[int64_t(s0 + jj) * p.max_blocks_per_seq + e];
   }
+  // Stage 0 leaves as soon as those entries are in.  The stream's first tiles are
+  // member 0's logical tiles 0, 1, ... (its prefix tiles, then its own), so while
+  // member 0 holds kStTiles tiles or more the first stage is its tiles 0 ..
+  // kStTiles - 1 whatever the prefix length.  Each producer initialises its own
+  // ring's barriers and issues that stage here, before the lengths are checked
+  // and the CTA synchronises; its loop below skips the stage.  The checks of the
+  // same entries (block range, the prefix promise) still run there.
+  bool early = false;
+  if (warp == kStKWarp || warp == kStVWarp) {
+    const bool is_k = warp == kStKWarp;
+    uint64_t* fullx = is_k ? fullk : fullv;
+    uint64_t* emptyx = is_k ? emptyk : emptyv;
+    if (lane == 0) {
+      for (int i = 0; i < kStRing; ++i) {
+        mbar_init(&fullx[i], 1);
+        mbar_init(&emptyx[i], 1);
+      }
+      fence_barrier_init();
+    }
+    const int L0 = p.seq_lens[s0];
+    const int32_t phys = spec ? nx[0] : -1;
+    const bool in_range = lane >= kStTiles || (spec && phys >= 0 && phys < p.num_blocks);
+    early = L0 > (kStTiles - 1) * kBlockSize && L0 <= p.cap && __all_sync(kFullMask, in_range);
+    if (early) {
+      const int e = lane / p.tiles_per_block;
+      const int row =
+          ((phys * p.num_kv_heads + kvh) * p.tiles_per_block + (lane - e * p.tiles_per_block)) *
+          kBlockSize;
+      if (lane == 0) mbar_arrive_expect_tx(&fullx[0], uint32_t(kStTiles) * kStRawTile);
+      __syncwarp();
+      if (lane < kStTiles)
+        tma_load_2d((is_k ? rawk : rawv) + lane * kStRawTile, is_k ? &sp.tmk : &sp.tmv, 0, row,
+                    &fullx[0], l2_policy_evict_first());
+    }
+  }
   // lengths and the shared prefix (device data: checked), as the mma.sync kernel;
   // every read is issued before the first check, whose error report would order
   // the reads after it one by one
@@ -805,12 +840,6 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       if (j < nseq) pos += (own_len[j] + kBlockSize - 1) / kBlockSize - pb;
     }
     own_start[kSharedCols] = pos;
-    for (int i = 0; i < kStRing; ++i) {
-      mbar_init(&fullk[i], 1);
-      mbar_init(&fullv[i], 1);
-      mbar_init(&emptyk[i], 1);
-      mbar_init(&emptyv[i], 1);
-    }
     mbar_init(&sfull[0], 1);
     mbar_init(&sfull[1], 1);
     mbar_init(pready, kStQuads);
@@ -909,10 +938,13 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       ok = __shfl_sync(kFullMask, ok, 0);
       if (!ok) break;
       const int n = min(kStTiles, ntotal - st * kStTiles);
-      if (lane == 0) mbar_arrive_expect_tx(&fullx[slot], uint32_t(n) * kStRawTile);
-      __syncwarp();
-      if (lane < n)
-        tma_load_2d(ring + slot * kStRawHalf + lane * kStRawTile, map, 0, row, &fullx[slot], policy);
+      if (st > 0 || !early) {  // stage 0 may have left before the CTA synchronised
+        if (lane == 0) mbar_arrive_expect_tx(&fullx[slot], uint32_t(n) * kStRawTile);
+        __syncwarp();
+        if (lane < n)
+          tma_load_2d(ring + slot * kStRawHalf + lane * kStRawTile, map, 0, row, &fullx[slot],
+                      policy);
+      }
       ++issued;
     }
     if (lane == 0) {  // no copy may still be landing when the CTA exits
