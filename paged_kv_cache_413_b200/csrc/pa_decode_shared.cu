@@ -1261,10 +1261,38 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       for (int n = 0; n < kSharedCols; ++n)
         o[n] = fmaf(fmaf(ot[2][n], 0.0625f, ot[1][n]), 0.0625f, ot[0][n]);
     }
+    // Thread r holds dim r of every column.  With a 16-byte aligned output the
+    // values go through shared memory (the K ring: every S has completed, every K
+    // copy has landed) so that each thread then writes 16-byte pieces of the
+    // columns' output rows instead of one element of each.
+    if ((reinterpret_cast<uintptr_t>(p.out) & 15u) == 0) {  // uniform
+      const int ob = p.out_dtype == PA_F32 ? 4 : 2;
+      uint8_t* ost = rawk;
 #pragma unroll
-    for (int n = 0; n < kSharedCols; ++n) {
-      const int64_t base = ebase[n];
-      if (base >= 0) store_out(p.out, base + r, o[n] * einv[n], p.out_dtype);
+      for (int n = 0; n < kSharedCols; ++n) {
+        const float v = o[n] * einv[n];
+        if (p.out_dtype == PA_F32)
+          reinterpret_cast<float*>(ost)[n * D + r] = v;
+        else if (p.out_dtype == PA_F16)
+          reinterpret_cast<__half*>(ost)[n * D + r] = __float2half_rn(v);
+        else
+          reinterpret_cast<__nv_bfloat16*>(ost)[n * D + r] = __float2bfloat16_rn(v);
+      }
+      named_bar_sync(1, kStQuads * 32);
+      const int per_col = D * ob / 16;  // 16-byte pieces of one column's output row
+      for (int c = r; c < kSharedCols * per_col; c += kStQuads * 32) {
+        const int n = c / per_col, k = c - n * per_col;
+        const int64_t base = ebase[n];
+        if (base >= 0)
+          *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + base * ob + k * 16) =
+              *reinterpret_cast<const uint4*>(ost + n * D * ob + k * 16);
+      }
+    } else {
+#pragma unroll
+      for (int n = 0; n < kSharedCols; ++n) {
+        const int64_t base = ebase[n];
+        if (base >= 0) store_out(p.out, base + r, o[n] * einv[n], p.out_dtype);
+      }
     }
     if (!ok && lane == 0) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
   }
