@@ -1261,11 +1261,11 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       for (int n = 0; n < kSharedCols; ++n)
         o[n] = fmaf(fmaf(ot[2][n], 0.0625f, ot[1][n]), 0.0625f, ot[0][n]);
     }
-    // Thread r holds dim r of every column.  With a 16-byte aligned output the
-    // values go through shared memory (the K ring: every S has completed, every K
-    // copy has landed) so that each thread then writes 16-byte pieces of the
-    // columns' output rows instead of one element of each.
-    if ((reinterpret_cast<uintptr_t>(p.out) & 15u) == 0) {  // uniform
+    // Thread r holds dim r of every column.  The values go through shared memory
+    // (the K ring: every S has completed, every K copy has landed) so that each
+    // thread then writes 16-byte pieces of the columns' output rows instead of one
+    // element of each (the entry point accepts only a 16-byte aligned output).
+    {
       const int ob = p.out_dtype == PA_F32 ? 4 : 2;
       uint8_t* ost = rawk;
 #pragma unroll
@@ -1286,12 +1286,6 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
         if (base >= 0)
           *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + base * ob + k * 16) =
               *reinterpret_cast<const uint4*>(ost + n * D * ob + k * 16);
-      }
-    } else {
-#pragma unroll
-      for (int n = 0; n < kSharedCols; ++n) {
-        const int64_t base = ebase[n];
-        if (base >= 0) store_out(p.out, base + r, o[n] * einv[n], p.out_dtype);
       }
     }
     if (!ok && lane == 0) atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);

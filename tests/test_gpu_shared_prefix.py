@@ -179,3 +179,34 @@ def test_fp8_persistent_walk_many_units_and_empty_contexts(qdt):
     ref = flow.oracle_decode(wl, kc, vc, rest)
     err = flow.max_abs_err(out[torch.as_tensor(rest, device="cuda")], ref)
     assert err <= flow.TOL["f32"], f"max abs error {err:.3e}"
+
+
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
+def test_fp8_unaligned_output_is_rejected(out_dtype):
+    """The tensor-core kernel writes its outputs in 16-byte pieces; the entry point
+    takes only 16-byte aligned data pointers and refuses an output that starts one
+    element past a boundary before anything is launched (the output stays as it
+    was), then decodes the same batch into an aligned output."""
+    wl = W.make_group_workload(12, (1, 5), (1, 4), (1, 40), num_heads=32, num_kv_heads=8,
+                               dtype="bf16", seed=37, cache_dtype="e4m3")
+    d = flow.to_device(wl)
+    pa.pa_reshape_and_cache(d.new_key, d.new_value, d.key_cache, d.value_cache, d.slot_mapping,
+                            k_scale=wl.k_scale, v_scale=wl.v_scale)
+    dt = flow.TORCH_DT[out_dtype]
+    flat = torch.full((d.query.numel() + 1,), 7.0, dtype=dt, device="cuda")
+    out = flat[1:].view(d.query.shape)
+    assert out.data_ptr() % 16 != 0
+    gs, pl = wl.group_starts.cuda(), wl.prefix_lens.cuda()
+    with pytest.raises(pa.PaError, match="INVALID_ARG"):
+        pa.pa_paged_attention_decode_shared_prefix(
+            out, d.query, d.key_cache, d.value_cache, d.block_tables, d.seq_lens, gs, pl,
+            max_seq_len=flow.max_seq_len(wl), max_group_size=int((gs[1:] - gs[:-1]).max()),
+            scale=wl.scale, k_scale=wl.k_scale, v_scale=wl.v_scale)
+    torch.cuda.synchronize()
+    assert torch.all(flat == 7.0)
+    got = _run_shared(wl, d, out_dtype)
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error() == 0
+    kc, vc = flow.oracle_caches(wl)
+    err = flow.max_abs_err(got, flow.oracle_decode(wl, kc, vc, None))
+    assert err <= flow.TOL[out_dtype], f"max abs error {err:.3e}"
