@@ -95,3 +95,16 @@ def test_committed_traffic_records_are_complete():
         assert int(r["dram_bytes_per_launch"]) > 0
         assert os.path.exists(os.path.join(bench.ROOT, "profiles", r["summary"])), name
         assert "ncu" in r["command"] and "--clock-control none" in r["command"]
+
+
+def test_committed_traffic_records_match_the_sources():
+    """No committed record is stale: the sources of every workload's captured kernel
+    still hash to the value recorded with its ncu capture, so bench.py reports each
+    traffic figure (a kernel edit without a new capture fails here)."""
+    import json
+
+    with open(bench.TRAFFIC_JSON) as f:
+        names = list(json.load(f)["workloads"])
+    assert names
+    for name in names:
+        assert bench.recorded_traffic(name) is not None, f"{name}: sources changed since the capture"
