@@ -905,7 +905,7 @@ __host__ __device__ constexpr uint32_t pp_tmem_o(int x) { return 256 + uint32_t(
 
 constexpr size_t pp_prefill_smem_bytes() {
   return 1024 + 2 * size_t(kTcStages) * kTcTileBytes + 2 * size_t(kPpQBytes) +
-         (4 * kTcStages + 9) * sizeof(uint64_t) + 16;
+         (4 * kTcStages + 11) * sizeof(uint64_t) + 16;
 }
 static_assert(kTcKv == 128, "one S buffer of 128 columns per tile");
 static_assert(pp_prefill_smem_bytes() <= 227 * 1024, "rings and Q fit 227 KB");
@@ -963,7 +963,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   uint64_t* o_full = s_full + 2;          // [2]: P.V of the tile's stage done
   uint64_t* p_ready = o_full + 2;         // [2]: P in TMEM, O rescaled (4 warps)
   uint64_t* q_ready = p_ready + 2;        // [2]: Q of the tile's pair in smem (4 warps)
-  uint64_t* done = q_ready + 2;
+  uint64_t* p_half = q_ready + 2;         // [2]: P of keys 0 .. 63 in TMEM (4 warps)
+  uint64_t* done = p_half + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -979,6 +980,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       mbar_init(&o_full[x], 1);
       mbar_init(&p_ready[x], 4);
       mbar_init(&q_ready[x], 4);
+      mbar_init(&p_half[x], 4);
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -1081,19 +1083,23 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         }
         umma_commit(&s_full[xt]);
       };
-      auto issue_pv = [&](int xt, int gs, int jb) {  // O_xt += P_xt . V(stage gs)
+      // O_xt += P_xt . V(stage gs) over keys 64 h .. 64 h + 63: the first half can
+      // start while the softmax is still writing the second
+      auto issue_pv = [&](int xt, int gs, int jb, int h) {
         tcgen05_fence_after();
         const uint64_t vd = vdesc0 + uint64_t(((gs % kTcStages) * kTcTileBytes) >> 4);
         const uint32_t pt = tmem + pp_tmem_s(xt);
 #pragma unroll
         for (int t = 0; t < (kSplitP ? 2 : 1); ++t) {
 #pragma unroll
-          for (int ks = 0; ks < kTcKv / 16; ++ks)
+          for (int kk = 0; kk < kTcKv / 32; ++kk) {
+            const int ks = h * (kTcKv / 32) + kk;
             umma_f16_ts(tmem + pp_tmem_o(xt), pt + uint32_t(t * (kTcKv / 2) + ks * 8),
                         vd + uint64_t((ks * 2048) >> 4), kIdescPV,
                         (jb > 0 || t > 0 || ks > 0) ? 1u : 0u);
+          }
         }
-        umma_commit(&o_full[xt]);
+        if (h == 1) umma_commit(&o_full[xt]);
       };
       int pair = -1;
       PpPair x;
@@ -1112,10 +1118,12 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           bool vwaited = false, kwaited = false;
           // P.V_A(jb), then S_A(jb + 1)
           if (in(0, jb)) {
-            if (!wait(&p_ready[0], cnt[0] & 1)) break;
+            if (!wait(&p_half[0], cnt[0] & 1)) break;
             if (!wait(&vfull[g % kTcStages], (g / kTcStages) & 1)) break;
             vwaited = true;
-            issue_pv(0, g, jb);
+            issue_pv(0, g, jb, 0);
+            if (!wait(&p_ready[0], cnt[0] & 1)) break;
+            issue_pv(0, g, jb, 1);
             ++cnt[0];
           }
           if (jb + 1 < nkb && in(0, jb + 1)) {
@@ -1125,9 +1133,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           }
           // P.V_B(jb), then S_B(jb + 1)
           if (in(1, jb)) {
-            if (!wait(&p_ready[1], cnt[1] & 1)) break;
+            if (!wait(&p_half[1], cnt[1] & 1)) break;
             if (!vwaited && !wait(&vfull[g % kTcStages], (g / kTcStages) & 1)) break;
-            issue_pv(1, g, jb);
+            issue_pv(1, g, jb, 0);
+            if (!wait(&p_ready[1], cnt[1] & 1)) break;
+            issue_pv(1, g, jb, 1);
             ++cnt[1];
           }
           umma_commit(&vempty[g % kTcStages]);  // the V stage's last P.V is issued
@@ -1247,8 +1257,27 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         const float2 me2 = make_float2(me, me), nmu2 = make_float2(-mu, -mu);
         float2 a4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
+        // The pair's last stage: V rows past its last visible token may be stale or
+        // NaN.  The tile whose P.V reads that stage first zeroes them (tile A if it
+        // takes part in the stage), before any of its P is announced.
+        if (jb == x.nkb - 1 && (xt == 0 || t.nkb != x.t[0].nkb || !x.has[0])) {
+          const int gs = gp + jb;
+          wait(&vfull[gs % kTcStages], (gs / kTcStages) & 1);
+          if (ok && jb * kTcKv + r > x.pos_last) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint8_t* vrow = vsm + (gs % kTcStages) * kTcTileBytes + half * (kTcTileBytes / 2) +
+                              r * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+            }
+          }
+          fence_proxy_async_smem();
+        }
         // exponentials, then P over S as 16-bit pairs: chunk q's hi term into columns
-        // [16 q, 16 q + 16), its lo term into [64 + 16 q, ...) (S is all in registers)
+        // [16 q, 16 q + 16), its lo term into [64 + 16 q, ...) (S is all in registers);
+        // keys 0 .. 63 are announced on their own, so that their P.V can start
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t pw[16];
@@ -1272,27 +1301,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             }
             tmem_st16(sb + kTcKv / 2 + 16 * q, lw);
           }
+          if (q == 1) {
+            tmem_wait_st();
+            arrive(&p_half[xt]);
+          }
         }
         const float2 a2 = add2(add2(a4[0], a4[1]), add2(a4[2], a4[3]));
         l += a2.x + a2.y;
-        // The pair's last stage: V rows past its last visible token may be stale or
-        // NaN.  The tile whose P.V reads that stage first zeroes them (tile A if it
-        // takes part in the stage), before its P is announced.
-        if (jb == x.nkb - 1 && (xt == 0 || t.nkb != x.t[0].nkb || !x.has[0])) {
-          const int gs = gp + jb;
-          wait(&vfull[gs % kTcStages], (gs / kTcStages) & 1);
-          if (ok && jb * kTcKv + r > x.pos_last) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              uint8_t* vrow = vsm + (gs % kTcStages) * kTcTileBytes + half * (kTcTileBytes / 2) +
-                              r * 128;
-#pragma unroll
-              for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
-            }
-          }
-          fence_proxy_async_smem();
-        }
         tmem_wait_st();
         arrive(&p_ready[xt]);
       }
