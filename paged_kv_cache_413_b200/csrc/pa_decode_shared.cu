@@ -652,7 +652,7 @@ constexpr uint32_t kStIdescPV = umma_idesc_f16_ab(0, 1, 1, 128, kSharedCols * kS
 template <int NQ>
 constexpr size_t shared_tc_smem_bytes() {
   return 1024 + size_t(2 * kStRing) * kStRawHalf + size_t(NQ + kStPTerms) * kStTerm +
-         (kStRing * 4 + 8) * sizeof(uint64_t) +
+         (kStRing * 4 + 10) * sizeof(uint64_t) +
          (8 + 2 * kStQuads * kSharedCols + kStQuads * kSharedCols + kSharedCols) * 4 +
          (2 * (kSharedCols + 1) + 2) * 4;
 }
@@ -733,7 +733,8 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   uint64_t* odone = pready + 1;                         // P.V of stage st done
   uint64_t* qready = odone + 1;                         // Q^T terms written
   uint64_t* done = qready + 1;                          // every MMA done
-  int* flags = reinterpret_cast<int*>(done + 2);        // [2][4] rescale votes
+  uint64_t* sread = done + 1;                           // [2] S buffer b read by the softmax
+  int* flags = reinterpret_cast<int*>(sread + 3);       // [2][4] rescale votes
   float* wmax = reinterpret_cast<float*>(flags + 8);    // [2][4][16] warp column maxima
   float* lsum = wmax + 2 * kStQuads * kSharedCols;      // [4][16] warp column sums
   float* colmult = lsum + kStQuads * kSharedCols;       // [16] score multiplier per column
@@ -846,6 +847,8 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     mbar_init(odone, 1);
     mbar_init(qready, kStQuads);
     mbar_init(done, 1);
+    mbar_init(&sread[0], kStQuads);
+    mbar_init(&sread[1], kStQuads);
     fence_barrier_init();
   }
   if (warp == kStMmaWarp) {  // the MMA warp owns the TMEM allocation
@@ -930,7 +933,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       // instruction does, so lanes issuing together keep many more in flight)
       const int row = __shfl_sync(kFullMask, ent, (st & 3) * kStTiles + (lane & (kStTiles - 1)));
       const int slot = st % kStRing;
-      if (lane == 0 && st >= kStRing &&
+      if (lane == 0 && st >= kStRing && !mbar_test(&emptyx[slot], ((st / kStRing) - 1) & 1) &&
           !mbar_wait_bounded(&emptyx[slot], ((st / kStRing) - 1) & 1)) {
         atomicOr(&g_shared_err, PA_DEVERR_PIPE_TIMEOUT);
         ok = false;
@@ -970,13 +973,15 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
       constexpr uint32_t kIdescS = umma_idesc_f16(0, 0, kStTokens, kSharedCols * NQ);
       bool ok = mbar_wait_bounded(qready, 0);
       // Polls the barriers and issues S(ns) as soon as its stage has landed and its
-      // S buffer is free (the P.V of stage ns - 2 is issued, so its softmax has read
-      // S(ns - 2)), and P.V(npv) as soon as P(npv) is written; sleeps otherwise.
+      // S buffer is free (every softmax warp has loaded S(ns - 2)), and P.V(npv) as
+      // soon as P(npv) is written; sleeps otherwise.
       int ns = 0, npv = 0, idle = 0;
       unsigned long long t_idle = 0;
       while (ok && npv < nstages) {
         bool prog = false;
-        if (ns < nstages && ns <= npv + 1 &&
+        // S(ns) goes into the buffer of S(ns - 2) as soon as every softmax warp has
+        // loaded that into its registers, not only once P.V(ns - 2) is issued
+        if (ns < nstages && (ns < 2 || mbar_test(&sread[ns & 1], ((ns - 2) >> 1) & 1)) &&
             mbar_test(&fullk[ns % kStRing], (ns / kStRing) & 1)) {
           tcgen05_fence_after();
           const uint64_t kd = kdesc + uint64_t(((ns % kStRing) * kStRawHalf) >> 4);
@@ -1028,8 +1033,9 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
     const int r = tid;                                       // 0..127
     const uint32_t tl = tmem + (uint32_t(32 * warp) << 16);  // this warp's lane quadrant
     bool ok = true;
+    // A phase that has completed is seen by a plain test, with no suspending try
     auto wait = [&](uint64_t* bar, uint32_t parity) {
-      if (ok) ok = __all_sync(kFullMask, mbar_wait_bounded(bar, parity));
+      if (ok) ok = __all_sync(kFullMask, mbar_test(bar, parity) || mbar_wait_bounded(bar, parity));
     };
     // ---- Q^T terms: thread t takes column n = t / 8, dims 16 (t % 8) .. + 15 ----
     {
@@ -1105,6 +1111,10 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
 #pragma unroll
         for (int t = 0; t < NQ; ++t) tmem_ld16(tl + kStTmemS + b * (16 * 3) + 16 * t, st_[t]);
         tmem_wait_ld();
+        // the S buffer is free for S(st + 2) once this warp's rows are in registers
+        tcgen05_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sread[b]);
 #pragma unroll
         for (int n = 0; n < kSharedCols; ++n) {
           float v = st_[NQ - 1][n];
