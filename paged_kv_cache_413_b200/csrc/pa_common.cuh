@@ -90,6 +90,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
 // Wait for the phase of the given parity to complete; false after ~1 s.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
   constexpr uint32_t kSuspendNs = PA_MBAR_SUSPEND_NS;  // per try; the loop bounds the total
+  {  // a phase that has completed is seen by a plain test, with no suspending try
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
   if (mbar_try_wait(bar, parity, kSuspendNs)) return true;
   const unsigned long long t0 = global_timer_ns();
   for (;;) {
