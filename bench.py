@@ -275,17 +275,28 @@ def cpu_baseline(wl: W.Workload, out_dtype: str, budget_s: float = 12.0):
     dt1, _ = oracle_sample(wl, order[:1], out_dtype)              # calibration
     k = int(max(1, min(n, budget_s / max(dt1, 1e-4))))
     dt, b = oracle_sample(wl, order[:k], out_dtype)
+    # the whole workload in well under the budget: time it repeatedly (the cache
+    # writes are idempotent) so that the figure rests on seconds of CPU work
+    reps = 1
+    if dt < 0.8 * budget_s:
+        more = min(1000, int((budget_s - dt) / max(dt, 1e-4)))
+        for _ in range(more):
+            dti, bi = oracle_sample(wl, order[:k], out_dtype)
+            dt += dti
+            b += bi
+        reps += more
     cores = oracle.num_threads()
     oracle.set_num_threads(1)
     try:
-        k1 = int(max(1, min(k, k * budget_s / max(dt * cores, 1e-4))))
+        k1 = int(max(1, min(k, k * reps * budget_s / max(dt * cores, 1e-4))))
         dt_1, b_1 = oracle_sample(wl, order[:k1], out_dtype)
     finally:
         oracle.set_num_threads(cores)
     return {"value": b / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"{k} of {n} sequences of the workload (cache write of their new "
-                      f"tokens + fp64 decode), {dt:.1f} s",
+                      f"tokens + fp64 decode)" + (f", {reps} times" if reps > 1 else "") +
+                      f", {dt:.1f} s",
             "single_thread": {"value": b_1 / dt_1 / 1e9, "unit": "GB/s", "cores": 1,
                               "sample": f"{k1} of the same sequences, {dt_1:.1f} s"}}
 
