@@ -45,6 +45,9 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(
     uint8_t* __restrict__ key_cache, uint8_t* __restrict__ value_cache,
     const int64_t* __restrict__ slot_mapping, int num_kv_heads, int head_dim, int block_size,
     int64_t num_slots, float k_scale, float v_scale) {
+  // the decode that reads these slots is a programmatic dependent: let its CTAs be
+  // scheduled now (it still waits for this grid to complete before reading)
+  grid_dependents_may_launch();
   const int64_t t = blockIdx.x;
   const int64_t slot = slot_mapping[t];
   if (slot < 0) return;  // padding token

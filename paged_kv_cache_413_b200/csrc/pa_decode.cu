@@ -286,6 +286,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   constexpr int SHIFT = NV == 32 ? 0 : 1;     // lanes per reduced value = 1 << SHIFT
   constexpr int NCH = kBlockSize / TC;        // chunks per block
   constexpr int GROUP_LANES = 32 / GT;        // lanes holding one head's scores
+  grid_dependency_wait();  // launched as a programmatic dependent
 
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr size_t tile_region = 2 * kStages * size_t(TILE);
@@ -508,7 +509,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
   __syncthreads();
   combine_and_store<D, GT>(cm, cl, cacc, cf, p, seq, part, head0, nparts);
   // let the merge kernel (launched as a programmatic dependent) get scheduled
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  grid_dependents_may_launch();
 }
 
 // ---------------------------------------------------------------------------
@@ -557,6 +558,7 @@ __global__ void __launch_bounds__(kThreads, GT == 8 ? PA_MMA8_MIN_CTAS : 4) deco
   static_assert(GT == 4 || GT == 8, "heads per CTA");
   static_assert(kStages % kConsumerWarps == 0, "each ring stage must belong to one warp");
   const Params& p = tp.p;
+  grid_dependency_wait();  // launched as a programmatic dependent
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -874,7 +876,7 @@ __global__ void __launch_bounds__(kThreads, GT == 8 ? PA_MMA8_MIN_CTAS : 4) deco
   __syncthreads();
   combine_and_store<D, GT>(cm, cl, cacc, cf, p, seq, part, head0, nparts);
   // let the merge kernel (launched as a programmatic dependent) get scheduled
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  grid_dependents_may_launch();
 }
 
 // Log-sum-exp merge of the partitions of sequences with more than one:
@@ -891,7 +893,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(
     void* out, const float* __restrict__ ws_m, const float* __restrict__ ws_l,
     const float* __restrict__ ws_o, const int32_t* __restrict__ seq_lens, int num_rows,
     int num_heads, int max_parts, int partition, int cap, int out_dtype) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  grid_dependency_wait();
   constexpr int DPL = D / 32;
   __shared__ float s_max[kReduceWarps];
   __shared__ float s_acc[kReduceWarps][D];
@@ -966,8 +968,8 @@ int launch_typed(const Params& p, int num_seqs, cudaStream_t stream) {
   if (set_smem_once(kern, smem, smem_set) != PA_OK) return PA_ERR_CUDA;
   const dim3 grid(unsigned(num_seqs) * unsigned(p.max_parts),
                   unsigned(p.num_kv_heads * p.head_groups));
-  kern<<<grid, kThreads, smem, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = launch_dependent(kern, grid, dim3(kThreads), smem, stream, p);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 template <int D, typename CT, typename QT>
@@ -1004,8 +1006,8 @@ int launch_mma_typed(const Params& p, const void* kc, const void* vc, int64_t ro
     return PA_ERR_CUDA;
   const dim3 grid(unsigned(num_seqs) * unsigned(p.max_parts),
                   unsigned(p.num_kv_heads * p.head_groups));
-  kern<<<grid, kThreads, smem, stream>>>(tp);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = launch_dependent(kern, grid, dim3(kThreads), smem, stream, tp);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 template <typename CT, typename QT>

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kThreads, PA_SHARED_MIN_CTAS) decode_shared_pr
   constexpr bool kSplitP = std::is_same<MT, __nv_bfloat16>::value;
   static_assert(kStages % kConsumerWarps == 0, "each ring stage must belong to one warp");
   const Params& p = sp.p;
+  grid_dependency_wait();  // launched as a programmatic dependent
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -716,6 +717,7 @@ __global__ void __launch_bounds__(kStThreads, 2) decode_shared_tc_kernel(
   constexpr int D = 128;
   constexpr int NQ = std::is_same<QT, __half>::value ? 3 : 2;  // terms of Q
   const Params& p = sp.p;
+  grid_dependency_wait();  // launched as a programmatic dependent
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* rawk = smem;                                 // [kStRing][8 K tiles]
@@ -1321,13 +1323,15 @@ int launch_shared_typed(const SharedParams& base, int grid_x, cudaStream_t strea
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = unsigned(base.cluster);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, base);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -1404,8 +1408,8 @@ int launch_decode_shared_prefix(const DecodeArgs& a, const int32_t* group_starts
       SharedParams tcp = sp;
       tcp.cluster = 1;
       if (set_smem_once(kern, smem, mask) != PA_OK) return PA_ERR_CUDA;
-      kern<<<grid, kStThreads, smem, stream>>>(tcp);
-      return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+      const cudaError_t e = launch_dependent(kern, grid, dim3(kStThreads), smem, stream, tcp);
+      return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
     };
     static std::atomic<unsigned long long> done_h{0}, done_b{0};
     static std::atomic<int> regs_h{0}, regs_b{0};
