@@ -4,13 +4,16 @@ The decode kernels are launched as programmatic dependents of the cache write
 before them: their CTAs may be scheduled while the write is still running, and
 each waits for it before touching global memory.  The split-K merge is in turn
 a dependent of the decode.  These tests run several steps on one stream with no
-host synchronisation.  Each step does three things:
+host synchronisation.  Each step does these things:
   1. sets the new tokens' slots to NaN again (a plain torch kernel);
-  2. writes that step's new K/V (different values every step);
-  3. decodes that step's queries into an output of its own.
+  2. (copy-on-write workloads) copies the diverging beams' blocks again;
+  3. writes that step's new K/V (different values every step);
+  4. decodes that step's queries into an output of its own.
 Consecutive decodes share one split-K workspace.  Two kinds of mistake would show:
   * a decode that read the pool before its step's write finished gives NaN or
     the wrong token;
+  * a write that ran before the copies finished is overwritten by them, which
+    also leaves the wrong token;
   * a decode whose partials overwrote a workspace the previous merge was still
     reading gives wrong outputs.
 Every step is checked against the oracle.  The same chain, captured in a CUDA
@@ -66,10 +69,13 @@ def _poisoner(wl, d):
 def _chain(wl, d, steps, outs, launch_decode):
     poison = _poisoner(wl, d)
     dev = [(s.new_key.cuda(), s.new_value.cuda(), s.query.cuda()) for s in steps]
+    copies = d.block_mapping if d.block_mapping is not None and d.block_mapping.numel() else None
 
     def run():
         for (nk, nv, q), out in zip(dev, outs):
             poison()
+            if copies is not None:
+                pa.pa_copy_blocks([d.key_cache], [d.value_cache], copies)
             pa.pa_reshape_and_cache(nk, nv, d.key_cache, d.value_cache, d.slot_mapping,
                                     k_scale=wl.k_scale, v_scale=wl.v_scale)
             launch_decode(q, out)
