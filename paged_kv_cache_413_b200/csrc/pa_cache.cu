@@ -38,7 +38,9 @@ __device__ __forceinline__ uint2 quantise8(uint4 x, float scale) {
                     uint32_t(q[2]) | (uint32_t(q[3]) << 16));
 }
 
-// One CTA per token; each thread moves 8 elements of K and 8 of V per step.
+// grid = (tokens, slices): the CTAs of a token split its row of 8-element chunks, so
+// that every thread moves one chunk of K and one of V (one DRAM round trip) when
+// the row has at most 128 x slices chunks.
 template <typename Tsrc, bool kQuant>
 __global__ void __launch_bounds__(128) reshape_and_cache_kernel(
     const uint16_t* __restrict__ key, const uint16_t* __restrict__ value,
@@ -52,13 +54,13 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(
   const int64_t slot = slot_mapping[t];
   if (slot < 0) return;  // padding token
   if (slot >= num_slots) {
-    if (threadIdx.x == 0) atomicOr(&g_cache_err, PA_DEVERR_SLOT_RANGE);
+    if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(&g_cache_err, PA_DEVERR_SLOT_RANGE);
     return;
   }
   const int64_t blk = slot / block_size, off = slot % block_size;
   const int row = num_kv_heads * head_dim;  // elements of one token
   const int chunks = row >> 3;
-  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+  for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < chunks; c += gridDim.y * blockDim.x) {
     const int e = c << 3;
     const int h = e / head_dim, d = e - h * head_dim;
     const int64_t src = t * row + e;
@@ -144,7 +146,10 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k
                                      int block_size, int64_t num_blocks, pa_dtype src_dtype,
                                      pa_dtype cache_dtype, float k_scale, float v_scale,
                                      cudaStream_t stream) {
-  const dim3 grid(num_tokens), block(128);
+  // up to 8 slices a token (a row of 8192 elements), one chunk a thread
+  const int chunks = (num_kv_heads * head_dim) >> 3;
+  const int slices = (chunks + 127) / 128 < 8 ? (chunks + 127) / 128 : 8;
+  const dim3 grid(unsigned(num_tokens), unsigned(slices > 0 ? slices : 1)), block(128);
   const int64_t num_slots = num_blocks * block_size;
   auto k = static_cast<const uint16_t*>(key);
   auto v = static_cast<const uint16_t*>(value);
