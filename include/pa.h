@@ -15,6 +15,12 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
  *     validates its host-visible arguments and enqueues work: it returns before
  *     the device has run it.  A return of PA_OK means "enqueued".
+ *   - Work on a stream runs in stream order.  The decode kernels are launched as
+ *     programmatic dependents (CUDA programmatic dependent launch).  Their CTAs
+ *     may be scheduled while the kernel before them on the stream is still
+ *     running, but they touch no memory until that kernel has completed and its
+ *     writes are visible.  The order a caller observes is that of ordinary
+ *     launches.
  *   - Tensors are dense, row-major (C order) with the shapes given below.
  *   - Data pointers must be 16-byte aligned (PA_ERR_INVALID_ARG otherwise).
  *   - Device data that the host cannot see (slots, block ids, sequence lengths) is
