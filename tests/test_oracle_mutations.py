@@ -3,13 +3,15 @@
 Each case plants one mistake in a copy of the oracle's C source (a dropped term,
 a wrong index, a transposed operand, a wrong rounding rule), builds it, and runs
 the oracle pin suites against that build in a child process.  The child must
-fail; a mutant that passes every pin would mean the pins do not pin.
+fail; a mutant that passes every pin would mean the pins do not pin.  The
+mutants build and run concurrently.
 """
 
 import os
 import subprocess
 import sys
 import tempfile
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -46,14 +48,26 @@ MUTANTS = {
                                "memcpy((char*)value_cache + dst_row * ec, (const char*)key + src_row * es,"),
     "bf16_shift": ("uint32_t u = (uint32_t)b << 16;", "uint32_t u = (uint32_t)b << 15;"),
     "merge_not_normalised": ("    for (int d = 0; d < head_dim; ++d) out[r * head_dim + d] /= W;\n", "\n"),
+    "decode_newest_token_dropped": (
+        "attend_rows(out + qrow, NULL, NULL, q, K, V, 0, L, head_dim, scale, sc);",
+        "attend_rows(out + qrow, NULL, NULL, q, K, V, 0, L - 1, head_dim, scale, sc);"),
+    "e4m3_saturates_to_nan": ("if (a >= 448.0) return (uint8_t)(sign | 0x7E);",
+                              "if (a >= 448.0) return (uint8_t)(sign | 0x7F);"),
+    "dequant_v_by_k_scale": ("        v *= v_scale;\n", "        v *= k_scale;\n"),
+    "quant_v_by_k_scale": ("float yv = xv / v_scale;", "float yv = xv / k_scale;"),
+    "f16_normal_bias": ("v = ldexp((double)(1024 + m), e - 25);", "v = ldexp((double)(1024 + m), e - 24);"),
+    "e4m3_subnormal_scale": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "partition_last_short": ("if (hi > L) hi = L;", "if (hi > L) hi = L - 1;"),
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name):
+def _run_mutant(name):
+    """Build the oracle with one planted mistake and run the pin suites on it in a
+    child process; returns (the child's exit status, the end of its output)."""
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    if src.count(old) != 1:
+        return None, f"mutation site for {name} not found exactly once"
     with tempfile.TemporaryDirectory() as tmp:
         csrc = os.path.join(tmp, "mutant.c")
         lib = os.path.join(tmp, "libmutant.so")
@@ -61,10 +75,25 @@ def test_pins_catch_mutant(name):
             f.write(src.replace(old, new))
         subprocess.run(["gcc", "-std=c11", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", lib,
                         csrc, "-lm"], check=True)
-        env = dict(os.environ, PA_ORACLE_LIB_OVERRIDE=lib)
+        env = dict(os.environ, PA_ORACLE_LIB_OVERRIDE=lib, OMP_NUM_THREADS="2")
         r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                             os.path.join(ROOT, "tests", "test_oracle_formats.py"),
                             os.path.join(ROOT, "tests", "test_oracle_cache_ops.py"),
                             os.path.join(ROOT, "tests", "test_oracle_decode.py")],
-                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-        assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
+                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+        return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def outcomes():
+    """Every mutant's outcome; the mutants build and run concurrently."""
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        return dict(zip(MUTANTS, ex.map(_run_mutant, MUTANTS)))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, outcomes):
+    rc, out = outcomes[name]
+    assert rc is not None, out
+    assert rc != 0, f"mutant {name} passed every pin:\n{out}"
