@@ -24,7 +24,9 @@ def _pool(nb, hkv, d, dtype, fill_seed=0):
 
 @pytest.mark.parametrize("src,cache", [("f16", "f16"), ("bf16", "bf16"), ("f16", "e4m3"),
                                        ("bf16", "e4m3")])
-@pytest.mark.parametrize("hkv,d", [(4, 64), (8, 128), (3, 40)])
+# rows of 8-element chunks: 32, 128, 15 (one CTA a token); 512 (4 CTAs, the 7B row);
+# 2048 (8 CTAs of two chunks a thread); 225 (2 CTAs, the second partly idle)
+@pytest.mark.parametrize("hkv,d", [(4, 64), (8, 128), (3, 40), (32, 128), (128, 128), (9, 200)])
 def test_reshape_and_cache_bit_exact(src, cache, hkv, d):
     nb, t = 37, 300
     rng = np.random.default_rng(hkv * 1000 + d)
