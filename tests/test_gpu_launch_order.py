@@ -188,3 +188,38 @@ def test_chain_in_a_cuda_graph(shared):
     for k, (a, b) in enumerate(zip(eager, replayed)):
         assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), f"step {k} differs"
     del g
+
+
+@pytest.mark.parametrize("name,over,part,shared", [
+    ("llama2_7b", dict(num_seqs=6), 256, False),
+    ("llama2_70b_gqa", dict(num_seqs=10), 0, False),
+    ("beam_cow_fp8", dict(num_seqs=3, shared_len=72), 0, True),
+])
+def test_query_written_by_the_kernel_just_before(name, over, part, shared):
+    """One query buffer for every step, filled by a torch elementwise kernel right
+    before each decode: a decode that read it early would see the previous step's
+    queries."""
+    wl = W.make_workload(name, **over)
+    d = flow.to_device(wl)
+    flow.gpu_prepare(wl, d)
+    pa.pa_reshape_and_cache(d.new_key, d.new_value, d.key_cache, d.value_cache, d.slot_mapping,
+                            k_scale=wl.k_scale, v_scale=wl.v_scale)
+    steps = _step_inputs(wl, STEPS, seed=77)
+    out_dtype = "f32"
+    outs = _outputs(wl, out_dtype, STEPS)
+    launch = _shared_launcher(wl, d) if shared else \
+        _decode_launcher(wl, d, part, flow.workspace_for(wl, part))
+    qs = [s.query.cuda() for s in steps]
+    qbuf = torch.empty_like(qs[0])
+    torch.cuda.synchronize()
+    for q, out in zip(qs, outs):
+        torch.mul(q, 1, out=qbuf)  # an elementwise kernel, not a copy
+        launch(qbuf, out)
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error() == 0
+    # the pool holds the workload's own new tokens; only the queries change
+    kc, vc = flow.oracle_caches(wl)
+    for k, (s, out) in enumerate(zip(steps, outs)):
+        ref = flow.oracle_decode(dataclasses.replace(wl, query=s.query), kc, vc)
+        err = flow.max_abs_err(out, ref)
+        assert err <= flow.TOL[out_dtype], f"step {k}: max abs error {err:.3e}"
