@@ -58,6 +58,23 @@ MUTANTS = {
     "f16_normal_bias": ("v = ldexp((double)(1024 + m), e - 25);", "v = ldexp((double)(1024 + m), e - 24);"),
     "e4m3_subnormal_scale": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
     "partition_last_short": ("if (hi > L) hi = L;", "if (hi > L) hi = L - 1;"),
+    "copy_value_skipped": ("      memcpy((char*)value_caches[l] + dst * block_bytes,\n"
+                           "             (char*)value_caches[l] + src * block_bytes, (size_t)block_bytes);\n",
+                           ""),
+    "copy_first_layer_only": ("    for (int l = 0; l < num_layers; ++l) {\n      memcpy((char*)key_caches[l]",
+                              "    for (int l = 0; l < 1; ++l) {\n      memcpy((char*)key_caches[l]"),
+    "swap_value_from_key": ("(const char*)src_value_caches[l] + src * block_bytes",
+                            "(const char*)src_key_caches[l] + src * block_bytes"),
+    "gather_kv_head_ignored": (
+        "int64_t row = ((phys * num_kv_heads + kvh) * block_size + off) * (int64_t)head_dim;",
+        "int64_t row = ((phys * num_kv_heads) * block_size + off) * (int64_t)head_dim;"),
+    "reshape_token_major": (
+        "int64_t dst_row = ((b * num_kv_heads + h) * block_size + o) * (int64_t)head_dim;",
+        "int64_t dst_row = ((b * block_size + o) * num_kv_heads + h) * (int64_t)head_dim;"),
+    "prefill_query_start_ignored": ("int64_t row = ((int64_t)(q0 + j) * num_heads + h) * head_dim;",
+                                    "int64_t row = ((int64_t)j * num_heads + h) * head_dim;"),
+    "partition_sum_lost": ("if (l_out) *l_out = sum;", "if (l_out) *l_out = 1.0;"),
+    "e4m3_nan_saturates": ("if (isnan(y)) return 0x7F;", "if (isnan(y)) return 0x7E;"),
 }
 
 
