@@ -259,8 +259,9 @@ int pa_copy_blocks(void* const* key_caches, void* const* value_caches, int num_l
 
 /*
  * pa_paged_attention_decode_static_workspace -- pa_paged_attention_decode for
- * callers that cannot allocate device memory.  The pages have no counterpart to
- * this entry point; it exists for the library's users.
+ * callers that cannot allocate device memory.  It computes the same decode
+ * ("vLLM 推理优化技术深度调研报告" sec 3 formulas 3 and 4); the pages have no
+ * counterpart to the fixed scratch, which exists for the library's users.
  *
  * Who needs it: a plugin inside a host process that owns every device allocation
  * and gives its plugins no allocator; a serving engine that has already reserved

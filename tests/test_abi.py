@@ -39,6 +39,30 @@ def test_every_declared_symbol_is_exported(lib):
         assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
 
 
+# the entry points that compute something the pages define; the rest are host
+# helpers (sizes, status strings, the device error word)
+COMPUTE_ENTRY_POINTS = ["pa_reshape_and_cache", "pa_paged_attention_decode",
+                        "pa_paged_attention_decode_shared_prefix", "pa_paged_attention_prefill",
+                        "pa_copy_blocks", "pa_swap_blocks",
+                        "pa_paged_attention_decode_static_workspace"]
+PAGES = ("vLLM 推理优化技术深度调研报告", "vLLM推理引擎PagedAttention原理与性能优化实战",
+         "vLLM 是什么")
+
+
+def test_every_compute_entry_point_cites_the_pages():
+    """The comment block before each compute entry point names the page (by its
+    title) and the section that defines the operation."""
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    for name in COMPUTE_ENTRY_POINTS:
+        m = re.search(r"/\*((?:(?!\*/).)*)\*/\s*int\s+" + name + r"\s*\(", src, re.S)
+        assert m, f"{name}: no comment block before its declaration"
+        com = m.group(1)
+        joined = re.sub(r"\s*\n\s*\*\s*", "", com)  # a title may wrap over lines
+        assert any(p in joined or p.replace(" ", "") in joined for p in PAGES), \
+            f"{name}: cites no page"
+        assert re.search(r"\bsec\b|§", com), f"{name}: cites no section"
+
+
 def test_status_strings(lib):
     assert pa.pa_status_string(0) == "PA_OK"
     assert pa.pa_status_string(-3) == "PA_ERR_WORKSPACE"
